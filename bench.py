@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the fused GDN decode step (gdn_decode_step) on the batch64 workload:
+B=64 sequences x 1 token, Hk=16 k-heads, Hv=32 v-heads, dk=dv=128, conv width 4,
+a 64-slot FP32 state pool (128 MiB) with seeded slot permutation.
+
+A step is one launch of the whole path (conv update, gate, gated delta rule, gated
+RMSNorm) over one batch. Four independent state pools (layers) are cycled, so the
+512 MiB working set exceeds L2 and every step reads its state from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+N > 1 runs under torchrun, one rank per GPU; each rank owns its own sequences and
+pools (sequences are independent: no collective on the data path), so per-GPU work
+is fixed as N grows. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s) at B=64"
+UNIT = "tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_NAME = "decode_fused_kernel"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=("b200", "reference"), default="b200")
+    ap.add_argument("--workload", default="batch64")
+    ap.add_argument("--pools", type=int, default=4, help="independent state pools cycled (layers)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(wl) -> int:
+    """Bytes one launch must move: per sequence the state read+write, the conv
+    history read+write, qkv, a, b, z in, out, the slot; per launch the weights."""
+    Hk, Hv, dk, dv, W, T, C = (wl.num_k_heads, wl.num_v_heads, wl.head_k_dim, wl.head_v_dim, wl.conv_width,
+                               wl.tokens, wl.channels)
+    per_seq = (2 * Hv * dk * dv * 4 + 2 * (W - 1) * C * 2 + T * C * 2 + 2 * T * Hv * 2 + T * Hv * dv * 2 +
+               T * Hv * dv * 2 + 4)
+    per_launch = C * W * 2 + 2 * Hv * 4 + dv * 2
+    return wl.batch * per_seq + per_launch
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_102_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(wl_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{KERNEL_NAME}_{wl_name}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
+    m_bytes = re.search(r"dram bytes per launch:\s*`?([0-9]+)", txt)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples, timestamped on arrival."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.samples = []
+        ident = str(device_index)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", ident], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        win = [p for (t, p) in self.samples if t0 <= t <= t1]
+        used = win if win else [p for (_, p) in self.samples]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in used if num(p[0]) is not None]
+        mx = [num(p[1]) for p in used if num(p[1]) is not None]
+        reasons = sorted({r for p in used for r, v in zip(self.REASONS, p[3:]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(win)}
+
+
+def cpu_baseline(wl, budget_s: float):
+    """The FP64 oracle, single-threaded, on whole steps of the same batch until the
+    time budget is spent."""
+    import numpy as np
+    import oracle
+    from gated_delta_rule_102_b200 import synth
+    sh = oracle.Shape.of(wl)
+    w = synth.weights(wl)
+    st = synth.initial_state(wl).astype(np.float64)
+    cv = synth.initial_conv_state(wl)
+    slots = synth.slots(wl)
+    steps, elapsed = 0, 0.0
+    while elapsed < budget_s:
+        x = synth.step_inputs(wl, steps)  # input generation is not timed
+        t = time.perf_counter()
+        oracle.decode_step(sh, x["qkv"], x["a"], x["b"], x["z"], w["conv_w"], w["A_log"], w["dt_bias"], w["norm_w"],
+                           cv, st, slots)
+        elapsed += time.perf_counter() - t
+        steps += 1
+    return {"value": wl.batch * wl.tokens * steps / elapsed, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{steps} full steps of {wl.name} ({wl.batch} sequences x {wl.tokens} token), "
+                      f"single-threaded FP64 C oracle, {elapsed:.1f} s"}
+
+
+def run_reference(args, wl, rank: int, world: int):
+    """The oracle as the reference arm: each step is one sequence-token of the
+    workload on the host cores."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from gated_delta_rule_102_b200 import synth
+    sh = oracle.Shape.of(wl)
+    w = synth.weights(wl)
+    slots = synth.slots(wl)
+    st = synth.initial_state(wl).astype(np.float64)
+    cv = synth.initial_conv_state(wl)
+    inputs = [synth.step_inputs(wl, s) for s in range(4)]  # generated before timing, cycled
+
+    def one(i):
+        launch, row = divmod(i, wl.batch)
+        x = inputs[launch % len(inputs)]
+        r = slice(row, row + 1)
+        oracle.decode_step(sh, x["qkv"][r], x["a"][r], x["b"][r], x["z"][r], w["conv_w"], w["A_log"],
+                           w["dt_bias"], w["norm_w"], cv, st, slots[r])
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        one(i)
+    el = time.perf_counter() - t0
+    value = args.steps * wl.tokens / el
+    sample = f"one sequence-token of {wl.name} per step, single-threaded FP64 C oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded SplitMix64 draws)", "config": workload_config(wl, args, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, args, world):
+    return {"workload": f"{wl.name}: B={wl.batch} sequences x T={wl.tokens} token, Hk={wl.num_k_heads}, "
+                        f"Hv={wl.num_v_heads}, dk={wl.head_k_dim}, dv={wl.head_v_dim}, conv width {wl.conv_width}, "
+                        f"{wl.pool_slots}-slot fp32 state pool per layer",
+            "batch_per_gpu": wl.batch, "tokens_per_sequence": wl.tokens, "state_pools_cycled": args.pools,
+            "l2": f"inputs larger than L2: {args.pools} state pools x "
+                  f"{wl.pool_slots * wl.num_v_heads * wl.head_k_dim * wl.head_v_dim * 4 >> 20} MiB cycled",
+            "parallelism": f"dp{world} (independent sequence shards, no collective)"}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        sys.exit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    from gated_delta_rule_102_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_102_b200 as gdn
+    from gated_delta_rule_102_b200 import build as gdn_build
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        gdn_build.build()
+    if world > 1:
+        dist.barrier()
+    gdn.lib()
+    wlr = wl.replace(seed=wl.seed + 7919 * rank)  # each rank owns different sequences
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    cfg = gdn.GdnConfig.make(wl.num_k_heads, wl.num_v_heads, wl.head_k_dim, wl.head_v_dim, wl.conv_width)
+    w = synth.weights(wlr)
+    conv_w, norm_w = bf16(w["conv_w"]), bf16(w["norm_w"])
+    A_log, dt_bias = torch.from_numpy(w["A_log"]).to(dev), torch.from_numpy(w["dt_bias"]).to(dev)
+    slots = torch.from_numpy(synth.slots(wlr)).to(dev)
+    states = [torch.from_numpy(synth.initial_state(wlr.replace(seed=wlr.seed + 101 * p))).to(dev)
+              for p in range(args.pools)]
+    convs = [bf16(synth.initial_conv_state(wlr)) for _ in range(args.pools)]
+    n_inputs = args.pools * 4
+    xs = [{k: bf16(v) for k, v in synth.step_inputs(wlr, s).items()} for s in range(n_inputs)]
+    out = torch.empty(wl.batch, wl.tokens, wl.num_v_heads, wl.head_v_dim, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    plans = [gdn.DecodePlan(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
+                            convs[i % args.pools], states[i % args.pools], slots, out, None, err, stream)
+             for i, x in enumerate(xs)]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    for i in range(args.warmup):
+        plans[i % n_inputs].launch()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps, events around each launch on the launching stream
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(K):
+        ev_s[i].record(stream)
+        plans[i % n_inputs].launch()
+        ev_e[i].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end))
+    kernel_ms = statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(K))
+    kernel_ms = max_over_ranks(kernel_ms)
+    if int(err.item()) != 0:
+        raise RuntimeError("device reported an out-of-range slot")
+
+    # ---- end to end through the C ABI: pinned host inputs in, host output back, every step
+    e2e = None
+    if not args.no_e2e:
+        hx = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in xs]
+        dx = {k: torch.empty_like(v) for k, v in xs[0].items()}
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        eplans = [gdn.DecodePlan(cfg, dx["qkv"], dx["a"], dx["b"], dx["z"], conv_w, A_log, dt_bias, norm_w,
+                                 convs[p], states[p], slots, out, None, err, stream) for p in range(args.pools)]
+        h2d = sum(v.numel() * v.element_size() for v in hx[0].values())
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step(i):
+            for k in dx:
+                dx[k].copy_(hx[i % n_inputs][k], non_blocking=True)
+            eplans[i % args.pools].launch()
+            hout.copy_(out, non_blocking=True)
+
+        for i in range(args.warmup):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * wl.batch * wl.tokens * K / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    clocks = None
+    if sampler is not None:
+        sampler.stop()
+        clocks = sampler.summary(t_wall0, t_wall1)
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    nbytes = algorithmic_bytes(wl)
+    peak, peak_kind = hbm_peak()
+    achieved = nbytes / (kernel_ms / 1e3) / 1e9
+    tokens = world * wl.batch * wl.tokens * K
+    value = tokens / (elapsed_ms / 1e3)
+    job_gbs = world * nbytes * K / (elapsed_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded SplitMix64 draws; bf16 inputs, fp32 state)",
+        "config": workload_config(wl, args, world),
+        "hbm_gbs": job_gbs / world, "frac_of_8tbs": job_gbs / world / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic(wl.name), "peak_source": f"{peak_kind} copy bandwidth",
+                     "kernel": KERNEL_NAME, "kernel_us": kernel_ms * 1e3, "algorithmic_bytes": nbytes},
+        "e2e": e2e, "clocks": clocks, "gpu_launches": K,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+"""ctypes binding of libgdn (include/gdn.h): the same entry points, argument
+marshalling only. Tensors are torch CUDA tensors (bf16 arguments as
+torch.bfloat16, whose storage is the bf16 bit pattern); the call goes to the
+caller's current CUDA stream unless ``stream`` is given.
+
+There is no fallback: if libgdn.so is missing or cannot be loaded, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARGUMENT = 1
+GDN_ERR_UNSUPPORTED = 2
+GDN_ERR_MISALIGNED = 3
+GDN_ERR_SLOT_RANGE = 4
+GDN_ERR_CUDA = 5
+GDN_DEVICE_ERR_SLOT_RANGE = 1
+
+EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
+           "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
+
+
+class GdnConfig(ctypes.Structure):
+    """Mirror of ``gdn_config``."""
+    _fields_ = [("num_k_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
+                ("head_k_dim", ctypes.c_int32), ("head_v_dim", ctypes.c_int32),
+                ("conv_width", ctypes.c_int32), ("l2_eps", ctypes.c_float),
+                ("rms_eps", ctypes.c_float), ("q_scale", ctypes.c_float)]
+
+    @classmethod
+    def make(cls, num_k_heads, num_v_heads, head_k_dim, head_v_dim, conv_width,
+             l2_eps=1e-6, rms_eps=1e-6, q_scale=0.0) -> "GdnConfig":
+        return cls(num_k_heads, num_v_heads, head_k_dim, head_v_dim, conv_width, l2_eps, rms_eps, q_scale)
+
+    @property
+    def channels(self) -> int:
+        return 2 * self.num_k_heads * self.head_k_dim + self.num_v_heads * self.head_v_dim
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdn with argument types declared (raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libgdn.so not built at {LIB_PATH}; run python -m gated_delta_rule_102_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32 = ctypes.c_void_p, ctypes.c_int32
+        cfgp = ctypes.POINTER(GdnConfig)
+        L.gdn_conv_update.argtypes = [cfgp, i32, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_recurrent_step.argtypes = [cfgp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+        L.gdn_gated_rmsnorm.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_decode_step.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp]
+        L.gdn_check_slots_host.argtypes = [vp, i32, i32]
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_abi_version.argtypes = []
+        for f in ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
+                  "gdn_check_slots_host", "gdn_abi_version"):
+            getattr(L, f).restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != GDN_OK:
+        raise GdnError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor], dtypes, name: str):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+_F32 = (torch.float32,)
+_I32 = (torch.int32,)
+
+
+def _stream(stream, ref: torch.Tensor):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(ref.device).cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def gdn_conv_update(cfg: GdnConfig, qkv, conv_w, conv_pool, slots, q_out, k_out, v_out,
+                    err_flag=None, stream=None) -> None:
+    B, T = qkv.shape[0], qkv.shape[1]
+    _check(lib().gdn_conv_update(ctypes.byref(cfg), B, T, _ptr(qkv, _BF16, "qkv"), _ptr(conv_w, _BF16, "conv_w"),
+                                 _ptr(conv_pool, _BF16, "conv_pool"), conv_pool.shape[0],
+                                 _ptr(slots, _I32, "slots"), _ptr(q_out, _F32, "q_out"),
+                                 _ptr(k_out, _F32, "k_out"), _ptr(v_out, _F32, "v_out"),
+                                 _ptr(err_flag, _I32, "err_flag"), _stream(stream, qkv)), "gdn_conv_update")
+
+
+def gdn_recurrent_step(cfg: GdnConfig, q, k, v, a, b, A_log, dt_bias, state_pool, slots, o,
+                       err_flag=None, stream=None) -> None:
+    B, T = q.shape[0], q.shape[1]
+    _check(lib().gdn_recurrent_step(ctypes.byref(cfg), B, T, _ptr(q, _F32, "q"), _ptr(k, _F32, "k"),
+                                    _ptr(v, _F32, "v"), _ptr(a, _BF16, "a"), _ptr(b, _BF16, "b"),
+                                    _ptr(A_log, _F32, "A_log"), _ptr(dt_bias, _F32, "dt_bias"),
+                                    _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0],
+                                    _ptr(slots, _I32, "slots"), _ptr(o, _F32, "o"),
+                                    _ptr(err_flag, _I32, "err_flag"), _stream(stream, q)), "gdn_recurrent_step")
+
+
+def gdn_gated_rmsnorm(cfg: GdnConfig, o, z, norm_w, out, out_f32=None, stream=None) -> None:
+    rows = o.numel() // cfg.head_v_dim
+    _check(lib().gdn_gated_rmsnorm(ctypes.byref(cfg), rows, _ptr(o, _F32, "o"), _ptr(z, _BF16, "z"),
+                                   _ptr(norm_w, _BF16, "norm_w"), _ptr(out, _BF16, "out"),
+                                   _ptr(out_f32, _F32, "out_f32"), _stream(stream, o)), "gdn_gated_rmsnorm")
+
+
+def gdn_decode_step(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
+                    slots, out, out_f32=None, err_flag=None, stream=None) -> None:
+    B, T = qkv.shape[0], qkv.shape[1]
+    _check(lib().gdn_decode_step(ctypes.byref(cfg), B, T, _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"),
+                                 _ptr(b, _BF16, "b"), _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"),
+                                 _ptr(A_log, _F32, "A_log"), _ptr(dt_bias, _F32, "dt_bias"),
+                                 _ptr(norm_w, _BF16, "norm_w"), _ptr(conv_pool, _BF16, "conv_pool"),
+                                 _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0],
+                                 _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
+                                 _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
+                                 _stream(stream, qkv)), "gdn_decode_step")
+
+
+def gdn_check_slots_host(slots, pool_slots: int) -> int:
+    """Status of the host-side slot check on a CPU int32 array-like."""
+    import numpy as np
+    s = np.ascontiguousarray(np.asarray(slots, dtype=np.int32))
+    return int(lib().gdn_check_slots_host(s.ctypes.data_as(ctypes.c_void_p), s.size, int(pool_slots)))
+
+
+def abi_version() -> int:
+    return int(lib().gdn_abi_version())
+
+
+class DecodePlan:
+    """gdn_decode_step with its arguments marshalled once: ``launch()`` makes the
+    same C call with the stored pointers, for loops that replay one set of tensors
+    (the tensors must stay alive and in place while the plan is used)."""
+
+    def __init__(self, cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
+                 slots, out, out_f32=None, err_flag=None, stream=None):
+        self._keep = (cfg, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots, out,
+                      out_f32, err_flag)
+        self._fn = lib().gdn_decode_step
+        self._args = (ctypes.byref(cfg), qkv.shape[0], qkv.shape[1], _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"),
+                      _ptr(b, _BF16, "b"), _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"),
+                      _ptr(A_log, _F32, "A_log"), _ptr(dt_bias, _F32, "dt_bias"), _ptr(norm_w, _BF16, "norm_w"),
+                      _ptr(conv_pool, _BF16, "conv_pool"), _ptr(state_pool, _F32, "state_pool"),
+                      state_pool.shape[0], _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
+                      _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"), _stream(stream, qkv))
+
+    def launch(self) -> None:
+        st = self._fn(*self._args)
+        if st != GDN_OK:
+            raise GdnError(st, "gdn_decode_step")

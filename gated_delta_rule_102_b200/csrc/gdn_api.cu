@@ -1,0 +1,160 @@
+// C-ABI entry points of libgdn (declared in include/gdn.h). Every argument is checked
+// here, on the host, before anything is enqueued, so an error return means nothing
+// was written; then one launch per entry point goes onto the caller's stream.
+// Following the "fail before the first launch" convention of the Metrale layer page
+// ("metrale_model_arch/glm5next_dsa/layer.rs", its invariants paragraph).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/gdn.h"
+#include "gdn_device.cuh"
+#include "gdn_internal.h"
+
+namespace {
+
+bool supported_head_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+gdn_status check_config(const gdn_config* cfg, gdn::Shape* sh) {
+    if (!cfg) return GDN_ERR_INVALID_ARGUMENT;
+    if (cfg->num_k_heads <= 0 || cfg->num_v_heads <= 0 || cfg->head_k_dim <= 0 || cfg->head_v_dim <= 0 ||
+        cfg->conv_width <= 0)
+        return GDN_ERR_INVALID_ARGUMENT;
+    if (cfg->num_v_heads % cfg->num_k_heads != 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (!(cfg->l2_eps >= 0.0f) || !(cfg->rms_eps >= 0.0f) || !isfinite(cfg->l2_eps) || !isfinite(cfg->rms_eps) ||
+        !isfinite(cfg->q_scale))
+        return GDN_ERR_INVALID_ARGUMENT;
+    if (cfg->num_v_heads / cfg->num_k_heads > 8) return GDN_ERR_UNSUPPORTED;
+    if (!supported_head_dim(cfg->head_k_dim) || !supported_head_dim(cfg->head_v_dim)) return GDN_ERR_UNSUPPORTED;
+    if (cfg->conv_width < 2 || cfg->conv_width > gdn::kMaxConvWidth) return GDN_ERR_UNSUPPORTED;
+    const long C = 2L * cfg->num_k_heads * cfg->head_k_dim + (long)cfg->num_v_heads * cfg->head_v_dim;
+    if (C > (1L << 30)) return GDN_ERR_UNSUPPORTED;
+    sh->Hk = cfg->num_k_heads;
+    sh->Hv = cfg->num_v_heads;
+    sh->dk = cfg->head_k_dim;
+    sh->dv = cfg->head_v_dim;
+    sh->W = cfg->conv_width;
+    sh->C = (int)C;
+    sh->l2_eps = cfg->l2_eps;
+    sh->rms_eps = cfg->rms_eps;
+    sh->q_scale = cfg->q_scale != 0.0f ? cfg->q_scale : 1.0f / sqrtf((float)cfg->head_k_dim);
+    return GDN_OK;
+}
+
+gdn_status check_batch(int32_t B, int32_t T, int32_t pool_slots, const gdn::Shape& sh) {
+    if (B < 0 || T <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (T > gdn::kMaxTokens) return GDN_ERR_UNSUPPORTED;
+    if (B > 0 && pool_slots <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    // grid: B * Hv * (at most 8 slices) CTAs
+    if ((long)B * sh.Hv * 8 > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+// All pointers non-null and 16-byte aligned (nullable ones checked only when set).
+gdn_status check_pointers(std::initializer_list<const void*> required, std::initializer_list<const void*> nullable) {
+    for (const void* p : required)
+        if (!p) return GDN_ERR_INVALID_ARGUMENT;
+    for (const void* p : required)
+        if (!aligned16(p)) return GDN_ERR_MISALIGNED;
+    for (const void* p : nullable)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    return GDN_OK;
+}
+
+gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_conv_update(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv, const uint16_t* conv_w,
+                           uint16_t* conv_pool, int32_t pool_slots, const int32_t* slots, float* q_out, float* k_out,
+                           float* v_out, int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((st = check_pointers({qkv, conv_w, conv_pool, slots, q_out, k_out, v_out}, {err_flag})) != GDN_OK) return st;
+    gdn::ConvArgs a{sh, B, T, pool_slots, qkv, conv_w, conv_pool, slots, q_out, k_out, v_out, err_flag};
+    return from_cuda(gdn::launch_conv_update(a, (cudaStream_t)stream));
+}
+
+gdn_status gdn_recurrent_step(const gdn_config* cfg, int32_t B, int32_t T, const float* q, const float* k,
+                              const float* v, const uint16_t* a, const uint16_t* b, const float* A_log,
+                              const float* dt_bias, float* state_pool, int32_t pool_slots, const int32_t* slots,
+                              float* o, int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((st = check_pointers({q, k, v, a, b, A_log, dt_bias, state_pool, slots, o}, {err_flag})) != GDN_OK)
+        return st;
+    gdn::RecurrentArgs r{sh, B, T, pool_slots, gdn::recurrent_column_splits(B, sh.Hv, sh.dv),
+                         q, k, v, a, b, A_log, dt_bias, state_pool, slots, o, err_flag};
+    return from_cuda(gdn::launch_recurrent(r, (cudaStream_t)stream));
+}
+
+gdn_status gdn_gated_rmsnorm(const gdn_config* cfg, int32_t rows, const float* o, const uint16_t* z,
+                             const uint16_t* norm_w, uint16_t* out_bf16, float* out_f32, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if (rows < 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (rows == 0) return GDN_OK;
+    if ((st = check_pointers({o, z, norm_w, out_bf16}, {out_f32})) != GDN_OK) return st;
+    gdn::NormArgs n{sh, rows, o, z, norm_w, out_bf16, out_f32};
+    return from_cuda(gdn::launch_gated_rmsnorm(n, (cudaStream_t)stream));
+}
+
+gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv, const uint16_t* a,
+                           const uint16_t* b, const uint16_t* z, const uint16_t* conv_w, const float* A_log,
+                           const float* dt_bias, const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                           int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16, float* out_f32,
+                           int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((st = check_pointers({qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots, out_bf16},
+                             {out_f32, err_flag})) != GDN_OK)
+        return st;
+    const int G = sh.Hv / sh.Hk;
+    gdn::DecodeArgs d{sh, B, T, pool_slots, gdn::decode_column_splits(B, sh.Hv, G, sh.dv),
+                      qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots,
+                      out_bf16, out_f32, err_flag};
+    return from_cuda(gdn::launch_decode_fused(d, (cudaStream_t)stream));
+}
+
+gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t pool_slots) {
+    if (B < 0 || pool_slots < 0 || (B > 0 && !slots_host)) return GDN_ERR_INVALID_ARGUMENT;
+    std::vector<unsigned char> seen((size_t)pool_slots, 0);
+    for (int32_t i = 0; i < B; ++i) {
+        const int32_t s = slots_host[i];
+        if (s < 0 || s >= pool_slots || seen[(size_t)s]) return GDN_ERR_SLOT_RANGE;
+        seen[(size_t)s] = 1;
+    }
+    return GDN_OK;
+}
+
+const char* gdn_status_string(gdn_status status) {
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported shape";
+        case GDN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case GDN_ERR_SLOT_RANGE: return "slot out of range or repeated";
+        case GDN_ERR_CUDA: return "CUDA launch failed";
+    }
+    return "unknown status";
+}
+
+int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+}  // extern "C"

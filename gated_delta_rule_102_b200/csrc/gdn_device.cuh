@@ -1,0 +1,230 @@
+// Device building blocks of the GDN decode step for sm_100a: bf16 handling, the
+// per-channel causal conv with its history roll, the gate, the cluster barrier and
+// the register-resident delta-rule pass over one state tile.
+//
+// Method: the page "spark_model/forward/qwen3_5/linear_attention.rs" (Atlas),
+// steps 3 (conv + SiLU + q/k L2 norm), 4 (gate), 5 (beta), 7 (gated delta rule)
+// and 8 (per-head RMSNorm) with the SiLU(z) gate of steps 9+10+11.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Longest conv supported (taps) and most tokens per launch.
+constexpr int kMaxConvWidth = 8;
+constexpr int kMaxTokens = 16;
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits) { return __uint_as_float(bits << 16); }
+
+// float -> bf16 bits, round to nearest even (finite inputs; NaN kept quiet).
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+__device__ __forceinline__ float sigmoid(float x) { return 1.0f / (1.0f + expf(-x)); }
+// log(1 + e^x) without overflow: max(x, 0) + log1p(e^-|x|).
+__device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x))); }
+
+// Step 4 and 5: decay alpha = exp(-exp(A_log) * softplus(a + dt_bias)), beta = sigmoid(b).
+__device__ __forceinline__ void gate_and_beta(uint16_t a_bits, uint16_t b_bits, float A_log, float dt_bias,
+                                              float& alpha, float& beta) {
+    const float g = -expf(A_log) * softplus(bf16_bits_to_float(a_bits) + dt_bias);
+    alpha = expf(g);
+    beta = sigmoid(bf16_bits_to_float(b_bits));
+}
+
+// ---------------------------------------------------------------------------------
+// Step 3 for one channel: a depthwise causal conv of width W over the slot's W-1
+// stored raw inputs followed by this launch's T raw inputs, SiLU on the result.
+// The window lives in registers with the newest input at the highest index, so
+// every register index is a compile-time constant whatever W is. After the T tokens
+// the last W-1 raw inputs are written back as the slot's history, bit for bit.
+//   hist : &conv_pool[slot][0][ch], row stride C
+//   x    : &qkv[seq][0][ch],        token stride C
+//   w    : &conv_w[ch][0]
+//   emit(t, s) receives SiLU(conv) of token t.
+template <typename Emit>
+__device__ __forceinline__ void conv_channel(uint16_t* hist, const uint16_t* x, const uint16_t* w,
+                                             int W, int T, size_t C, Emit emit) {
+    uint32_t win[kMaxConvWidth];
+    float wt[kMaxConvWidth];
+#pragma unroll
+    for (int m = 0; m < kMaxConvWidth; ++m) {
+        const int e = kMaxConvWidth - 1 - m;  // tokens before the newest history row
+        const int r = W - 2 - e;              // history row held at win[m]
+        win[m] = r >= 0 ? (uint32_t)hist[(size_t)r * C] : 0u;
+    }
+    // After the shift at token t, win[kMax-1-d] holds the input d tokens back, which
+    // conv tap W-1-d multiplies.
+#pragma unroll
+    for (int m = 0; m < kMaxConvWidth; ++m) {
+        const int d = kMaxConvWidth - 1 - m;
+        wt[m] = d < W ? bf16_bits_to_float(w[W - 1 - d]) : 0.0f;
+    }
+    for (int t = 0; t < T; ++t) {
+#pragma unroll
+        for (int m = 0; m < kMaxConvWidth - 1; ++m) win[m] = win[m + 1];
+        win[kMaxConvWidth - 1] = x[(size_t)t * C];
+        float u = 0.0f;
+#pragma unroll
+        for (int m = 0; m < kMaxConvWidth; ++m) u = fmaf(wt[m], bf16_bits_to_float(win[m]), u);
+        emit(t, silu(u));
+    }
+#pragma unroll
+    for (int m = 0; m < kMaxConvWidth; ++m) {
+        const int r = W - 2 - (kMaxConvWidth - 1 - m);
+        if (r >= 0) hist[(size_t)r * C] = (uint16_t)win[m];
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Cluster barrier, split into arrive and wait so independent work can sit between.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of this cluster.
+template <typename Tp>
+__device__ __forceinline__ Tp* cluster_map(Tp* p, int rank) {
+    uint64_t out;
+    asm volatile("mapa.u64 %0, %1, %2;\n" : "=l"(out) : "l"((uint64_t)p), "r"(rank));
+    return (Tp*)out;
+}
+
+// ---------------------------------------------------------------------------------
+// Geometry of the register tile: a CTA holds S[0:DK][col0:col0+DVS] of one head.
+// A thread owns RPT consecutive rows and 4 consecutive columns (one float4 per row);
+// TPR threads span a row, so each row segment is read and written as whole sectors.
+template <int DK, int DVS>
+struct Tile {
+    static constexpr int NT = (DK * DVS / 64) < 64 ? 64 : ((DK * DVS / 64) > 256 ? 256 : DK * DVS / 64);
+    static constexpr int TPR = DVS / 4;
+    static constexpr int RPP = NT / TPR;
+    static constexpr int RPT = DK / RPP;
+    static constexpr int NW = NT / 32;
+    static_assert(DVS % 4 == 0 && TPR <= 32 && 32 % TPR == 0, "column slice");
+    static_assert(NT % TPR == 0 && RPP <= DK && DK % RPP == 0, "row split");
+};
+
+// Shared-memory block the delta-rule pass reads: per token the raw (unnormalised)
+// q and k of the k-head, the v slice and the per-token scalars.
+struct TokenScalars {
+    float alpha, beta;  // decay exp(g) and write strength
+    float nq, nk;       // factors turning the raw q, k into the normalised (scaled) q, k
+    float kq;           // k . q of the normalised vectors
+};
+
+// The gated delta rule on a register tile for tokens 0..T-1, one pass over S:
+//   m = S^T k (old S), delta = beta (v - alpha m), S <- alpha S + k delta^T,
+//   o = alpha S^T q + delta (k . q)   (= S_new^T q)
+// qk  : [T][2*DK] raw q then raw k (shared)
+// vs  : [T][DVS] v slice (shared);  os : [T][DVS] receives o (shared)
+// red : [2][NW][2][DVS] scratch for the cross-warp sums (shared)
+template <int DK, int DVS>
+__device__ __forceinline__ void delta_rule_tile(float4 (&S)[Tile<DK, DVS>::RPT], const float* qk,
+                                                const float* vs, const TokenScalars* sc, float* os,
+                                                float* red, int T) {
+    using Geo = Tile<DK, DVS>;
+    constexpr int RPT = Geo::RPT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cg = tid % Geo::TPR, rp = tid / Geo::TPR;
+    const int row0 = rp * RPT;
+    for (int t = 0; t < T; ++t) {
+        const float* qr = qk + t * 2 * DK;
+        const float* kr = qr + DK;
+        float kreg[RPT];
+        float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
+#pragma unroll
+        for (int s = 0; s < RPT; ++s) {
+            const float ki = kr[row0 + s], qi = qr[row0 + s];
+            kreg[s] = ki;
+            mk.x = fmaf(S[s].x, ki, mk.x); mk.y = fmaf(S[s].y, ki, mk.y);
+            mk.z = fmaf(S[s].z, ki, mk.z); mk.w = fmaf(S[s].w, ki, mk.w);
+            mq.x = fmaf(S[s].x, qi, mq.x); mq.y = fmaf(S[s].y, qi, mq.y);
+            mq.z = fmaf(S[s].z, qi, mq.z); mq.w = fmaf(S[s].w, qi, mq.w);
+        }
+        // rows held by the other lanes of this warp with the same column group
+#pragma unroll
+        for (int off = Geo::TPR; off < 32; off <<= 1) {
+            mk.x += __shfl_xor_sync(0xffffffffu, mk.x, off); mk.y += __shfl_xor_sync(0xffffffffu, mk.y, off);
+            mk.z += __shfl_xor_sync(0xffffffffu, mk.z, off); mk.w += __shfl_xor_sync(0xffffffffu, mk.w, off);
+            mq.x += __shfl_xor_sync(0xffffffffu, mq.x, off); mq.y += __shfl_xor_sync(0xffffffffu, mq.y, off);
+            mq.z += __shfl_xor_sync(0xffffffffu, mq.z, off); mq.w += __shfl_xor_sync(0xffffffffu, mq.w, off);
+        }
+        float* rb = red + (t & 1) * (Geo::NW * 2 * DVS);
+        if (lane < Geo::TPR) {
+            reinterpret_cast<float4*>(rb + (warp * 2 + 0) * DVS)[cg] = mk;
+            reinterpret_cast<float4*>(rb + (warp * 2 + 1) * DVS)[cg] = mq;
+        }
+        __syncthreads();
+        mk = make_float4(0.f, 0.f, 0.f, 0.f);
+        mq = mk;
+#pragma unroll
+        for (int w = 0; w < Geo::NW; ++w) {
+            const float4 a = reinterpret_cast<const float4*>(rb + (w * 2 + 0) * DVS)[cg];
+            const float4 b = reinterpret_cast<const float4*>(rb + (w * 2 + 1) * DVS)[cg];
+            mk.x += a.x; mk.y += a.y; mk.z += a.z; mk.w += a.w;
+            mq.x += b.x; mq.y += b.y; mq.z += b.z; mq.w += b.w;
+        }
+        const TokenScalars c = sc[t];
+        const float4 v = reinterpret_cast<const float4*>(vs + t * DVS)[cg];
+        const float am = c.alpha * c.nk, aq = c.alpha * c.nq;
+        float4 d, o;
+        d.x = c.beta * fmaf(-am, mk.x, v.x); d.y = c.beta * fmaf(-am, mk.y, v.y);
+        d.z = c.beta * fmaf(-am, mk.z, v.z); d.w = c.beta * fmaf(-am, mk.w, v.w);
+        o.x = fmaf(aq, mq.x, d.x * c.kq); o.y = fmaf(aq, mq.y, d.y * c.kq);
+        o.z = fmaf(aq, mq.z, d.z * c.kq); o.w = fmaf(aq, mq.w, d.w * c.kq);
+        if (rp == 0) reinterpret_cast<float4*>(os + t * DVS)[cg] = o;
+        // the raw k times nk is the normalised k: fold nk into delta
+        const float4 dn = make_float4(d.x * c.nk, d.y * c.nk, d.z * c.nk, d.w * c.nk);
+#pragma unroll
+        for (int s = 0; s < RPT; ++s) {
+            S[s].x = fmaf(c.alpha, S[s].x, kreg[s] * dn.x); S[s].y = fmaf(c.alpha, S[s].y, kreg[s] * dn.y);
+            S[s].z = fmaf(c.alpha, S[s].z, kreg[s] * dn.z); S[s].w = fmaf(c.alpha, S[s].w, kreg[s] * dn.w);
+        }
+    }
+}
+
+// Per-token sums over the raw q and k of one k-head held in shared memory:
+// |q|^2, |k|^2 and q.k, one warp per token. Writes nq, nk, kq of `sc`.
+template <int DK>
+__device__ __forceinline__ void qk_norms(const float* qk, TokenScalars* sc, int T, float l2_eps, float q_scale,
+                                         int nwarps) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int t = warp; t < T; t += nwarps) {
+        const float* qr = qk + t * 2 * DK;
+        const float* kr = qr + DK;
+        float sq = 0.f, sk = 0.f, dot = 0.f;
+        for (int i = lane; i < DK; i += 32) {
+            const float a = qr[i], b = kr[i];
+            sq = fmaf(a, a, sq);
+            sk = fmaf(b, b, sk);
+            dot = fmaf(a, b, dot);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        }
+        if (lane == 0) {
+            const float nq = rsqrtf(sq + l2_eps) * q_scale, nk = rsqrtf(sk + l2_eps);
+            sc[t].nq = nq;
+            sc[t].nk = nk;
+            sc[t].kq = dot * nq * nk;
+        }
+    }
+}
+
+}  // namespace gdn

@@ -1,0 +1,87 @@
+// Internal interface between the C-ABI layer (argument checks) and the kernel
+// launchers. Nothing here is exported.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct Shape {
+    int Hk, Hv, dk, dv, W;  // heads, head dims, conv width
+    int C;                  // 2*Hk*dk + Hv*dv
+    float l2_eps, rms_eps, q_scale;
+};
+
+struct DecodeArgs {
+    Shape sh;
+    int B, T, P;
+    int NS;  // column slices per v-head (dv / NS columns per CTA)
+    const uint16_t* qkv;
+    const uint16_t* a;
+    const uint16_t* b;
+    const uint16_t* z;
+    const uint16_t* conv_w;
+    const float* A_log;
+    const float* dt_bias;
+    const uint16_t* norm_w;
+    uint16_t* conv_pool;
+    float* state_pool;
+    const int32_t* slots;
+    uint16_t* out;
+    float* out_f32;
+    int32_t* err_flag;
+};
+
+struct ConvArgs {
+    Shape sh;
+    int B, T, P;
+    const uint16_t* qkv;
+    const uint16_t* conv_w;
+    uint16_t* conv_pool;
+    const int32_t* slots;
+    float* q;
+    float* k;
+    float* v;
+    int32_t* err_flag;
+};
+
+struct RecurrentArgs {
+    Shape sh;
+    int B, T, P;
+    int NS;
+    const float* q;
+    const float* k;
+    const float* v;
+    const uint16_t* a;
+    const uint16_t* b;
+    const float* A_log;
+    const float* dt_bias;
+    float* state_pool;
+    const int32_t* slots;
+    float* o;
+    int32_t* err_flag;
+};
+
+struct NormArgs {
+    Shape sh;
+    int rows;
+    const float* o;
+    const uint16_t* z;
+    const uint16_t* norm_w;
+    uint16_t* out;
+    float* out_f32;
+};
+
+// Column slices per v-head for the fused kernel: the cluster of one (sequence,
+// k-head) holds G * NS CTAs, at most 8.
+int decode_column_splits(int B, int Hv, int G, int dv);
+// Column slices per v-head for the stand-alone recurrence (no cluster).
+int recurrent_column_splits(int B, int Hv, int dv);
+
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_conv_update(const ConvArgs& a, cudaStream_t stream);
+cudaError_t launch_recurrent(const RecurrentArgs& a, cudaStream_t stream);
+cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,160 @@
+/*
+ * gdn.h — C ABI of libgdn: the Gated DeltaNet (GDN) decode step on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the single-token (or short multi-token) decode of one GDN
+ * linear-attention layer, as dispatched on the page
+ * "spark_model/forward/qwen3_5/linear_attention.rs" (Atlas), steps 3 to 8 plus the
+ * SiLU(z) gate of the fused steps 9+10+11:
+ *
+ *   conv   : per channel, a depthwise causal conv of width W over the stored W-1 raw
+ *            inputs and the new ones (no bias), SiLU; per-head L2 norm of the Q and K
+ *            channels, x / sqrt(sum x^2 + l2_eps); q additionally times q_scale
+ *   gate   : g = -exp(A_log) * softplus(a + dt_bias), alpha = exp(g); beta = sigmoid(b)
+ *   update : per (sequence, v-head h) with k-head h / (Hv/Hk), FP32 state S[dk][dv]:
+ *            S <- alpha S;  S <- S + beta k (v - S^T k)^T;  o = S^T q
+ *   norm   : out = o / sqrt(mean_j o_j^2 + rms_eps) * norm_w * silu(z)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers. Every tensor argument is a DEVICE pointer owned by the caller,
+ *   contiguous, row-major in the layout stated, and 16-byte aligned. bf16 values are
+ *   passed as their uint16_t bit patterns. The library allocates nothing, keeps no
+ *   state between calls and never synchronizes; it only enqueues kernels on `stream`
+ *   (a cudaStream_t; NULL means the legacy default stream). Outputs must not alias
+ *   inputs or one another.
+ * Shapes. Hk = num_k_heads, Hv = num_v_heads (a multiple of Hk, Hv/Hk <= 8),
+ *   dk = head_k_dim, dv = head_v_dim (each 16, 32, 64 or 128), W = conv_width (2..8),
+ *   C = 2*Hk*dk + Hv*dv qkv channels ordered Q | K | V, head-major inside each block.
+ *   B = sequences in this call (B = 0 is a no-op), T = tokens per sequence (1..16),
+ *   P = pool_slots.
+ * Pools. conv_pool [P][W-1][C] bf16 holds each slot's last W-1 raw (pre-conv) inputs,
+ *   row 0 the oldest; state_pool [P][Hv][dk][dv] fp32. Sequence b uses slot slots[b]
+ *   of both pools; slots[] (int32, device) must hold distinct values. Pools are
+ *   updated in place; slots that no sequence names are never read or written.
+ * Multi-token calls (T > 1) are defined as T single-token calls in order.
+ * Errors. Every argument check runs on the host before anything is enqueued, so a
+ *   call that returns an error has written nothing. Slot VALUES live on the device:
+ *   a sequence whose slot is outside [0, P) is skipped entirely (its pools and
+ *   outputs untouched) and, when err_flag is non-NULL, *err_flag is set to
+ *   GDN_DEVICE_ERR_SLOT_RANGE (the caller zeroes it; the library never clears it).
+ *   Duplicate slots are not detected on the device and give undefined results;
+ *   gdn_check_slots_host() checks a host copy. A failed launch returns GDN_ERR_CUDA.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, eps < 0, bad pool size */
+    GDN_ERR_UNSUPPORTED = 2,      /* a shape outside the supported set above */
+    GDN_ERR_MISALIGNED = 3,       /* a tensor pointer not 16-byte aligned */
+    GDN_ERR_SLOT_RANGE = 4,       /* gdn_check_slots_host: slot out of range or repeated */
+    GDN_ERR_CUDA = 5              /* the CUDA launch itself failed */
+} gdn_status;
+
+/* Value a kernel stores into *err_flag when a sequence's slot is out of range. */
+#define GDN_DEVICE_ERR_SLOT_RANGE 1
+
+typedef struct {
+    int32_t num_k_heads; /* Hk */
+    int32_t num_v_heads; /* Hv, a multiple of Hk */
+    int32_t head_k_dim;  /* dk */
+    int32_t head_v_dim;  /* dv */
+    int32_t conv_width;  /* W */
+    float l2_eps;        /* q/k L2-norm epsilon (inside the root); the page uses 1e-6 */
+    float rms_eps;       /* output RMSNorm epsilon (inside the root) */
+    float q_scale;       /* factor on the normalised q; 0 selects 1/sqrt(dk) */
+} gdn_config;
+
+/*
+ * Stage 1 — step 3 of the page, "fused causal_conv1d_update_l2norm", with the
+ * 1/sqrt(d_k) q scale it applies at the kernel output, and the Q|K|V split of step 6.
+ *   qkv     [B][T][C] bf16        this call's raw projections
+ *   conv_w  [C][W] bf16           tap W-1 multiplies the current token
+ *   conv_pool, pool_slots, slots  as above; the slot's history is rolled in place
+ *   q_out   [B][T][Hk][dk] fp32   L2-normalised, times q_scale
+ *   k_out   [B][T][Hk][dk] fp32   L2-normalised
+ *   v_out   [B][T][Hv][dv] fp32   SiLU output, no norm
+ *   err_flag nullable device int32
+ */
+gdn_status gdn_conv_update(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv,
+                           const uint16_t* conv_w, uint16_t* conv_pool, int32_t pool_slots,
+                           const int32_t* slots, float* q_out, float* k_out, float* v_out,
+                           int32_t* err_flag, void* stream);
+
+/*
+ * Stage 2 — steps 4, 5 and 7 of the page: the gate, beta and
+ * "gated_delta_rule_decode" on the FP32 state pool, one pass over each state.
+ *   q, k    [B][T][Hk][dk] fp32   as produced by gdn_conv_update (q already scaled)
+ *   v       [B][T][Hv][dv] fp32
+ *   a, b    [B][T][Hv] bf16       raw gate and beta projections
+ *   A_log, dt_bias [Hv] fp32
+ *   state_pool, pool_slots, slots as above; each named state is read once and
+ *                                 written once (after all T tokens)
+ *   o       [B][T][Hv][dv] fp32   S^T q with S after the token's update
+ */
+gdn_status gdn_recurrent_step(const gdn_config* cfg, int32_t B, int32_t T, const float* q,
+                              const float* k, const float* v, const uint16_t* a, const uint16_t* b,
+                              const float* A_log, const float* dt_bias, float* state_pool,
+                              int32_t pool_slots, const int32_t* slots, float* o,
+                              int32_t* err_flag, void* stream);
+
+/*
+ * Stage 3 — step 8 of the page (per-head RMSNorm over dv with one weight vector
+ * shared by all heads) and the SiLU(z) gate of steps 9+10+11.
+ *   rows     number of (sequence, token, v-head) rows, i.e. B*T*Hv
+ *   o        [rows][dv] fp32
+ *   z        [rows][dv] bf16
+ *   norm_w   [dv] bf16
+ *   out_bf16 [rows][dv] bf16      round-to-nearest-even of the fp32 result
+ *   out_f32  [rows][dv] fp32      nullable; the same result before rounding
+ */
+gdn_status gdn_gated_rmsnorm(const gdn_config* cfg, int32_t rows, const float* o, const uint16_t* z,
+                             const uint16_t* norm_w, uint16_t* out_bf16, float* out_f32,
+                             void* stream);
+
+/*
+ * The fused decode step: the three stages above in ONE kernel launch. Each state
+ * tile is streamed from HBM once and written back in place; the conv history of
+ * every channel is read and rolled by exactly one CTA; q, k, v, the gates and o
+ * never leave the chip.
+ *   qkv [B][T][C], a [B][T][Hv], b [B][T][Hv], z [B][T][Hv][dv]   bf16 inputs
+ *   conv_w [C][W] bf16, A_log [Hv] fp32, dt_bias [Hv] fp32, norm_w [dv] bf16
+ *   conv_pool, state_pool, pool_slots, slots                     as above
+ *   out_bf16 [B][T][Hv][dv] bf16
+ *   out_f32  [B][T][Hv][dv] fp32, nullable (the unrounded output, for parity checks)
+ *   err_flag nullable device int32
+ */
+gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv,
+                           const uint16_t* a, const uint16_t* b, const uint16_t* z,
+                           const uint16_t* conv_w, const float* A_log, const float* dt_bias,
+                           const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                           int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
+                           float* out_f32, int32_t* err_flag, void* stream);
+
+/*
+ * Host-side check of a HOST copy of slots[]: GDN_OK when all B values are distinct
+ * and in [0, pool_slots), GDN_ERR_SLOT_RANGE otherwise, GDN_ERR_INVALID_ARGUMENT for
+ * a null pointer or negative size. Touches no device.
+ */
+gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t pool_slots);
+
+/* A static, human-readable name for a status code. */
+const char* gdn_status_string(gdn_status status);
+
+/* ABI version of this header: (major << 16) | minor. */
+#define GDN_ABI_VERSION ((1 << 16) | 0)
+int32_t gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

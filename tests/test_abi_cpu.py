@@ -1,0 +1,148 @@
+"""The C-ABI library on the host, without a GPU: it loads, exports every entry
+point that include/gdn.h declares, and rejects bad arguments before enqueuing
+anything. Every call here fails a host check on purpose (fake pointer values are
+never dereferenced), so the file is safe to run on a machine with a GPU too."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import gated_delta_rule_102_b200 as gdn
+from gated_delta_rule_102_b200 import build as gdn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = open(os.path.join(ROOT, "include", "gdn.h")).read()
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdn_build.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    body = re.sub(r"/\*.*?\*/", "", HEADER, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_\w+)\s*\(", body)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {gdn.LIB_PATH}").read()
+    exported = set(re.findall(r" T (gdn_\w+)", out))
+    assert set(declared_functions()) <= exported
+    assert set(gdn._abi.EXPORTS) == set(declared_functions())
+
+
+def test_abi_version_matches_header(L):
+    m = re.search(r"#define GDN_ABI_VERSION \(\((\d+) << 16\) \| (\d+)\)", HEADER)
+    assert gdn.abi_version() == (int(m.group(1)) << 16) | int(m.group(2))
+
+
+def test_status_codes_match_header(L):
+    for name in ("GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_MISALIGNED",
+                 "GDN_ERR_SLOT_RANGE", "GDN_ERR_CUDA"):
+        m = re.search(rf"\b{name} = (\d+)", HEADER)
+        assert m and int(m.group(1)) == getattr(gdn, name)
+        assert gdn.status_string(getattr(gdn, name))
+    m = re.search(r"#define GDN_DEVICE_ERR_SLOT_RANGE (\d+)", HEADER)
+    assert int(m.group(1)) == gdn.GDN_DEVICE_ERR_SLOT_RANGE
+
+
+def test_check_slots_host(L):
+    assert gdn.gdn_check_slots_host([0, 3, 1], 4) == gdn.GDN_OK
+    assert gdn.gdn_check_slots_host([], 4) == gdn.GDN_OK
+    assert gdn.gdn_check_slots_host([0, 4], 4) == gdn.GDN_ERR_SLOT_RANGE
+    assert gdn.gdn_check_slots_host([-1], 4) == gdn.GDN_ERR_SLOT_RANGE
+    assert gdn.gdn_check_slots_host([2, 1, 2], 4) == gdn.GDN_ERR_SLOT_RANGE
+    assert L.gdn_check_slots_host(None, 3, 4) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert L.gdn_check_slots_host(None, -1, 4) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
+FAKE = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced
+FAKE_ODD = ctypes.c_void_p((1 << 20) + 2)
+
+
+def good_cfg(**kw):
+    base = dict(num_k_heads=16, num_v_heads=32, head_k_dim=128, head_v_dim=128, conv_width=4)
+    base.update(kw)
+    return gdn.GdnConfig.make(**base)
+
+
+def decode(L, cfg, B=4, T=1, ptrs=None, pool=8, out_f32=None, err=None):
+    p = [FAKE] * 10 if ptrs is None else ptrs
+    return L.gdn_decode_step(ctypes.byref(cfg) if cfg is not None else None, B, T, *p, pool, FAKE, FAKE,
+                             out_f32, err, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_k_heads=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(num_v_heads=-2), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(num_v_heads=24, num_k_heads=16), gdn.GDN_ERR_INVALID_ARGUMENT),  # Hv not a multiple of Hk
+    (dict(num_v_heads=160, num_k_heads=16), gdn.GDN_ERR_UNSUPPORTED),      # Hv/Hk = 10 > 8
+    (dict(head_k_dim=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(head_v_dim=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(head_v_dim=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(conv_width=1), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(conv_width=9), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(l2_eps=-1.0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(rms_eps=float("nan")), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(q_scale=float("inf")), gdn.GDN_ERR_INVALID_ARGUMENT),
+])
+def test_decode_rejects_bad_config(L, kw, status):
+    assert decode(L, good_cfg(**kw)) == status
+
+
+def test_decode_rejects_bad_sizes_and_pointers(L):
+    cfg = good_cfg()
+    assert decode(L, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert decode(L, cfg, B=-1) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert decode(L, cfg, T=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert decode(L, cfg, T=17) == gdn.GDN_ERR_UNSUPPORTED
+    assert decode(L, cfg, pool=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    for i in range(10):
+        ptrs = [FAKE] * 10
+        ptrs[i] = None
+        assert decode(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
+        ptrs[i] = FAKE_ODD
+        assert decode(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
+    assert decode(L, cfg, out_f32=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    assert decode(L, cfg, err=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+
+
+def test_empty_batch_is_a_no_op(L):
+    # B = 0 returns before any pointer is looked at or any launch is made
+    assert decode(L, good_cfg(), B=0, ptrs=[None] * 10) == gdn.GDN_OK
+    assert L.gdn_conv_update(ctypes.byref(good_cfg()), 0, 1, *([None] * 3), 4, *([None] * 6)) == gdn.GDN_OK
+    assert L.gdn_gated_rmsnorm(ctypes.byref(good_cfg()), 0, *([None] * 5), None) == gdn.GDN_OK
+
+
+def test_stage_entry_points_check_arguments(L):
+    cfg = good_cfg()
+    assert L.gdn_conv_update(ctypes.byref(cfg), 2, 1, FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, FAKE, None,
+                             None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert L.gdn_conv_update(ctypes.byref(good_cfg(conv_width=12)), 2, 1, *([FAKE] * 3), 4,
+                             *([FAKE] * 4), None, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_recurrent_step(ctypes.byref(cfg), 2, 1, *([FAKE] * 7), FAKE_ODD, 4, FAKE, FAKE, None,
+                                None) == gdn.GDN_ERR_MISALIGNED
+    assert L.gdn_recurrent_step(ctypes.byref(cfg), 2, 20, *([FAKE] * 8), 4, FAKE, FAKE, None,
+                                None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_gated_rmsnorm(ctypes.byref(cfg), -1, *([FAKE] * 4), None, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert L.gdn_gated_rmsnorm(ctypes.byref(cfg), 4, FAKE, FAKE, None, FAKE, None,
+                               None) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    cfg = good_cfg(num_k_heads=1, num_v_heads=1, head_k_dim=16, head_v_dim=16)
+    x = torch.zeros(1, 1, cfg.channels, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, TypeError)):
+        gdn.gdn_decode_step(cfg, x, x, x, x, x, x, x, x, x, x, x, x)

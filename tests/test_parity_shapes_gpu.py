@@ -1,0 +1,215 @@
+"""GPU parity across shapes and edge cases: head dims 16..128 with dk != dv, GQA
+ratios 1..8 (including 3, a non power of two cluster), conv widths 2..8, T = 1..16,
+ragged batches, sparse pools; the three stage entry points one by one; bad slots;
+empty batches; split runs; determinism."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_102_b200 as gdn
+import oracle
+from gated_delta_rule_102_b200 import synth
+from gdn_harness import (GpuRun, OracleRun, bf16_dev, bf16_host, compare_out, compare_state, conv_pool_reference,
+                         f32_dev)
+
+pytestmark = pytest.mark.gpu
+
+BASE = synth.WORKLOADS["tiny_d16"]
+
+
+def wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed, slot_mode="sample", std=0.02):
+    if slot_mode == "permutation":
+        P = B
+    return BASE.replace(name=name, num_k_heads=Hk, num_v_heads=Hv, head_k_dim=dk, head_v_dim=dv, conv_width=W,
+                        batch=B, tokens=T, pool_slots=P, steps=steps, seed=seed, slot_mode=slot_mode,
+                        state_std=std)
+
+
+SHAPES = [
+    # name            Hk Hv  dk   dv  W  B  T  P  steps
+    ("dk64_dv128_g2", 2, 4, 64, 128, 4, 3, 1, 5, 3),
+    ("dk128_dv32_g8", 1, 8, 128, 32, 3, 2, 2, 3, 3),
+    ("dk32_dv64_g1", 3, 3, 32, 64, 2, 5, 4, 7, 2),
+    ("dk16_dv128_g3", 2, 6, 16, 128, 4, 2, 3, 2, 3),
+    ("dk128_g4_t16", 4, 16, 128, 128, 4, 2, 16, 3, 2),
+    ("d16_t16", 1, 2, 16, 16, 4, 3, 16, 4, 2),
+    ("w8_t5", 2, 4, 32, 32, 8, 2, 5, 2, 3),
+    ("w2_t1_b1", 16, 32, 128, 128, 2, 1, 1, 1, 3),
+    ("dk64_dv16_g4_t7", 2, 8, 64, 16, 3, 4, 7, 9, 2),
+    ("b33_ragged", 2, 4, 128, 64, 4, 33, 1, 40, 2),
+    ("dk64_dv128_g8_t16", 1, 8, 64, 128, 4, 2, 16, 2, 2),
+]
+
+
+@pytest.mark.parametrize("spec", SHAPES, ids=[s[0] for s in SHAPES])
+def test_fused_matches_oracle(spec):
+    name, Hk, Hv, dk, dv, W, B, T, P, steps = spec
+    wl = wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed=zlib.crc32(name.encode()) % 10000)
+    g = GpuRun(wl)
+    rows = list(range(B))
+    o = OracleRun(wl, rows)
+    pool0 = g.state.clone()
+    for s in range(steps):
+        out, out32 = g.step(g.inputs(s))
+        r = o.step(s)
+        compare_out(out, out32, r["out"], rows, f"{name} step {s}")
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == 0
+    compare_state(g.state, o.state, o.slot_ids, name)
+    np.testing.assert_array_equal(bf16_host(g.conv), conv_pool_reference(wl, steps))
+    idle = sorted(set(range(P)) - set(g.slots_np.tolist()))
+    if idle:
+        idx = torch.tensor(idle, device="cuda")
+        assert torch.equal(g.state[idx], pool0[idx])
+
+
+def _stage_problem(seed=5, Hk=2, Hv=4, dk=64, dv=128, W=4, B=3, T=3, P=4):
+    wl = wl_of("stages", Hk, Hv, dk, dv, W, B, T, P, 1, seed)
+    return wl, GpuRun(wl), synth.step_inputs(wl, 0)
+
+
+def test_conv_stage_matches_oracle():
+    wl, g, x = _stage_problem()
+    B, T = wl.batch, wl.tokens
+    q = torch.empty(B, T, wl.num_k_heads, wl.head_k_dim, device="cuda")
+    k = torch.empty_like(q)
+    v = torch.empty(B, T, wl.num_v_heads, wl.head_v_dim, device="cuda")
+    gdn.gdn_conv_update(g.cfg, bf16_dev(x["qkv"]), g.conv_w, g.conv, g.slots, q, k, v, g.err)
+    pool = synth.initial_conv_state(wl)
+    w = synth.weights(wl)
+    rq, rk, rv = oracle.conv_update(oracle.Shape.of(wl), x["qkv"], w["conv_w"], pool, g.slots_np)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(q.cpu().numpy(), rq, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(k.cpu().numpy(), rk, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(v.cpu().numpy(), rv, rtol=2e-6, atol=2e-6)
+    np.testing.assert_array_equal(bf16_host(g.conv), pool)
+
+
+def test_recurrent_stage_matches_oracle():
+    wl, g, x = _stage_problem(seed=6, T=5)
+    B, T = wl.batch, wl.tokens
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((B, T, wl.num_k_heads, wl.head_k_dim)).astype(np.float32)
+    k = rng.standard_normal(q.shape).astype(np.float32)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, wl.num_v_heads, wl.head_v_dim)).astype(np.float32)
+    o = torch.empty(B, T, wl.num_v_heads, wl.head_v_dim, device="cuda")
+    gdn.gdn_recurrent_step(g.cfg, f32_dev(q), f32_dev(k), f32_dev(v), bf16_dev(x["a"]), bf16_dev(x["b"]),
+                           g.A_log, g.dt_bias, g.state, g.slots, o, g.err)
+    w = synth.weights(wl)
+    sh = oracle.Shape.of(wl)
+    al, be = oracle.gate(sh, x["a"], x["b"], w["A_log"], w["dt_bias"])
+    st = synth.initial_state(wl).astype(np.float64)
+    ro = oracle.delta_rule(sh, q, k, v, al, be, st, g.slots_np)
+    torch.cuda.synchronize()
+    scale = np.abs(ro).max()
+    assert np.abs(o.cpu().numpy() - ro).max() <= 1e-5 * scale
+    compare_state(g.state, st[g.slots_np], [int(s) for s in g.slots_np], "recurrent stage")
+
+
+def test_gated_rmsnorm_stage_matches_oracle():
+    wl, g, x = _stage_problem(seed=7)
+    rng = np.random.default_rng(1)
+    o = rng.standard_normal((wl.batch, wl.tokens, wl.num_v_heads, wl.head_v_dim)).astype(np.float32)
+    out = torch.empty(o.shape, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.empty(o.shape, dtype=torch.float32, device="cuda")
+    gdn.gdn_gated_rmsnorm(g.cfg, f32_dev(o), bf16_dev(x["z"]), g.norm_w, out, out32)
+    ref = oracle.gated_rmsnorm(oracle.Shape.of(wl), o, x["z"], synth.weights(wl)["norm_w"])
+    compare_out(out, out32, ref, list(range(wl.batch)), "gated rmsnorm")
+    assert np.abs(out32.cpu().numpy() - ref).max() < 1e-5
+
+
+def test_fused_equals_stage_chain():
+    wl, g, x = _stage_problem(seed=8, T=2)
+    g2 = GpuRun(wl)
+    B, T = wl.batch, wl.tokens
+    out, out32 = g.step({k: bf16_dev(v) for k, v in x.items()})
+    q = torch.empty(B, T, wl.num_k_heads, wl.head_k_dim, device="cuda")
+    k = torch.empty_like(q)
+    v = torch.empty(B, T, wl.num_v_heads, wl.head_v_dim, device="cuda")
+    gdn.gdn_conv_update(g2.cfg, bf16_dev(x["qkv"]), g2.conv_w, g2.conv, g2.slots, q, k, v)
+    o = torch.empty_like(v)
+    gdn.gdn_recurrent_step(g2.cfg, q, k, v, bf16_dev(x["a"]), bf16_dev(x["b"]), g2.A_log, g2.dt_bias,
+                           g2.state, g2.slots, o)
+    out2 = torch.empty_like(out)
+    out2_32 = torch.empty_like(out32)
+    gdn.gdn_gated_rmsnorm(g2.cfg, o, bf16_dev(x["z"]), g2.norm_w, out2, out2_32)
+    torch.cuda.synchronize()
+    assert (out32 - out2_32).abs().max().item() < 1e-4
+    assert torch.equal(g.conv, g2.conv)
+    assert ((g.state - g2.state).abs().max() / g.state.abs().max()).item() < 1e-5
+
+
+def test_out_of_range_slot_is_skipped_and_flagged():
+    wl = wl_of("badslot", 2, 4, 32, 32, 4, 3, 1, 4, 1, seed=9)
+    g = GpuRun(wl)
+    g.slots = torch.tensor([1, 7, 3], dtype=torch.int32, device="cuda")  # 7 is outside the 4-slot pool
+    g.slots_np = g.slots.cpu().numpy()
+    state0, conv0 = g.state.clone(), g.conv.clone()
+    x = g.inputs(0)
+    shape = (3, 1, 4, 32)
+    out = torch.full(shape, 7.0, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.full(shape, 7.0, device="cuda")
+    gdn.gdn_decode_step(g.cfg, x["qkv"], x["a"], x["b"], x["z"], g.conv_w, g.A_log, g.dt_bias, g.norm_w,
+                        g.conv, g.state, g.slots, out, out32, g.err)
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == gdn.GDN_DEVICE_ERR_SLOT_RANGE
+    assert torch.all(out32[1] == 7.0) and torch.all(out[1].float() == 7.0)
+    for s in (0, 2):  # untouched slots keep their bytes
+        assert torch.equal(g.state[s], state0[s]) and torch.equal(g.conv[s], conv0[s])
+    # the valid sequences were computed as usual
+    o = OracleRun(wl.replace(pool_slots=4), [0, 2], state0=state0.cpu().numpy())
+    o.slot_ids = [1, 3]
+    o.state = state0.cpu().numpy()[[1, 3]].astype(np.float64)
+    r = o.step(0)
+    compare_out(out, out32, r["out"], [0, 2], "valid rows beside a bad slot")
+    # and the stage kernels flag it too
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = torch.empty(3, 1, 2, 32, device="cuda")
+    gdn.gdn_conv_update(g.cfg, x["qkv"], g.conv_w, g.conv, g.slots, q, q.clone(),
+                        torch.empty(3, 1, 4, 32, device="cuda"), err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == gdn.GDN_DEVICE_ERR_SLOT_RANGE
+
+
+def test_empty_batch_is_a_no_op_on_device():
+    wl = wl_of("empty", 2, 4, 32, 32, 4, 2, 1, 2, 1, seed=10)
+    g = GpuRun(wl)
+    st, cv = g.state.clone(), g.conv.clone()
+    e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device="cuda")  # noqa: E731
+    gdn.gdn_decode_step(g.cfg, e(0, 1, wl.channels), e(0, 1, 4), e(0, 1, 4), e(0, 1, 4, 32), g.conv_w, g.A_log,
+                        g.dt_bias, g.norm_w, g.conv, g.state, e(0, dt=torch.int32), e(0, 1, 4, 32))
+    torch.cuda.synchronize()
+    assert torch.equal(g.state, st) and torch.equal(g.conv, cv)
+
+
+def test_split_run_resumes_bit_identically():
+    # N steps, pools copied to the host and back into fresh buffers, M more steps:
+    # the same bits as N + M steps in one go (the pools are the whole resumable state).
+    wl = wl_of("resume", 2, 4, 64, 64, 4, 4, 2, 6, 6, seed=11)
+    a = GpuRun(wl)
+    for s in range(6):
+        out_a, _ = a.step(a.inputs(s))
+    b = GpuRun(wl)
+    for s in range(3):
+        b.step(b.inputs(s))
+    state_host, conv_host = b.state.cpu(), b.conv.cpu()
+    c = GpuRun(wl)
+    c.state.copy_(state_host.cuda())
+    c.conv.copy_(conv_host.cuda())
+    for s in range(3, 6):
+        out_c, _ = c.step(c.inputs(s))
+    torch.cuda.synchronize()
+    assert torch.equal(a.state, c.state) and torch.equal(a.conv, c.conv) and torch.equal(out_a, out_c)
+
+
+def test_deterministic():
+    wl = wl_of("det", 2, 4, 128, 128, 4, 8, 1, 8, 1, seed=12, slot_mode="permutation")
+    a, b = GpuRun(wl), GpuRun(wl)
+    x = a.inputs(0)
+    oa, oa32 = a.step(x)
+    ob, ob32 = b.step(x)
+    torch.cuda.synchronize()
+    assert torch.equal(oa, ob) and torch.equal(oa32, ob32) and torch.equal(a.state, b.state)

@@ -24,6 +24,7 @@ GDN_ERR_MISALIGNED = 3
 GDN_ERR_SLOT_RANGE = 4
 GDN_ERR_CUDA = 5
 GDN_DEVICE_ERR_SLOT_RANGE = 1
+GDN_DEVICE_ERR_TIMEOUT = 2
 
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
            "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")

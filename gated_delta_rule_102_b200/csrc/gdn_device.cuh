@@ -12,6 +12,10 @@
 
 namespace gdn {
 
+// Bits a kernel ORs into the caller's error flag (values of the public header).
+constexpr int GDN_DEVICE_ERR_SLOT_RANGE_BIT = 1;
+constexpr int GDN_DEVICE_ERR_TIMEOUT_BIT = 2;
+
 // Longest conv supported (taps) and most tokens per launch.
 constexpr int kMaxConvWidth = 8;
 constexpr int kMaxTokens = 16;
@@ -225,6 +229,156 @@ __device__ __forceinline__ void qk_norms(const float* qk, TokenScalars* sc, int 
             sc[t].kq = dot * nq * nk;
         }
     }
+}
+
+}  // namespace gdn
+
+namespace gdn {
+
+// ---------------------------------------------------------------------------------
+// TMA bulk copies (global -> shared, completion counted on an mbarrier) and bounded
+// mbarrier waits. No multicast anywhere.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+// Makes the initialised barrier visible to the async proxy and the cluster.
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for phase `parity` of the barrier; gives up after `limit` polls (each poll
+// may suspend the thread for a short hardware-defined time) and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+// One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into
+// this CTA's shared memory, counted on `bar`.
+__device__ __forceinline__ void tma_load_1d(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// The gated delta rule on a DK x DVS tile held in shared memory, for tokens 0..T-1.
+// Same arithmetic as delta_rule_tile; S lives in shared memory between tokens and
+// each thread reads it twice per token (reductions, then update), so registers stay
+// few. After the last token the updated rows go straight to global memory `Sg`
+// (this thread's first float4, row pitch `pitch4` float4s) with streaming stores.
+template <int DK, int DVS>
+__device__ __forceinline__ void delta_rule_smem(float* tile, const float* qk, const float* vs, const TokenScalars* sc,
+                                                float* os, float* red, int T, float4* Sg, size_t pitch4) {
+    using Geo = Tile<DK, DVS>;
+    constexpr int RPT = Geo::RPT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cg = tid % Geo::TPR, rp = tid / Geo::TPR;
+    const int row0 = rp * RPT;
+    float4* tl = reinterpret_cast<float4*>(tile) + (size_t)row0 * (DVS / 4) + cg;
+    for (int t = 0; t < T; ++t) {
+        const float* qr = qk + t * 2 * DK;
+        const float* kr = qr + DK;
+        float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
+#pragma unroll
+        for (int s = 0; s < RPT; ++s) {
+            const float4 v = tl[s * (DVS / 4)];
+            const float ki = kr[row0 + s], qi = qr[row0 + s];
+            mk.x = fmaf(v.x, ki, mk.x); mk.y = fmaf(v.y, ki, mk.y);
+            mk.z = fmaf(v.z, ki, mk.z); mk.w = fmaf(v.w, ki, mk.w);
+            mq.x = fmaf(v.x, qi, mq.x); mq.y = fmaf(v.y, qi, mq.y);
+            mq.z = fmaf(v.z, qi, mq.z); mq.w = fmaf(v.w, qi, mq.w);
+        }
+#pragma unroll
+        for (int off = Geo::TPR; off < 32; off <<= 1) {
+            mk.x += __shfl_xor_sync(0xffffffffu, mk.x, off); mk.y += __shfl_xor_sync(0xffffffffu, mk.y, off);
+            mk.z += __shfl_xor_sync(0xffffffffu, mk.z, off); mk.w += __shfl_xor_sync(0xffffffffu, mk.w, off);
+            mq.x += __shfl_xor_sync(0xffffffffu, mq.x, off); mq.y += __shfl_xor_sync(0xffffffffu, mq.y, off);
+            mq.z += __shfl_xor_sync(0xffffffffu, mq.z, off); mq.w += __shfl_xor_sync(0xffffffffu, mq.w, off);
+        }
+        float* rb = red + (t & 1) * (Geo::NW * 2 * DVS);
+        if (lane < Geo::TPR) {
+            reinterpret_cast<float4*>(rb + (warp * 2 + 0) * DVS)[cg] = mk;
+            reinterpret_cast<float4*>(rb + (warp * 2 + 1) * DVS)[cg] = mq;
+        }
+        __syncthreads();
+        mk = make_float4(0.f, 0.f, 0.f, 0.f);
+        mq = mk;
+#pragma unroll
+        for (int w = 0; w < Geo::NW; ++w) {
+            const float4 a = reinterpret_cast<const float4*>(rb + (w * 2 + 0) * DVS)[cg];
+            const float4 b = reinterpret_cast<const float4*>(rb + (w * 2 + 1) * DVS)[cg];
+            mk.x += a.x; mk.y += a.y; mk.z += a.z; mk.w += a.w;
+            mq.x += b.x; mq.y += b.y; mq.z += b.z; mq.w += b.w;
+        }
+        const TokenScalars c = sc[t];
+        const float4 v = reinterpret_cast<const float4*>(vs + t * DVS)[cg];
+        const float am = c.alpha * c.nk, aq = c.alpha * c.nq;
+        float4 d, o;
+        d.x = c.beta * fmaf(-am, mk.x, v.x); d.y = c.beta * fmaf(-am, mk.y, v.y);
+        d.z = c.beta * fmaf(-am, mk.z, v.z); d.w = c.beta * fmaf(-am, mk.w, v.w);
+        o.x = fmaf(aq, mq.x, d.x * c.kq); o.y = fmaf(aq, mq.y, d.y * c.kq);
+        o.z = fmaf(aq, mq.z, d.z * c.kq); o.w = fmaf(aq, mq.w, d.w * c.kq);
+        if (rp == 0) reinterpret_cast<float4*>(os + t * DVS)[cg] = o;
+        const float4 dn = make_float4(d.x * c.nk, d.y * c.nk, d.z * c.nk, d.w * c.nk);
+        const bool last = t == T - 1;
+#pragma unroll
+        for (int s = 0; s < RPT; ++s) {
+            float4 w = tl[s * (DVS / 4)];
+            const float ki = kr[row0 + s];
+            w.x = fmaf(c.alpha, w.x, ki * dn.x); w.y = fmaf(c.alpha, w.y, ki * dn.y);
+            w.z = fmaf(c.alpha, w.z, ki * dn.z); w.w = fmaf(c.alpha, w.w, ki * dn.w);
+            if (last) __stcs(Sg + (size_t)s * pitch4, w);
+            else tl[s * (DVS / 4)] = w;
+        }
+    }
+}
+
+}  // namespace gdn
+
+namespace gdn {
+
+// ---------------------------------------------------------------------------------
+// Distributed-shared-memory messages completed on the receiver's mbarrier, and the
+// async-proxy fence used before a bulk copy reuses a buffer the threads have read.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_map_u32(uint32_t smem_cta_addr, int rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(out) : "r"(smem_cta_addr), "r"(rank));
+    return out;
+}
+// Store one float into the shared memory of the cluster CTA that owns `remote_addr`
+// and count 4 bytes on that CTA's mbarrier `remote_bar` (both shared::cluster).
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];\n" ::"r"(remote_addr),
+                 "r"(__float_as_uint(v)), "r"(remote_bar)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
 }
 
 }  // namespace gdn

@@ -80,6 +80,9 @@ int decode_column_splits(int B, int Hv, int G, int dv);
 int recurrent_column_splits(int B, int Hv, int dv);
 
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
+// Persistent single-token kernel: co-resident cluster capacity, and the launch.
+cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters);
+cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_conv_update(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_recurrent(const RecurrentArgs& a, cudaStream_t stream);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);

@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_update_kernel(const ConvArg
     const int T = p.T, C = p.sh.C, dk = p.sh.dk, dv = p.sh.dv;
     const int slot = __ldg(p.slots + seq);
     if (slot < 0 || slot >= p.P) {
-        if (threadIdx.x == 0 && seg == 0 && p.err_flag) atomicExch(p.err_flag, 1);
+        if (threadIdx.x == 0 && seg == 0 && p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
         return;
     }
     const bool is_v = seg >= 2 * p.sh.Hk;
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(Tile<DK, DVS>::NT) recurrent_kernel(const Recu
     const int tid = threadIdx.x;
     const int slot = __ldg(p.slots + seq);
     if (slot < 0 || slot >= p.P) {
-        if (tid == 0 && h == 0 && sl == 0 && p.err_flag) atomicExch(p.err_flag, 1);
+        if (tid == 0 && h == 0 && sl == 0 && p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
         return;
     }
     float4 S[RPT];

@@ -35,10 +35,14 @@
  * Errors. Every argument check runs on the host before anything is enqueued, so a
  *   call that returns an error has written nothing. Slot VALUES live on the device:
  *   a sequence whose slot is outside [0, P) is skipped entirely (its pools and
- *   outputs untouched) and, when err_flag is non-NULL, *err_flag is set to
- *   GDN_DEVICE_ERR_SLOT_RANGE (the caller zeroes it; the library never clears it).
- *   Duplicate slots are not detected on the device and give undefined results;
- *   gdn_check_slots_host() checks a host copy. A failed launch returns GDN_ERR_CUDA.
+ *   outputs untouched) and, when err_flag is non-NULL, the bit
+ *   GDN_DEVICE_ERR_SLOT_RANGE is OR-ed into *err_flag (the caller zeroes it; the
+ *   library never clears it). Duplicate slots are not detected on the device and
+ *   give undefined results; gdn_check_slots_host() checks a host copy. Every wait
+ *   inside a kernel is bounded: a CTA whose staged state copy has not landed after
+ *   more than a second gives up, ORs GDN_DEVICE_ERR_TIMEOUT into *err_flag and writes
+ *   neither that state tile nor its outputs (their values are then unspecified).
+ *   A failed launch returns GDN_ERR_CUDA.
  */
 #ifndef GDN_H_
 #define GDN_H_
@@ -59,8 +63,9 @@ typedef enum {
     GDN_ERR_CUDA = 5              /* the CUDA launch itself failed */
 } gdn_status;
 
-/* Value a kernel stores into *err_flag when a sequence's slot is out of range. */
-#define GDN_DEVICE_ERR_SLOT_RANGE 1
+/* Bits a kernel ORs into *err_flag. */
+#define GDN_DEVICE_ERR_SLOT_RANGE 1 /* a sequence's slot is outside [0, pool_slots) */
+#define GDN_DEVICE_ERR_TIMEOUT 2    /* a bounded wait inside the kernel ran out */
 
 typedef struct {
     int32_t num_k_heads; /* Hk */

@@ -53,8 +53,9 @@ def test_status_codes_match_header(L):
         m = re.search(rf"\b{name} = (\d+)", HEADER)
         assert m and int(m.group(1)) == getattr(gdn, name)
         assert gdn.status_string(getattr(gdn, name))
-    m = re.search(r"#define GDN_DEVICE_ERR_SLOT_RANGE (\d+)", HEADER)
-    assert int(m.group(1)) == gdn.GDN_DEVICE_ERR_SLOT_RANGE
+    for name in ("GDN_DEVICE_ERR_SLOT_RANGE", "GDN_DEVICE_ERR_TIMEOUT"):
+        m = re.search(rf"#define {name} (\d+)", HEADER)
+        assert int(m.group(1)) == getattr(gdn, name)
 
 
 def test_check_slots_host(L):

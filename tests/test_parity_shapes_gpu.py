@@ -65,6 +65,48 @@ def test_fused_matches_oracle(spec):
         assert torch.equal(g.state[idx], pool0[idx])
 
 
+# Single-token launches with many (sequence, k-head) groups take the persistent
+# pipelined kernel (at least two groups per co-resident cluster).
+PERSISTENT_SHAPES = [
+    # name              Hk Hv   dk   dv  W    B  T    P  steps
+    ("p_d128_g2", 4, 8, 128, 128, 4, 40, 1, 48, 3),
+    ("p_d128_g1_w2", 2, 2, 128, 128, 2, 160, 1, 170, 2),
+    ("p_dk128_dv64_g4", 2, 8, 128, 64, 4, 80, 1, 80, 2),
+    ("p_dk64_dv128_g8_w3", 1, 8, 64, 128, 3, 100, 1, 101, 2),
+    ("p_d32_g2_many", 2, 4, 32, 32, 3, 800, 1, 800, 3),
+]
+
+
+@pytest.mark.parametrize("spec", PERSISTENT_SHAPES, ids=[s[0] for s in PERSISTENT_SHAPES])
+def test_persistent_path_matches_oracle(spec):
+    test_fused_matches_oracle(spec)
+
+
+def test_persistent_path_bad_slot():
+    wl = wl_of("p_badslot", 4, 8, 128, 128, 4, 40, 1, 40, 1, seed=21, slot_mode="permutation")
+    g = GpuRun(wl)
+    slots = g.slots_np.copy()
+    slots[17] = 40  # outside the 40-slot pool
+    g.slots = torch.from_numpy(slots).cuda()
+    state0, conv0 = g.state.clone(), g.conv.clone()
+    x = g.inputs(0)
+    shape = (40, 1, 8, 128)
+    out = torch.full(shape, 3.0, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.full(shape, 3.0, device="cuda")
+    gdn.gdn_decode_step(g.cfg, x["qkv"], x["a"], x["b"], x["z"], g.conv_w, g.A_log, g.dt_bias, g.norm_w,
+                        g.conv, g.state, g.slots, out, out32, g.err)
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == gdn.GDN_DEVICE_ERR_SLOT_RANGE
+    assert torch.all(out32[17] == 3.0)
+    skipped = int(g.slots_np[17])  # the slot sequence 17 would have used: nobody touched it
+    assert torch.equal(g.state[skipped], state0[skipped]) and torch.equal(g.conv[skipped], conv0[skipped])
+    rows = [0, 16, 18, 39]
+    o = OracleRun(wl, rows)
+    r = o.step(0)
+    compare_out(out, out32, r["out"], rows, "persistent rows beside a bad slot")
+    compare_state(g.state, o.state, o.slot_ids, "persistent rows beside a bad slot")
+
+
 def _stage_problem(seed=5, Hk=2, Hv=4, dk=64, dv=128, W=4, B=3, T=3, P=4):
     wl = wl_of("stages", Hk, Hv, dk, dv, W, B, T, P, 1, seed)
     return wl, GpuRun(wl), synth.step_inputs(wl, 0)

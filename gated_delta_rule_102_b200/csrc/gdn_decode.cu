@@ -182,10 +182,6 @@ decode_fused_kernel(const DecodeArgs p) {
     }
 }
 
-// Bound on mbarrier polls before a CTA gives up on its state tile (each poll may
-// suspend for a short hardware-defined time, so this is well above a second).
-constexpr uint32_t kTmaWaitPolls = 1u << 24;
-
 template <int DK, int DVS>
 struct TmaSmem {
     using F = FusedSmem<DK, DVS>;
@@ -289,7 +285,7 @@ decode_fused_tma_kernel(const DecodeArgs p) {
         __syncthreads();
     }
     qk_norms<DK>(qk, sc, T, p.sh.l2_eps, p.sh.q_scale, Geo::NW);
-    const bool ready = mbar_wait_bounded(bar, 0, kTmaWaitPolls);
+    const bool ready = mbar_wait_bounded(bar, 0);
     const bool timed_out = __syncthreads_or(!ready);
     if (!timed_out) {
         const int cg = tid % Geo::TPR, rp = tid / Geo::TPR;
@@ -320,7 +316,7 @@ decode_fused_tma_kernel(const DecodeArgs p) {
         __syncthreads();
     }
     if (timed_out) {  // the tile never arrived: wait (bounded) for the copies, write nothing
-        mbar_wait_bounded(bar, 0, kTmaWaitPolls);
+        mbar_wait_bounded(bar, 0);
         return;
     }
     const float inv_dv = 1.0f / (float)dv;
@@ -417,7 +413,7 @@ int decode_column_splits(int B, int Hv, int G, int dv) {
 }
 
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream) {
-    if (a.T == 1) {  // many groups: the persistent pipelined kernel
+    if (persistent_supported(a)) {  // single token, many groups: the persistent pipelined kernel
         int cap = 0;
         cudaError_t e = persistent_capacity(a, &cap);
         if (e != cudaSuccess) return e;

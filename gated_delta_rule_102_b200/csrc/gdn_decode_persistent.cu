@@ -1,25 +1,33 @@
-// Persistent, software-pipelined form of the fused GDN decode step for single-token
+// Persistent, warp-specialised form of the fused GDN decode step for single-token
 // launches over many sequences (steps 3 to 8 and the SiLU(z) gate of steps 9+10+11
 // on the page "spark_model/forward/qwen3_5/linear_attention.rs").
 //
-// A cluster of G = Hv/Hk CTAs (one per v-head sharing a k-head) stays resident and
-// walks (sequence, k-head) groups cid, cid + ncl, cid + 2 ncl, ... Each CTA owns one
-// v-head of the group: its whole dk x dv fp32 state tile, which is contiguous in the
-// pool. Tiles stream through a ring of NSTAGE shared-memory stages filled by TMA bulk
-// copies, so while unit u is computed the tiles of units u+1 .. u+NSTAGE-1 are in
-// flight and the updated tile of unit u-1 drains from registers: the SM keeps HBM
-// busy instead of alternating between load, compute and store phases.
+// Work. A cluster of G = Hv/Hk CTAs (one per v-head sharing a k-head) stays resident
+// and walks (sequence, k-head) groups cid, cid + ncl, cid + 2 ncl, ... Each CTA owns
+// one v-head of every group it visits: the whole dk x dv fp32 state tile of that
+// head, contiguous in the pool.
 //
-// Conv ownership: the group's q and k channels are split over the G CTAs and each
-// CTA owns its v-head's v channels, so every channel's history is read and rolled
-// by exactly one CTA. The raw q/k values travel to every CTA of the cluster with
-// st.async into distributed shared memory, completed on the receiver's mbarrier
-// (no release fence that would wait for this CTA's outstanding state stores). The
-// conv inputs of unit u+1 are loaded into registers while unit u is computed.
+// Roles inside a CTA.
+//  * Warp 0, the producer, runs ahead of the math. For unit v it waits until stage
+//    v % NSTAGE is free, starts the TMA bulk copies of the state tile and the z row
+//    into it, convolves this CTA's channels (its share of the k-head's q/k channels
+//    plus its v-head's v channels) from inputs it loaded one unit earlier, sends the
+//    raw q/k share to every CTA of the cluster with st.async (completed on the
+//    receiver's mbarrier), rolls the conv history, waits for the other shares, and
+//    publishes the q/k norms, k.q, the gates and the slot for the stage.
+//  * Warps 1..8 form teams that take units in turn. A team owns a unit: each warp
+//    holds a band of columns (the columns of S are independent under the update),
+//    reads the tile from shared memory twice (S^T k and S^T q, then the update),
+//    reduces over dk with two shuffle stages, streams the new rows to HBM, and then
+//    the team applies the RMSNorm, the norm weight and SiLU(z).
+// Every channel's conv history is therefore read and rolled by exactly one CTA, the
+// state is read once and written once, and HBM sees a steady stream of TMA loads and
+// row stores instead of alternating load, compute and store phases.
 //
-// Every wait is an mbarrier poll with a bound; on expiry the CTA sets the timeout
-// bit of the error flag, stops issuing copies, waits (bounded) for the copies it
-// has in flight and leaves through the final cluster barrier.
+// Every wait is an mbarrier poll with a bound. When one expires the CTA sets the
+// timeout bit of the error flag, all roles leave their loops, the producer waits
+// (bounded) for its copies in flight, and the CTA leaves through the final cluster
+// barrier.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -29,266 +37,351 @@
 namespace gdn {
 namespace {
 
-constexpr uint32_t kPollLimit = 1u << 24;
 constexpr int kTileChunk = 16384;  // bytes per bulk copy of a state tile
+constexpr int kMaxConvWidthPersistent = 4;
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+__host__ __device__ constexpr int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
 
-template <int DK, int DV>
-struct PLayout {
-    using Geo = Tile<DK, DV>;
-    static constexpr int NT = Geo::NT;
-    static constexpr int TILE_BYTES = DK * DV * 4;
-    static constexpr int NSTAGE = TILE_BYTES * 4 <= 196608 ? 4 : (TILE_BYTES * 3 <= 196608 ? 3 : 2);
-    // most channels one CTA convolves: all 2*DK q/k channels (G = 1) plus its DV v channels
-    static constexpr int MAXC = (2 * DK + DV + NT - 1) / NT;
-    static constexpr int TILES = 0;
-    static constexpr int ZB = TILES + NSTAGE * TILE_BYTES;       // [NSTAGE][DV] bf16
-    static constexpr int QK = ZB + round_up(NSTAGE * DV * 2, 16);  // [2][2*DK] f32, raw q then raw k
-    static constexpr int VS = QK + 2 * 2 * DK * 4;                // [2][DV] f32
-    static constexpr int OS = VS + 2 * DV * 4;                    // [DV] f32
-    static constexpr int RED = OS + DV * 4;                       // [2][NW][2][DV] f32
-    static constexpr int SC = RED + 2 * Geo::NW * 2 * DV * 4;     // [2] TokenScalars
-    static constexpr int PART = SC + 48;                          // [NW] f32
-    static constexpr int BARS = round_up(PART + Geo::NW * 4, 16);  // [NSTAGE] tile bars, [2] q/k bars
-    static constexpr int TOTAL = BARS + (NSTAGE + 2) * 8;
-    static_assert(TOTAL <= 232448, "shared memory");
+struct StageInfo {  // what the producer publishes for a staged unit
+    float alpha, beta, nq, nk, kq;
+    int slot;  // -1: the unit's slot is out of range
+    int pad[2];
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(PLayout<DK, DV>::NT, 1)
-decode_persistent_kernel(const DecodeArgs p, const int ncl) {
-    using Lay = PLayout<DK, DV>;
-    using Geo = Tile<DK, DV>;
-    constexpr int NT = Lay::NT, NSTAGE = Lay::NSTAGE, MAXC = Lay::MAXC, WM = kMaxConvWidth;
+struct WS {
+    static constexpr int CONSUMER_WARPS = 8;
+    static constexpr int NT = 32 * (1 + CONSUMER_WARPS);
+    static constexpr int TEAM_WARPS = DV >= 128 ? 4 : (DV >= 64 ? 2 : 1);
+    static constexpr int NTEAMS = CONSUMER_WARPS / TEAM_WARPS;
+    static constexpr int CPW = DV / TEAM_WARPS;  // columns per consumer warp (32, or 16 when dv = 16)
+    static constexpr int CG = CPW / 4;           // float4 column groups per warp
+    static constexpr int RG = 32 / CG;           // row groups per warp
+    static constexpr int RPL = DK / RG;          // rows per lane
+    static constexpr int TILE_BYTES = DK * DV * 4;
+    static constexpr int NSTAGE = clampi(196608 / TILE_BYTES, 2, 8);
+    static constexpr int QB = NSTAGE + 1;        // q/k buffers: one more than stages (see the producer)
+    static constexpr int MAXCH = (2 * DK + DV + 31) / 32;  // conv channels per producer lane
+    // shared-memory byte offsets
+    static constexpr int TILES = 0;
+    static constexpr int ZB = TILES + NSTAGE * TILE_BYTES;          // [NSTAGE][DV] bf16
+    static constexpr int VS = ZB + round_up(NSTAGE * DV * 2, 16);    // [NSTAGE][DV] f32
+    static constexpr int SI = VS + NSTAGE * DV * 4;                  // [NSTAGE] StageInfo
+    static constexpr int QK = SI + NSTAGE * (int)sizeof(StageInfo);  // [QB][2*DK] f32
+    static constexpr int PART = QK + QB * 2 * DK * 4;                // [NTEAMS][2][TEAM_WARPS] f32
+    static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
+    static constexpr int BARS = FLAG + 16;                           // full, empty [NSTAGE]; qk [QB]
+    static constexpr int TOTAL = BARS + (2 * NSTAGE + QB) * 8;
+    static_assert(CG >= 1 && RG >= 1 && RPL >= 1 && RG * CG == 32, "consumer geometry");
+    static_assert(TOTAL <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(WS<DK, DV>::NT, 1)
+decode_ws_kernel(const DecodeArgs p, const int ncl) {
+    using L = WS<DK, DV>;
+    constexpr int NSTAGE = L::NSTAGE, QB = L::QB, WM = kMaxConvWidthPersistent;
     extern __shared__ __align__(128) unsigned char smem[];
-    float* tiles = reinterpret_cast<float*>(smem + Lay::TILES);
-    uint16_t* zb = reinterpret_cast<uint16_t*>(smem + Lay::ZB);
-    float* qkb = reinterpret_cast<float*>(smem + Lay::QK);
-    float* vsb = reinterpret_cast<float*>(smem + Lay::VS);
-    float* os = reinterpret_cast<float*>(smem + Lay::OS);
-    float* red = reinterpret_cast<float*>(smem + Lay::RED);
-    TokenScalars* scb = reinterpret_cast<TokenScalars*>(smem + Lay::SC);
-    float* part = reinterpret_cast<float*>(smem + Lay::PART);
-    uint64_t* tbar = reinterpret_cast<uint64_t*>(smem + Lay::BARS);
-    uint64_t* qbar = tbar + NSTAGE;
+    float* tiles = reinterpret_cast<float*>(smem + L::TILES);
+    uint16_t* zb = reinterpret_cast<uint16_t*>(smem + L::ZB);
+    float* vsb = reinterpret_cast<float*>(smem + L::VS);
+    StageInfo* si = reinterpret_cast<StageInfo*>(smem + L::SI);
+    float* qkb = reinterpret_cast<float*>(smem + L::QK);
+    float* part = reinterpret_cast<float*>(smem + L::PART);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::FLAG);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
+    uint64_t* empty = full + NSTAGE;
+    uint64_t* qkbar = empty + NSTAGE;
 
     const int Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk, C = p.sh.C, W = p.sh.W;
     const int rank = (int)cluster_ctarank(), cid = blockIdx.x / G;
     const int ngroups = p.B * Hk;
     const int n = cid < ngroups ? (ngroups - cid + ncl - 1) / ncl : 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int qk_lo = (rank * 2 * DK) / G, qk_hi = ((rank + 1) * 2 * DK) / G, nqk = qk_hi - qk_lo;
-    const int nch = nqk + DV;
 
     if (tid == 0) {
-        for (int s = 0; s < NSTAGE; ++s) mbar_init(tbar + s, 1);
-        mbar_init(qbar + 0, 1);
-        mbar_init(qbar + 1, 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(full + s, 2);                // the producer's copy arrival and its publish arrival
+            mbar_init(empty + s, L::TEAM_WARPS);   // one arrival per warp of the consuming team
+        }
+        for (int q = 0; q < QB; ++q) mbar_init(qkbar + q, 1);
+        *abort_flag = 0;
         mbar_init_fence();
     }
     __syncthreads();
     cluster_arrive_relaxed();  // every CTA of the cluster runs before any st.async targets it
     cluster_wait_acquire();
 
+    auto fail = [&]() {
+        if (lane == 0) {
+            *abort_flag = 1;
+            if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_TIMEOUT_BIT);
+        }
+    };
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return mbar_wait_deadline(bar, parity, kWaitTimeoutNs, [&] { return *abort_flag != 0; });
+    };
     auto group_seq = [&](int u) { return (cid + u * ncl) / Hk; };
     auto group_hk = [&](int u) { return (cid + u * ncl) % Hk; };
     auto slot_ok = [&](int s) { return s >= 0 && s < p.P; };
-    auto slot_of = [&](int u) { return u < n ? __ldg(p.slots + group_seq(u)) : -1; };
 
-    // thread 0: stage unit u's state tile and its z row into stage u % NSTAGE
-    auto issue_tile = [&](int u) {
-        const int seq = group_seq(u), h = group_hk(u) * G + rank;
-        const int slot = __ldg(p.slots + seq);
-        uint64_t* bar = tbar + (u % NSTAGE);
-        if (!slot_ok(slot)) {
-            mbar_arrive(bar);
-            return;
-        }
-        mbar_arrive_expect_tx(bar, Lay::TILE_BYTES + DV * 2);
-        const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h) * (size_t)(DK * DV));
-        char* dst = reinterpret_cast<char*>(tiles) + (size_t)(u % NSTAGE) * Lay::TILE_BYTES;
-        for (int c = 0; c < Lay::TILE_BYTES; c += kTileChunk)
-            tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, Lay::TILE_BYTES - c), bar);
-        tma_load_1d(zb + (u % NSTAGE) * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, bar);
-    };
-
-    // conv inputs of one unit, one channel per (thread, i)
-    uint32_t ph[MAXC][WM - 1], px[MAXC], pw[MAXC][WM];
-    uint16_t pa = 0, pb = 0;
-    float pA = 0.f, pdt = 0.f;
-    auto channel_of = [&](int c, int hk, int h) {
-        if (c < nqk) {
-            const int j = qk_lo + c;
-            return j < DK ? hk * DK + j : Hk * DK + hk * DK + (j - DK);
-        }
-        return 2 * Hk * DK + h * DV + (c - nqk);
-    };
-    auto prefetch = [&](int u, int slot) {
-        const int seq = group_seq(u), hk = group_hk(u), h = hk * G + rank;
-        const uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
-#pragma unroll
-        for (int i = 0; i < MAXC; ++i) {
-            const int c = tid + i * NT;
-            if (c < nch) {
-                const int ch = channel_of(c, hk, h);
-#pragma unroll
-                for (int r = 0; r < WM - 1; ++r) ph[i][r] = r < W - 1 ? hist[(size_t)r * C + ch] : 0u;
-                px[i] = p.qkv[(size_t)seq * C + ch];
-#pragma unroll
-                for (int j = 0; j < WM; ++j) pw[i][j] = j < W ? p.conv_w[(size_t)ch * W + j] : 0u;
+    if (warp == 0) {
+        // ============================== producer ==============================
+        const int qk_lo = (rank * 2 * DK) / G, qk_hi = ((rank + 1) * 2 * DK) / G, nqk = qk_hi - qk_lo;
+        const int nch = nqk + DV;
+        auto slot_of = [&](int u) { return u < n ? __ldg(p.slots + group_seq(u)) : -1; };
+        auto channel_of = [&](int c, int hk, int h) {
+            if (c < nqk) {
+                const int j = qk_lo + c;
+                return j < DK ? hk * DK + j : Hk * DK + hk * DK + (j - DK);
             }
-        }
-        if (tid == 0) {
-            pa = p.a[(size_t)seq * Hv + h];
-            pb = p.b[(size_t)seq * Hv + h];
-            pA = p.A_log[h];
-            pdt = p.dt_bias[h];
-        }
-    };
-    // step 3 for unit u from the prefetched inputs: q/k shares to every cluster CTA,
-    // v to this CTA, the rolled history back to the pool
-    auto conv_finish = [&](int u, int slot) {
-        const int hk = group_hk(u), h = hk * G + rank, buf = u & 1;
-        uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
+            return 2 * Hk * DK + h * DV + (c - nqk);
+        };
+        uint32_t ph[L::MAXCH][WM - 1], px[L::MAXCH], pw[L::MAXCH][WM];
+        uint16_t pa = 0, pb = 0;
+        float pA = 0.f, pdt = 0.f;
+        auto prefetch = [&](int u, int slot) {
+            const int seq = group_seq(u), hk = group_hk(u), h = hk * G + rank;
+            const uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
 #pragma unroll
-        for (int i = 0; i < MAXC; ++i) {
-            const int c = tid + i * NT;
-            if (c < nch) {
-                const int ch = channel_of(c, hk, h);
-                float acc = 0.f;
+            for (int i = 0; i < L::MAXCH; ++i) {
+                const int c = lane + 32 * i;
+                if (c < nch) {
+                    const int ch = channel_of(c, hk, h);
 #pragma unroll
-                for (int j = 0; j < WM; ++j) {
-                    if (j < W) {
-                        const uint32_t xb = j < W - 1 ? ph[i][j] : px[i];
-                        acc = fmaf(bf16_bits_to_float(pw[i][j]), bf16_bits_to_float(xb), acc);
+                    for (int r = 0; r < WM - 1; ++r) ph[i][r] = r < W - 1 ? hist[(size_t)r * C + ch] : 0u;
+                    px[i] = p.qkv[(size_t)seq * C + ch];
+#pragma unroll
+                    for (int j = 0; j < WM; ++j) pw[i][j] = j < W ? p.conv_w[(size_t)ch * W + j] : 0u;
+                }
+            }
+            if (lane == 0) {
+                pa = p.a[(size_t)seq * Hv + h];
+                pb = p.b[(size_t)seq * Hv + h];
+                pA = p.A_log[h];
+                pdt = p.dt_bias[h];
+            }
+        };
+        int sl0 = slot_of(0), sl1 = slot_of(1), sl2 = slot_of(2);
+        if (n > 0 && slot_ok(sl0)) prefetch(0, sl0);
+        for (int v = 0; v < n; ++v) {
+            const int s = v % NSTAGE, q = v % QB;
+            const int seq = group_seq(v), hk = group_hk(v), h = hk * G + rank;
+            const bool valid = slot_ok(sl0);
+            if (v >= NSTAGE && !wait(empty + s, ((v / NSTAGE) - 1) & 1)) {
+                fail();
+                break;
+            }
+            // ---- the state tile and z row of unit v into stage s
+            if (lane == 0) {
+                if (valid) mbar_arrive_expect_tx(full + s, L::TILE_BYTES + DV * 2);
+                else mbar_arrive(full + s);
+            }
+            __syncwarp();
+            if (valid) {
+                const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)sl0 * Hv + h) * (size_t)(DK * DV));
+                char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
+                constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
+                if (lane < nchunk) {
+                    const int c = lane * kTileChunk;
+                    tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
+                } else if (lane == nchunk) {
+                    tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
+                }
+            }
+            // ---- step 3 for this CTA's channels of unit v
+            const uint16_t ga = pa, gb = pb;
+            const float gA = pA, gdt = pdt;
+            if (valid) {
+                uint16_t* hist = p.conv_pool + (size_t)sl0 * (W - 1) * C;
+                const uint32_t q_loc = smem_addr(qkb + q * 2 * DK + qk_lo), bar_loc = smem_addr(qkbar + q);
+#pragma unroll
+                for (int i = 0; i < L::MAXCH; ++i) {
+                    const int c = lane + 32 * i;
+                    if (c < nch) {
+                        const int ch = channel_of(c, hk, h);
+                        float acc = 0.f;
+#pragma unroll
+                        for (int j = 0; j < WM; ++j) {
+                            if (j < W) {
+                                const uint32_t xb = j < W - 1 ? ph[i][j < WM - 1 ? j : 0] : px[i];
+                                acc = fmaf(bf16_bits_to_float(pw[i][j]), bf16_bits_to_float(xb), acc);
+                            }
+                        }
+                        const float sv = silu(acc);
+                        if (c < nqk) {
+                            for (int r = 0; r < G; ++r)
+                                st_async_f32(cluster_map_u32(q_loc + 4 * c, r), sv, cluster_map_u32(bar_loc, r));
+                        } else {
+                            vsb[s * DV + (c - nqk)] = sv;
+                        }
+#pragma unroll
+                        for (int r = 0; r < WM - 1; ++r) {
+                            if (r < W - 1) {
+                                uint32_t nb = px[i];
+                                if (r + 1 < W - 1) nb = ph[i][r + 1 < WM - 1 ? r + 1 : 0];
+                                hist[(size_t)r * C + ch] = (uint16_t)nb;
+                            }
+                        }
                     }
                 }
-                const float s = silu(acc);
-                if (c < nqk) {
-                    const uint32_t a_loc = smem_addr(qkb + buf * 2 * DK + qk_lo + c);
-                    const uint32_t b_loc = smem_addr(qbar + buf);
-                    for (int r = 0; r < G; ++r) st_async_f32(cluster_map_u32(a_loc, r), s, cluster_map_u32(b_loc, r));
-                } else {
-                    vsb[buf * DV + (c - nqk)] = s;
+            }
+            // ---- inputs of unit v+1 (they land while this unit's shares are exchanged)
+            const int sl3 = slot_of(v + 3);
+            if (v + 1 < n && slot_ok(sl1)) prefetch(v + 1, sl1);
+            // ---- all q/k shares of unit v: norms, k.q, gates
+            if (lane == 0) {
+                if (valid) mbar_arrive_expect_tx(qkbar + q, 2 * DK * 4);
+                else mbar_arrive(qkbar + q);
+            }
+            if (!wait(qkbar + q, (v / QB) & 1)) {
+                fail();
+                break;
+            }
+            if (valid) {
+                const float* qr = qkb + q * 2 * DK;
+                float sq = 0.f, sk = 0.f, dot = 0.f;
+                for (int i = lane; i < DK; i += 32) {
+                    const float a = qr[i], b = qr[DK + i];
+                    sq = fmaf(a, a, sq);
+                    sk = fmaf(b, b, sk);
+                    dot = fmaf(a, b, dot);
                 }
 #pragma unroll
-                for (int r = 0; r < WM - 1; ++r) {
-                    if (r < W - 1) {
-                        uint32_t nb = px[i];
-                        if (r + 1 < WM - 1 && r + 1 < W - 1) nb = ph[i][r + 1 < WM - 1 ? r + 1 : 0];
-                        hist[(size_t)r * C + ch] = (uint16_t)nb;
-                    }
+                for (int off = 16; off > 0; off >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    dot += __shfl_xor_sync(0xffffffffu, dot, off);
                 }
+                if (lane == 0) {
+                    StageInfo& st = si[s];
+                    st.nq = rsqrtf(sq + p.sh.l2_eps) * p.sh.q_scale;
+                    st.nk = rsqrtf(sk + p.sh.l2_eps);
+                    st.kq = dot * st.nq * st.nk;
+                    gate_and_beta(ga, gb, gA, gdt, st.alpha, st.beta);
+                    st.slot = sl0;
+                }
+            } else if (lane == 0) {
+                si[s].slot = -1;
+                if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full + s);
+            sl0 = sl1;
+            sl1 = sl2;
+            sl2 = sl3;
         }
-    };
-
-    int issued = 0;
-    if (tid == 0)
-        for (; issued < NSTAGE && issued < n; ++issued) issue_tile(issued);
-    int slot_c = slot_of(0), slot_n1 = slot_of(1);
-    if (n > 0 && slot_ok(slot_c)) {
-        prefetch(0, slot_c);
-        conv_finish(0, slot_c);
-    } else if (n > 0 && tid == 0 && p.err_flag) {
-        atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
-    }
-    uint16_t ga = pa, gb = pb;
-    float gA = pA, gdt = pdt;
-
-    bool failed = false;
-    int consumed = 0;
-    for (int u = 0; u < n; ++u) {
-        const bool valid = slot_ok(slot_c);
-        const int slot_n2 = slot_of(u + 2);
-        if (u + 1 < n && slot_ok(slot_n1)) prefetch(u + 1, slot_n1);
-
-        // ---- q/k of unit u have arrived from every cluster CTA: norms and gates
-        const int buf = u & 1;
-        if (tid == 0) {
-            if (valid) mbar_arrive_expect_tx(qbar + buf, 2 * DK * 4);
-            else mbar_arrive(qbar + buf);
+        if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
+            for (int i = 0; i < 1024; ++i) __nanosleep(64);
         }
-        bool ok = mbar_wait_bounded(qbar + buf, (u >> 1) & 1, kPollLimit);
-        if (valid) {
-            if (warp == 0) qk_norms<DK>(qkb + buf * 2 * DK, scb + buf, 1, p.sh.l2_eps, p.sh.q_scale, 1);
-            if (tid == 0) gate_and_beta(ga, gb, gA, gdt, scb[buf].alpha, scb[buf].beta);
-        }
-        // ---- the state tile of unit u
-        ok = mbar_wait_bounded(tbar + (u % NSTAGE), (u / NSTAGE) & 1, kPollLimit) && ok;
-        ++consumed;
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        const int seq = group_seq(u), h = group_hk(u) * G + rank;
-        if (valid) {
-            const int cg = tid % Geo::TPR, rp = tid / Geo::TPR;
-            float4* Sg = reinterpret_cast<float4*>(p.state_pool + ((size_t)slot_c * Hv + h) * (size_t)(DK * DV)) +
-                         (size_t)(rp * Geo::RPT) * (DV / 4) + cg;
-            delta_rule_smem<DK, DV>(tiles + (size_t)(u % NSTAGE) * (DK * DV), qkb + buf * 2 * DK, vsb + buf * DV,
-                                    scb + buf, os, red, 1, Sg, DV / 4);
-        } else if (tid == 0 && p.err_flag) {
-            atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
-        }
-        __syncthreads();
-        // ---- step 8: RMSNorm over the head, norm weight, SiLU(z) gate
-        if (valid) {
-            float ss = 0.f;
-            for (int j = tid; j < DV; j += NT) ss = fmaf(os[j], os[j], ss);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            if (lane == 0) part[warp] = ss;
-            __syncthreads();
-            float tot = 0.f;
-#pragma unroll
-            for (int w = 0; w < Geo::NW; ++w) tot += part[w];
-            const float inv = rsqrtf(tot / (float)DV + p.sh.rms_eps);
-            for (int j = tid; j < DV; j += NT) {
-                const float zz = bf16_bits_to_float(zb[(u % NSTAGE) * DV + j]);
-                const float y = os[j] * inv * bf16_bits_to_float(p.norm_w[j]) * silu(zz);
-                const size_t oi = ((size_t)seq * Hv + h) * DV + j;
-                p.out[oi] = float_to_bf16_bits(y);
-                if (p.out_f32) p.out_f32[oi] = y;
+    } else {
+        // ============================== consumers ==============================
+        const int cw = warp - 1, team = cw / L::TEAM_WARPS, wt = cw - team * L::TEAM_WARPS;
+        const int rg = lane / L::CG, cg = lane - rg * L::CG;
+        const int col = wt * L::CPW + 4 * cg;
+        int parity_part = 0;
+        for (int u = team; u < n; u += L::NTEAMS) {
+            const int s = u % NSTAGE, q = u % QB;
+            if (!wait(full + s, (u / NSTAGE) & 1)) {
+                fail();
+                break;
             }
+            const StageInfo st = si[s];
+            if (st.slot >= 0) {
+                const int seq = group_seq(u), h = group_hk(u) * G + rank;
+                const float4* tl = reinterpret_cast<const float4*>(tiles + (size_t)s * (DK * DV)) + col / 4;
+                const float* qr = qkb + q * 2 * DK;
+                const float* kr = qr + DK;
+                float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
+#pragma unroll 8
+                for (int i = 0; i < L::RPL; ++i) {
+                    const int row = rg + L::RG * i;
+                    const float4 x = tl[(size_t)row * (DV / 4)];
+                    const float ki = kr[row], qi = qr[row];
+                    mk.x = fmaf(x.x, ki, mk.x); mk.y = fmaf(x.y, ki, mk.y);
+                    mk.z = fmaf(x.z, ki, mk.z); mk.w = fmaf(x.w, ki, mk.w);
+                    mq.x = fmaf(x.x, qi, mq.x); mq.y = fmaf(x.y, qi, mq.y);
+                    mq.z = fmaf(x.z, qi, mq.z); mq.w = fmaf(x.w, qi, mq.w);
+                }
+#pragma unroll
+                for (int off = L::CG; off < 32; off <<= 1) {
+                    mk.x += __shfl_xor_sync(0xffffffffu, mk.x, off); mk.y += __shfl_xor_sync(0xffffffffu, mk.y, off);
+                    mk.z += __shfl_xor_sync(0xffffffffu, mk.z, off); mk.w += __shfl_xor_sync(0xffffffffu, mk.w, off);
+                    mq.x += __shfl_xor_sync(0xffffffffu, mq.x, off); mq.y += __shfl_xor_sync(0xffffffffu, mq.y, off);
+                    mq.z += __shfl_xor_sync(0xffffffffu, mq.z, off); mq.w += __shfl_xor_sync(0xffffffffu, mq.w, off);
+                }
+                const float4 vv = *reinterpret_cast<const float4*>(vsb + s * DV + col);
+                const float am = st.alpha * st.nk, aq = st.alpha * st.nq;
+                float4 d, o;
+                d.x = st.beta * fmaf(-am, mk.x, vv.x); d.y = st.beta * fmaf(-am, mk.y, vv.y);
+                d.z = st.beta * fmaf(-am, mk.z, vv.z); d.w = st.beta * fmaf(-am, mk.w, vv.w);
+                o.x = fmaf(aq, mq.x, d.x * st.kq); o.y = fmaf(aq, mq.y, d.y * st.kq);
+                o.z = fmaf(aq, mq.z, d.z * st.kq); o.w = fmaf(aq, mq.w, d.w * st.kq);
+                const float4 dn = make_float4(d.x * st.nk, d.y * st.nk, d.z * st.nk, d.w * st.nk);
+                float4* Sg = reinterpret_cast<float4*>(p.state_pool + ((size_t)st.slot * Hv + h) * (size_t)(DK * DV) +
+                                                       col);
+#pragma unroll 8
+                for (int i = 0; i < L::RPL; ++i) {
+                    const int row = rg + L::RG * i;
+                    float4 x = tl[(size_t)row * (DV / 4)];
+                    const float ki = kr[row];
+                    x.x = fmaf(st.alpha, x.x, ki * dn.x); x.y = fmaf(st.alpha, x.y, ki * dn.y);
+                    x.z = fmaf(st.alpha, x.z, ki * dn.z); x.w = fmaf(st.alpha, x.w, ki * dn.w);
+                    __stcs(Sg + (size_t)row * (DV / 4), x);
+                }
+                // ---- step 8 over the whole head: the team's warps pool their sums of o^2
+                float ss = rg == 0 ? o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w : 0.f;
+#pragma unroll
+                for (int off = 1; off < L::CG; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                float* pt = part + (team * 2 + parity_part) * L::TEAM_WARPS;
+                if (lane == 0) pt[wt] = ss;
+                if (L::TEAM_WARPS > 1) named_barrier(1 + team, 32 * L::TEAM_WARPS);
+                else __syncwarp();
+                float tot = 0.f;
+#pragma unroll
+                for (int w = 0; w < L::TEAM_WARPS; ++w) tot += pt[w];
+                if (rg == 0) {
+                    const float inv = rsqrtf(tot / (float)DV + p.sh.rms_eps);
+                    const uint2 zz = *reinterpret_cast<const uint2*>(zb + s * DV + col);
+                    const uint2 ww = *reinterpret_cast<const uint2*>(p.norm_w + col);
+                    const float y0 = o.x * inv * bf16_bits_to_float(ww.x & 0xffffu) * silu(bf16_bits_to_float(zz.x & 0xffffu));
+                    const float y1 = o.y * inv * bf16_bits_to_float(ww.x >> 16) * silu(bf16_bits_to_float(zz.x >> 16));
+                    const float y2 = o.z * inv * bf16_bits_to_float(ww.y & 0xffffu) * silu(bf16_bits_to_float(zz.y & 0xffffu));
+                    const float y3 = o.w * inv * bf16_bits_to_float(ww.y >> 16) * silu(bf16_bits_to_float(zz.y >> 16));
+                    const size_t oi = ((size_t)seq * Hv + h) * DV + col;
+                    uint2 packed;
+                    packed.x = (uint32_t)float_to_bf16_bits(y0) | ((uint32_t)float_to_bf16_bits(y1) << 16);
+                    packed.y = (uint32_t)float_to_bf16_bits(y2) | ((uint32_t)float_to_bf16_bits(y3) << 16);
+                    *reinterpret_cast<uint2*>(p.out + oi) = packed;
+                    if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + oi) = make_float4(y0, y1, y2, y3);
+                }
+                parity_part ^= 1;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);
         }
-        __syncthreads();  // stage u % NSTAGE and its z row are free again
-        if (tid == 0 && issued < n) {
-            fence_proxy_async_smem();
-            issue_tile(issued++);
-        }
-        if (u + 1 < n && slot_ok(slot_n1)) conv_finish(u + 1, slot_n1);
-        ga = pa;  // the prefetched inputs of unit u+1 have long arrived by now
-        gb = pb;
-        gA = pA;
-        gdt = pdt;
-        slot_c = slot_n1;
-        slot_n1 = slot_n2;
     }
-    if (failed) {
-        if (tid == 0) {
-            if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_TIMEOUT_BIT);
-            for (int u = consumed; u < issued; ++u) mbar_wait_bounded(tbar + (u % NSTAGE), (u / NSTAGE) & 1, kPollLimit);
-        }
-        __syncthreads();
-    }
+    __syncthreads();
     cluster_arrive_release();  // no CTA leaves while a peer may still send to it
     cluster_wait_acquire();
 }
 
 template <int DK, int DV>
-cudaError_t launch_persistent_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap_out) {
-    using Lay = PLayout<DK, DV>;
-    auto kern = decode_persistent_kernel<DK, DV>;
-    // co-resident cluster capacity, queried once per (device, cluster size)
-    static int cap_cache[16][9];
+cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap_out) {
+    using L = WS<DK, DV>;
+    auto kern = decode_ws_kernel<DK, DV>;
+    static int cap_cache[16][9];  // co-resident clusters per (device, cluster size), queried once
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(Lay::NT);
-    cfg.dynamicSmemBytes = Lay::TOTAL;
+    cfg.blockDim = dim3(L::NT);
+    cfg.dynamicSmemBytes = L::TOTAL;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -297,9 +390,9 @@ cudaError_t launch_persistent_tile(const DecodeArgs& a, int G, cudaStream_t stre
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int& cap = cap_cache[dev & 15][G & 7 ? G : 8];
+    int& cap = cap_cache[dev & 15][G];
     if (cap <= 0) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::TOTAL);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
         if (e != cudaSuccess) return e;
         cfg.gridDim = dim3((unsigned)G);
         int maxc = 0;
@@ -317,35 +410,40 @@ cudaError_t launch_persistent_tile(const DecodeArgs& a, int G, cudaStream_t stre
 }
 
 template <int DK>
-cudaError_t persistent_dispatch(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap) {
+cudaError_t ws_dispatch(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap) {
     switch (a.sh.dv) {
-        case 16: return launch_persistent_tile<DK, 16>(a, G, stream, query_only, cap);
-        case 32: return launch_persistent_tile<DK, 32>(a, G, stream, query_only, cap);
-        case 64: return launch_persistent_tile<DK, 64>(a, G, stream, query_only, cap);
-        case 128: return launch_persistent_tile<DK, 128>(a, G, stream, query_only, cap);
+        case 16: return launch_ws_tile<DK, 16>(a, G, stream, query_only, cap);
+        case 32: return launch_ws_tile<DK, 32>(a, G, stream, query_only, cap);
+        case 64: return launch_ws_tile<DK, 64>(a, G, stream, query_only, cap);
+        case 128: return launch_ws_tile<DK, 128>(a, G, stream, query_only, cap);
     }
     return cudaErrorInvalidValue;
 }
 
-cudaError_t persistent_call(const DecodeArgs& a, cudaStream_t stream, bool query_only, int* cap) {
+cudaError_t ws_call(const DecodeArgs& a, cudaStream_t stream, bool query_only, int* cap) {
     const int G = a.sh.Hv / a.sh.Hk;
+    if (a.T != 1 || a.sh.W > kMaxConvWidthPersistent || G > 8) return cudaErrorInvalidValue;
     switch (a.sh.dk) {
-        case 16: return persistent_dispatch<16>(a, G, stream, query_only, cap);
-        case 32: return persistent_dispatch<32>(a, G, stream, query_only, cap);
-        case 64: return persistent_dispatch<64>(a, G, stream, query_only, cap);
-        case 128: return persistent_dispatch<128>(a, G, stream, query_only, cap);
+        case 16: return ws_dispatch<16>(a, G, stream, query_only, cap);
+        case 32: return ws_dispatch<32>(a, G, stream, query_only, cap);
+        case 64: return ws_dispatch<64>(a, G, stream, query_only, cap);
+        case 128: return ws_dispatch<128>(a, G, stream, query_only, cap);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
+bool persistent_supported(const DecodeArgs& a) {
+    return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && a.sh.Hv / a.sh.Hk <= 8;
+}
+
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters) {
-    return persistent_call(a, nullptr, true, max_clusters);
+    return ws_call(a, nullptr, true, max_clusters);
 }
 
 cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream) {
-    return persistent_call(a, stream, false, nullptr);
+    return ws_call(a, stream, false, nullptr);
 }
 
 }  // namespace gdn

@@ -261,12 +261,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Waits for phase `parity` of the barrier; gives up after `limit` polls (each poll
-// may suspend the thread for a short hardware-defined time) and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+// Like mbar_try_wait, suspending for at most about `hint_ns` while the phase is open.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+// Bound on every wait inside the kernels, in nanoseconds of the global timer.
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
+// Waits for phase `parity` of the barrier; gives up after about `timeout_ns` and
+// returns false. `give_up` is polled now and then so a CTA can stop waiting early.
+template <typename GiveUp>
+__device__ __forceinline__ bool mbar_wait_deadline(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, GiveUp give_up) {
+    if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
+        if ((i & 15) == 0) {
+            if (give_up()) return false;
+            if (globaltimer_ns() - t0 > timeout_ns) return false;
+        }
+    }
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = kWaitTimeoutNs) {
+    return mbar_wait_deadline(bar, parity, timeout_ns, [] { return false; });
 }
 // One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into
 // this CTA's shared memory, counted on `bar`.

@@ -80,7 +80,9 @@ int decode_column_splits(int B, int Hv, int G, int dv);
 int recurrent_column_splits(int B, int Hv, int dv);
 
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
-// Persistent single-token kernel: co-resident cluster capacity, and the launch.
+// Persistent single-token kernel: whether it handles the shape, its co-resident
+// cluster capacity, and the launch.
+bool persistent_supported(const DecodeArgs& a);
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters);
 cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_conv_update(const ConvArgs& a, cudaStream_t stream);

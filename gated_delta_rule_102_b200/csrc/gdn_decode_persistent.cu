@@ -60,19 +60,26 @@ struct WS {
     static constexpr int RG = 32 / CG;           // row groups per warp
     static constexpr int RPL = DK / RG;          // rows per lane
     static constexpr int TILE_BYTES = DK * DV * 4;
-    static constexpr int NSTAGE = clampi(196608 / TILE_BYTES, 2, 8);
+    static constexpr int MAXNCH = 2 * DK + DV;   // most conv channels one CTA owns (G = 1)
+    // staged conv inputs of one unit: W rows (W-1 history rows, then x) of the CTA's
+    // channels, then the channels' W weights
+    static constexpr int CROWS = kMaxConvWidthPersistent * MAXNCH * 2;
+    static constexpr int CSTAGE = round_up(CROWS, 16) + round_up(MAXNCH * kMaxConvWidthPersistent * 2, 16);
+    // as many stages as fit: each costs its tile, conv inputs, z, v, info and a q/k buffer
+    static constexpr int PER_STAGE = TILE_BYTES + CSTAGE + DV * 6 + 32 + 2 * DK * 4 + 24;
+    static constexpr int NSTAGE = clampi((232448 - 2048 - 2 * DK * 4) / PER_STAGE, 2, 8);
     static constexpr int QB = NSTAGE + 1;        // q/k buffers: one more than stages (see the producer)
-    static constexpr int MAXCH = (2 * DK + DV + 31) / 32;  // conv channels per producer lane
     // shared-memory byte offsets
     static constexpr int TILES = 0;
-    static constexpr int ZB = TILES + NSTAGE * TILE_BYTES;          // [NSTAGE][DV] bf16
+    static constexpr int CONV = TILES + NSTAGE * TILE_BYTES;        // [NSTAGE] staged conv inputs
+    static constexpr int ZB = CONV + NSTAGE * CSTAGE;               // [NSTAGE][DV] bf16
     static constexpr int VS = ZB + round_up(NSTAGE * DV * 2, 16);    // [NSTAGE][DV] f32
     static constexpr int SI = VS + NSTAGE * DV * 4;                  // [NSTAGE] StageInfo
     static constexpr int QK = SI + NSTAGE * (int)sizeof(StageInfo);  // [QB][2*DK] f32
     static constexpr int PART = QK + QB * 2 * DK * 4;                // [NTEAMS][2][TEAM_WARPS] f32
     static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
-    static constexpr int BARS = FLAG + 16;                           // full, empty [NSTAGE]; qk [QB]
-    static constexpr int TOTAL = BARS + (2 * NSTAGE + QB) * 8;
+    static constexpr int BARS = FLAG + 16;  // full, empty, conv [NSTAGE]; qk [QB]
+    static constexpr int TOTAL = BARS + (3 * NSTAGE + QB) * 8;
     static_assert(CG >= 1 && RG >= 1 && RPL >= 1 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
 };
@@ -85,7 +92,7 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(WS<DK, DV>::NT, 1)
 decode_ws_kernel(const DecodeArgs p, const int ncl) {
     using L = WS<DK, DV>;
-    constexpr int NSTAGE = L::NSTAGE, QB = L::QB, WM = kMaxConvWidthPersistent;
+    constexpr int NSTAGE = L::NSTAGE, QB = L::QB;
     extern __shared__ __align__(128) unsigned char smem[];
     float* tiles = reinterpret_cast<float*>(smem + L::TILES);
     uint16_t* zb = reinterpret_cast<uint16_t*>(smem + L::ZB);
@@ -96,7 +103,8 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::FLAG);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
     uint64_t* empty = full + NSTAGE;
-    uint64_t* qkbar = empty + NSTAGE;
+    uint64_t* cbar = empty + NSTAGE;
+    uint64_t* qkbar = cbar + NSTAGE;
 
     const int Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk, C = p.sh.C, W = p.sh.W;
     const int rank = (int)cluster_ctarank(), cid = blockIdx.x / G;
@@ -108,6 +116,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(full + s, 2);                // the producer's copy arrival and its publish arrival
             mbar_init(empty + s, L::TEAM_WARPS);   // one arrival per warp of the consuming team
+            mbar_init(cbar + s, 1);                // the staged conv inputs
         }
         for (int q = 0; q < QB; ++q) mbar_init(qkbar + q, 1);
         *abort_flag = 0;
@@ -132,117 +141,107 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
 
     if (warp == 0) {
         // ============================== producer ==============================
-        const int qk_lo = (rank * 2 * DK) / G, qk_hi = ((rank + 1) * 2 * DK) / G, nqk = qk_hi - qk_lo;
-        const int nch = nqk + DV;
+        // This CTA's conv channels, in local order: its share of the k-head's q/k
+        // channels, then its v-head's v channels. They form at most three runs of
+        // consecutive pool channels (q, k, v), each staged by bulk copies.
+        const int qk_lo = (rank * 2 * DK) / G, nqk = (2 * DK) / G, nch = nqk + DV;
+        const int nseg = G == 1 ? 3 : 2;
+        auto seg_info = [&](int sg, int hk, int h, int& lc, int& ch, int& cnt) {
+            if (G == 1 && sg < 2) {
+                lc = sg * DK;
+                ch = sg * Hk * DK + hk * DK;
+                cnt = DK;
+            } else if (sg == 0) {
+                lc = 0;
+                ch = qk_lo < DK ? hk * DK + qk_lo : Hk * DK + hk * DK + (qk_lo - DK);
+                cnt = nqk;
+            } else {
+                lc = nqk;
+                ch = 2 * Hk * DK + h * DV;
+                cnt = DV;
+            }
+        };
         auto slot_of = [&](int u) { return u < n ? __ldg(p.slots + group_seq(u)) : -1; };
-        auto channel_of = [&](int c, int hk, int h) {
-            if (c < nqk) {
-                const int j = qk_lo + c;
-                return j < DK ? hk * DK + j : Hk * DK + hk * DK + (j - DK);
-            }
-            return 2 * Hk * DK + h * DV + (c - nqk);
-        };
-        uint32_t ph[L::MAXCH][WM - 1], px[L::MAXCH], pw[L::MAXCH][WM];
-        uint16_t pa = 0, pb = 0;
-        float pA = 0.f, pdt = 0.f;
-        auto prefetch = [&](int u, int slot) {
-            const int seq = group_seq(u), hk = group_hk(u), h = hk * G + rank;
-            const uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
-#pragma unroll
-            for (int i = 0; i < L::MAXCH; ++i) {
-                const int c = lane + 32 * i;
-                if (c < nch) {
-                    const int ch = channel_of(c, hk, h);
-#pragma unroll
-                    for (int r = 0; r < WM - 1; ++r) ph[i][r] = r < W - 1 ? hist[(size_t)r * C + ch] : 0u;
-                    px[i] = p.qkv[(size_t)seq * C + ch];
-#pragma unroll
-                    for (int j = 0; j < WM; ++j) pw[i][j] = j < W ? p.conv_w[(size_t)ch * W + j] : 0u;
+        const int conv_bytes = 2 * W * nch * 2;  // W rows and W weights per channel, bf16
+        // copies of unit v into stage v % NSTAGE: tile + z row, and the conv inputs
+        auto issue = [&](int v, int slot) {
+            const int s = v % NSTAGE, seq = group_seq(v), hk = group_hk(v), h = hk * G + rank;
+            const bool valid = slot_ok(slot);
+            if (lane == 0) {
+                if (valid) {
+                    mbar_arrive_expect_tx(full + s, L::TILE_BYTES + DV * 2);
+                    mbar_arrive_expect_tx(cbar + s, conv_bytes);
+                } else {
+                    mbar_arrive(full + s);
+                    mbar_arrive(cbar + s);
                 }
-            }
-            if (lane == 0) {
-                pa = p.a[(size_t)seq * Hv + h];
-                pb = p.b[(size_t)seq * Hv + h];
-                pA = p.A_log[h];
-                pdt = p.dt_bias[h];
-            }
-        };
-        int sl0 = slot_of(0), sl1 = slot_of(1), sl2 = slot_of(2);
-        if (n > 0 && slot_ok(sl0)) prefetch(0, sl0);
-        for (int v = 0; v < n; ++v) {
-            const int s = v % NSTAGE, q = v % QB;
-            const int seq = group_seq(v), hk = group_hk(v), h = hk * G + rank;
-            const bool valid = slot_ok(sl0);
-            if (v >= NSTAGE && !wait(empty + s, ((v / NSTAGE) - 1) & 1)) {
-                fail();
-                break;
-            }
-            // ---- the state tile and z row of unit v into stage s
-            if (lane == 0) {
-                if (valid) mbar_arrive_expect_tx(full + s, L::TILE_BYTES + DV * 2);
-                else mbar_arrive(full + s);
             }
             __syncwarp();
-            if (valid) {
-                const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)sl0 * Hv + h) * (size_t)(DK * DV));
-                char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
-                constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
-                if (lane < nchunk) {
-                    const int c = lane * kTileChunk;
-                    tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
-                } else if (lane == nchunk) {
-                    tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
+            if (!valid) return;
+            constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
+            const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h) * (size_t)(DK * DV));
+            char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
+            if (lane < nchunk) {
+                const int c = lane * kTileChunk;
+                tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
+            } else if (lane == nchunk) {
+                tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
+            }
+            // conv inputs: per run, W-1 history rows, the x row and the weights
+            const int k = lane - 8;
+            if (k >= 0 && k < nseg * (W + 1)) {
+                const int sg = k / (W + 1), kind = k - sg * (W + 1);
+                int lc, ch, cnt;
+                seg_info(sg, hk, h, lc, ch, cnt);
+                unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
+                if (kind < W - 1) {
+                    tma_load_1d(cst + (kind * nch + lc) * 2, p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch,
+                                cnt * 2, cbar + s);
+                } else if (kind == W - 1) {
+                    tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
+                } else {
+                    tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W, cnt * W * 2,
+                                cbar + s);
                 }
             }
-            // ---- step 3 for this CTA's channels of unit v
-            const uint16_t ga = pa, gb = pb;
-            const float gA = pA, gdt = pdt;
+        };
+        // step 3 for unit v from its staged inputs, the q/k exchange, then the norms,
+        // k.q and gates; finally the stage is published to the consumers
+        uint16_t ga = 0, gb = 0;
+        float gA = 0.f, gdt = 0.f;
+        auto finish = [&](int v, int slot) {
+            const int s = v % NSTAGE, q = v % QB, hk = group_hk(v), h = hk * G + rank;
+            const bool valid = slot_ok(slot);
             if (valid) {
-                uint16_t* hist = p.conv_pool + (size_t)sl0 * (W - 1) * C;
+                if (!wait(cbar + s, (v / NSTAGE) & 1)) return false;
+                const uint16_t* rows = reinterpret_cast<const uint16_t*>(smem + L::CONV + s * L::CSTAGE);
+                const uint16_t* wts = reinterpret_cast<const uint16_t*>(smem + L::CONV + s * L::CSTAGE +
+                                                                         round_up(W * nch * 2, 16));
+                uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
                 const uint32_t q_loc = smem_addr(qkb + q * 2 * DK + qk_lo), bar_loc = smem_addr(qkbar + q);
-#pragma unroll
-                for (int i = 0; i < L::MAXCH; ++i) {
-                    const int c = lane + 32 * i;
-                    if (c < nch) {
-                        const int ch = channel_of(c, hk, h);
-                        float acc = 0.f;
-#pragma unroll
-                        for (int j = 0; j < WM; ++j) {
-                            if (j < W) {
-                                const uint32_t xb = j < W - 1 ? ph[i][j < WM - 1 ? j : 0] : px[i];
-                                acc = fmaf(bf16_bits_to_float(pw[i][j]), bf16_bits_to_float(xb), acc);
-                            }
-                        }
-                        const float sv = silu(acc);
-                        if (c < nqk) {
-                            for (int r = 0; r < G; ++r)
-                                st_async_f32(cluster_map_u32(q_loc + 4 * c, r), sv, cluster_map_u32(bar_loc, r));
-                        } else {
-                            vsb[s * DV + (c - nqk)] = sv;
-                        }
-#pragma unroll
-                        for (int r = 0; r < WM - 1; ++r) {
-                            if (r < W - 1) {
-                                uint32_t nb = px[i];
-                                if (r + 1 < W - 1) nb = ph[i][r + 1 < WM - 1 ? r + 1 : 0];
-                                hist[(size_t)r * C + ch] = (uint16_t)nb;
-                            }
-                        }
+                for (int c = lane; c < nch; c += 32) {
+                    float acc = 0.f;
+                    for (int j = 0; j < W; ++j)
+                        acc = fmaf(bf16_bits_to_float(wts[c * W + j]), bf16_bits_to_float(rows[j * nch + c]), acc);
+                    const float sv = silu(acc);
+                    int lc, ch, cnt;
+                    const int sg = G == 1 ? (c < DK ? 0 : (c < 2 * DK ? 1 : 2)) : (c < nqk ? 0 : 1);
+                    seg_info(sg, hk, h, lc, ch, cnt);
+                    ch += c - lc;
+                    if (c < nqk) {
+                        for (int r = 0; r < G; ++r)
+                            st_async_f32(cluster_map_u32(q_loc + 4 * c, r), sv, cluster_map_u32(bar_loc, r));
+                    } else {
+                        vsb[s * DV + (c - nqk)] = sv;
                     }
+                    for (int r = 0; r < W - 1; ++r) hist[(size_t)r * C + ch] = rows[(r + 1) * nch + c];
                 }
             }
-            // ---- inputs of unit v+1 (they land while this unit's shares are exchanged)
-            const int sl3 = slot_of(v + 3);
-            if (v + 1 < n && slot_ok(sl1)) prefetch(v + 1, sl1);
-            // ---- all q/k shares of unit v: norms, k.q, gates
             if (lane == 0) {
                 if (valid) mbar_arrive_expect_tx(qkbar + q, 2 * DK * 4);
                 else mbar_arrive(qkbar + q);
             }
-            if (!wait(qkbar + q, (v / QB) & 1)) {
-                fail();
-                break;
-            }
+            if (!wait(qkbar + q, (v / QB) & 1)) return false;
             if (valid) {
                 const float* qr = qkb + q * 2 * DK;
                 float sq = 0.f, sk = 0.f, dot = 0.f;
@@ -264,7 +263,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                     st.nk = rsqrtf(sk + p.sh.l2_eps);
                     st.kq = dot * st.nq * st.nk;
                     gate_and_beta(ga, gb, gA, gdt, st.alpha, st.beta);
-                    st.slot = sl0;
+                    st.slot = slot;
                 }
             } else if (lane == 0) {
                 si[s].slot = -1;
@@ -272,9 +271,43 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(full + s);
+            return true;
+        };
+        // unit v's copies go out, then unit v-1 is finished: the conv inputs of a unit
+        // have a whole iteration to land before they are needed
+        int sl_prev = -1, sl0 = slot_of(0), sl1 = slot_of(1);
+        uint16_t na = 0, nb = 0;
+        float nA = 0.f, ndt = 0.f;
+        for (int v = 0; v <= n; ++v) {
+            if (v < n) {
+                if (v >= NSTAGE && !wait(empty + v % NSTAGE, ((v / NSTAGE) - 1) & 1)) {
+                    fail();
+                    break;
+                }
+                issue(v, sl0);
+            }
+            const uint16_t a_v = (v < n && lane == 0) ? p.a[(size_t)group_seq(v) * Hv + group_hk(v) * G + rank] : 0;
+            const uint16_t b_v = (v < n && lane == 0) ? p.b[(size_t)group_seq(v) * Hv + group_hk(v) * G + rank] : 0;
+            const float A_v = (v < n && lane == 0) ? p.A_log[group_hk(v) * G + rank] : 0.f;
+            const float dt_v = (v < n && lane == 0) ? p.dt_bias[group_hk(v) * G + rank] : 0.f;
+            const int sl2 = slot_of(v + 2);
+            if (v >= 1) {
+                ga = na;
+                gb = nb;
+                gA = nA;
+                gdt = ndt;
+                if (!finish(v - 1, sl_prev)) {
+                    fail();
+                    break;
+                }
+            }
+            na = a_v;
+            nb = b_v;
+            nA = A_v;
+            ndt = dt_v;
+            sl_prev = sl0;
             sl0 = sl1;
             sl1 = sl2;
-            sl2 = sl3;
         }
         if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
             for (int i = 0; i < 1024; ++i) __nanosleep(64);
@@ -422,7 +455,8 @@ cudaError_t ws_dispatch(const DecodeArgs& a, int G, cudaStream_t stream, bool qu
 
 cudaError_t ws_call(const DecodeArgs& a, cudaStream_t stream, bool query_only, int* cap) {
     const int G = a.sh.Hv / a.sh.Hk;
-    if (a.T != 1 || a.sh.W > kMaxConvWidthPersistent || G > 8) return cudaErrorInvalidValue;
+    if (a.T != 1 || a.sh.W > kMaxConvWidthPersistent || G > 8 || (2 * a.sh.dk) % (8 * G) != 0)
+        return cudaErrorInvalidValue;
     switch (a.sh.dk) {
         case 16: return ws_dispatch<16>(a, G, stream, query_only, cap);
         case 32: return ws_dispatch<32>(a, G, stream, query_only, cap);
@@ -435,7 +469,10 @@ cudaError_t ws_call(const DecodeArgs& a, cudaStream_t stream, bool query_only, i
 }  // namespace
 
 bool persistent_supported(const DecodeArgs& a) {
-    return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && a.sh.Hv / a.sh.Hk <= 8;
+    // the q/k share of each CTA must be a whole number of 16-byte bf16 runs for the
+    // bulk copies of the conv inputs
+    const int G = a.sh.Hv / a.sh.Hk;
+    return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && G <= 8 && (2 * a.sh.dk) % (8 * G) == 0;
 }
 
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters) {

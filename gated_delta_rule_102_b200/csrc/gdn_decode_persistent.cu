@@ -8,14 +8,16 @@
 // head, contiguous in the pool.
 //
 // Roles inside a CTA.
-//  * Warp 0, the producer, runs ahead of the math. For unit v it waits until stage
-//    v % NSTAGE is free, starts the TMA bulk copies of the state tile and the z row
-//    into it, convolves this CTA's channels (its share of the k-head's q/k channels
-//    plus its v-head's v channels) from inputs it loaded one unit earlier, sends the
-//    raw q/k share to every CTA of the cluster with st.async (completed on the
-//    receiver's mbarrier), rolls the conv history, waits for the other shares, and
-//    publishes the q/k norms, k.q, the gates and the slot for the stage.
-//  * Warps 1..8 form teams that take units in turn. A team owns a unit: each warp
+//  * Warp 0, the loader, only issues TMA bulk copies: as soon as stage v % NSTAGE is
+//    free it starts the copies of unit v's state tile and z row (completing on the
+//    stage's `full` barrier) and of its conv inputs (history rows, x, weights) and
+//    a/b values (completing on `cbar`).
+//  * Warp 1, the finisher, takes units in order once their conv inputs have landed:
+//    it convolves this CTA's channels (its share of the k-head's q/k channels plus
+//    its v-head's v channels), sends the raw q/k share to every CTA of the cluster
+//    with st.async (completed on the receiver's mbarrier), rolls the conv history,
+//    waits for the other shares, and publishes the q/k norms, k.q and the gates.
+//  * Warps 2..9 form teams that take units in turn. A team owns a unit: each warp
 //    holds a band of columns (the columns of S are independent under the update),
 //    reads the tile from shared memory twice (S^T k and S^T q, then the update),
 //    reduces over dk with two shuffle stages, streams the new rows to HBM, and then
@@ -24,10 +26,10 @@
 // state is read once and written once, and HBM sees a steady stream of TMA loads and
 // row stores instead of alternating load, compute and store phases.
 //
-// Every wait is an mbarrier poll with a bound. When one expires the CTA sets the
-// timeout bit of the error flag, all roles leave their loops, the producer waits
-// (bounded) for its copies in flight, and the CTA leaves through the final cluster
-// barrier.
+// Every wait is an mbarrier poll bounded by the global timer. When one expires the
+// CTA sets the timeout bit of the error flag, all roles leave their loops, the loader
+// gives its copies in flight time to land, and the CTA leaves through the final
+// cluster barrier.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -52,7 +54,9 @@ struct StageInfo {  // what the producer publishes for a staged unit
 template <int DK, int DV>
 struct WS {
     static constexpr int CONSUMER_WARPS = 8;
-    static constexpr int NT = 32 * (1 + CONSUMER_WARPS);
+    static constexpr int PRODUCER_WARPS = 2;  // a copy-issuing warp and a conv/gate warp
+    static constexpr int NT = 32 * (PRODUCER_WARPS + CONSUMER_WARPS);
+    static constexpr int MAX_HV = 128;        // A_log, dt_bias held in shared memory
     static constexpr int TEAM_WARPS = DV >= 128 ? 4 : (DV >= 64 ? 2 : 1);
     static constexpr int NTEAMS = CONSUMER_WARPS / TEAM_WARPS;
     static constexpr int CPW = DV / TEAM_WARPS;  // columns per consumer warp (32, or 16 when dv = 16)
@@ -66,13 +70,15 @@ struct WS {
     static constexpr int CROWS = kMaxConvWidthPersistent * MAXNCH * 2;
     static constexpr int CSTAGE = round_up(CROWS, 16) + round_up(MAXNCH * kMaxConvWidthPersistent * 2, 16);
     // as many stages as fit: each costs its tile, conv inputs, z, v, info and a q/k buffer
-    static constexpr int PER_STAGE = TILE_BYTES + CSTAGE + DV * 6 + 32 + 2 * DK * 4 + 24;
-    static constexpr int NSTAGE = clampi((232448 - 2048 - 2 * DK * 4) / PER_STAGE, 2, 8);
+    static constexpr int PER_STAGE = TILE_BYTES + CSTAGE + DV * 6 + 32 + 2 * DK * 4 + 24 + 32;
+    static constexpr int NSTAGE = clampi((232448 - 3072 - 2 * DK * 4) / PER_STAGE, 2, 8);
     static constexpr int QB = NSTAGE + 1;        // q/k buffers: one more than stages (see the producer)
     // shared-memory byte offsets
     static constexpr int TILES = 0;
     static constexpr int CONV = TILES + NSTAGE * TILE_BYTES;        // [NSTAGE] staged conv inputs
-    static constexpr int ZB = CONV + NSTAGE * CSTAGE;               // [NSTAGE][DV] bf16
+    static constexpr int AB = CONV + NSTAGE * CSTAGE;               // [NSTAGE][2][8] bf16: a, b groups
+    static constexpr int GP = AB + NSTAGE * 32;                     // [2][MAX_HV] f32: A_log, dt_bias
+    static constexpr int ZB = GP + 2 * MAX_HV * 4;                  // [NSTAGE][DV] bf16
     static constexpr int VS = ZB + round_up(NSTAGE * DV * 2, 16);    // [NSTAGE][DV] f32
     static constexpr int SI = VS + NSTAGE * DV * 4;                  // [NSTAGE] StageInfo
     static constexpr int QK = SI + NSTAGE * (int)sizeof(StageInfo);  // [QB][2*DK] f32
@@ -139,35 +145,49 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     auto group_hk = [&](int u) { return (cid + u * ncl) % Hk; };
     auto slot_ok = [&](int s) { return s >= 0 && s < p.P; };
 
+    // This CTA's conv channels, in local order: its share of the k-head's q/k
+    // channels, then its v-head's v channels. They form at most three runs of
+    // consecutive pool channels (q, k, v), each staged by bulk copies.
+    const int qk_lo = (rank * 2 * DK) / G, nqk = (2 * DK) / G, nch = nqk + DV;
+    const int nseg = G == 1 ? 3 : 2;
+    auto seg_info = [&](int sg, int hk, int h, int& lc, int& ch, int& cnt) {
+        if (G == 1 && sg < 2) {
+            lc = sg * DK;
+            ch = sg * Hk * DK + hk * DK;
+            cnt = DK;
+        } else if (sg == 0) {
+            lc = 0;
+            ch = qk_lo < DK ? hk * DK + qk_lo : Hk * DK + hk * DK + (qk_lo - DK);
+            cnt = nqk;
+        } else {
+            lc = nqk;
+            ch = 2 * Hk * DK + h * DV;
+            cnt = DV;
+        }
+    };
+    float* gparams = reinterpret_cast<float*>(smem + L::GP);  // A_log then dt_bias
+
     if (warp == 0) {
-        // ============================== producer ==============================
-        // This CTA's conv channels, in local order: its share of the k-head's q/k
-        // channels, then its v-head's v channels. They form at most three runs of
-        // consecutive pool channels (q, k, v), each staged by bulk copies.
-        const int qk_lo = (rank * 2 * DK) / G, nqk = (2 * DK) / G, nch = nqk + DV;
-        const int nseg = G == 1 ? 3 : 2;
-        auto seg_info = [&](int sg, int hk, int h, int& lc, int& ch, int& cnt) {
-            if (G == 1 && sg < 2) {
-                lc = sg * DK;
-                ch = sg * Hk * DK + hk * DK;
-                cnt = DK;
-            } else if (sg == 0) {
-                lc = 0;
-                ch = qk_lo < DK ? hk * DK + qk_lo : Hk * DK + hk * DK + (qk_lo - DK);
-                cnt = nqk;
-            } else {
-                lc = nqk;
-                ch = 2 * Hk * DK + h * DV;
-                cnt = DV;
-            }
-        };
-        auto slot_of = [&](int u) { return u < n ? __ldg(p.slots + group_seq(u)) : -1; };
-        const int conv_bytes = 2 * W * nch * 2;  // W rows and W weights per channel, bf16
-        // copies of unit v into stage v % NSTAGE: tile + z row, and the conv inputs
-        auto issue = [&](int v, int slot) {
+        // ============================== loader ==============================
+        // Unit v's copies into stage v % NSTAGE as soon as the stage is free: the
+        // state tile and z row (completing on full), the conv inputs and the a/b
+        // groups (completing on cbar). The slot goes along in the stage info.
+        const int conv_bytes = 2 * W * nch * 2 + 32;
+        int slots32 = -1;
+        for (int v = 0; v < n; ++v) {
             const int s = v % NSTAGE, seq = group_seq(v), hk = group_hk(v), h = hk * G + rank;
+            if ((v & 31) == 0) {  // the next 32 units' slots, one per lane
+                const int u = v + lane;
+                slots32 = u < n ? __ldg(p.slots + group_seq(u)) : -1;
+            }
+            const int slot = __shfl_sync(0xffffffffu, slots32, v & 31);
+            if (v >= NSTAGE && !wait(empty + s, ((v / NSTAGE) - 1) & 1)) {
+                fail();
+                break;
+            }
             const bool valid = slot_ok(slot);
             if (lane == 0) {
+                si[s].slot = valid ? slot : -1;
                 if (valid) {
                     mbar_arrive_expect_tx(full + s, L::TILE_BYTES + DV * 2);
                     mbar_arrive_expect_tx(cbar + s, conv_bytes);
@@ -177,43 +197,58 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 }
             }
             __syncwarp();
-            if (!valid) return;
+            if (!valid) continue;
             constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
             const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h) * (size_t)(DK * DV));
             char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
+            unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
             if (lane < nchunk) {
                 const int c = lane * kTileChunk;
                 tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
             } else if (lane == nchunk) {
                 tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
-            }
-            // conv inputs: per run, W-1 history rows, the x row and the weights
-            const int k = lane - 8;
-            if (k >= 0 && k < nseg * (W + 1)) {
-                const int sg = k / (W + 1), kind = k - sg * (W + 1);
-                int lc, ch, cnt;
-                seg_info(sg, hk, h, lc, ch, cnt);
-                unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
-                if (kind < W - 1) {
-                    tma_load_1d(cst + (kind * nch + lc) * 2, p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch,
-                                cnt * 2, cbar + s);
-                } else if (kind == W - 1) {
-                    tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
-                } else {
-                    tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W, cnt * W * 2,
-                                cbar + s);
+            } else if (lane == 6 || lane == 7) {  // the 8-aligned group of a (lane 6) or b (lane 7) holding h
+                const uint16_t* srcab = (lane == 6 ? p.a : p.b) + (size_t)seq * Hv + (h & ~7);
+                tma_load_1d(smem + L::AB + s * 32 + (lane - 6) * 16, srcab, 16, cbar + s);
+            } else {
+                const int k = lane - 8;
+                if (k >= 0 && k < nseg * (W + 1)) {
+                    const int sg = k / (W + 1), kind = k - sg * (W + 1);
+                    int lc, ch, cnt;
+                    seg_info(sg, hk, h, lc, ch, cnt);
+                    if (kind < W - 1) {
+                        tma_load_1d(cst + (kind * nch + lc) * 2,
+                                    p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch, cnt * 2, cbar + s);
+                    } else if (kind == W - 1) {
+                        tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
+                    } else {
+                        tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W,
+                                    cnt * W * 2, cbar + s);
+                    }
                 }
             }
-        };
-        // step 3 for unit v from its staged inputs, the q/k exchange, then the norms,
-        // k.q and gates; finally the stage is published to the consumers
-        uint16_t ga = 0, gb = 0;
-        float gA = 0.f, gdt = 0.f;
-        auto finish = [&](int v, int slot) {
+        }
+        if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
+            for (int i = 0; i < 1024; ++i) __nanosleep(64);
+        }
+    } else if (warp == 1) {
+        // ============================== finisher ==============================
+        // Unit v in order: step 3 from its staged inputs, the q/k exchange, the norms,
+        // k.q and gates; then the stage is published to the consumers.
+        for (int i = lane; i < Hv; i += 32) {
+            gparams[i] = p.A_log[i];
+            gparams[L::MAX_HV + i] = p.dt_bias[i];
+        }
+        __syncwarp();
+        for (int v = 0; v < n; ++v) {
             const int s = v % NSTAGE, q = v % QB, hk = group_hk(v), h = hk * G + rank;
-            const bool valid = slot_ok(slot);
+            if (!wait(cbar + s, (v / NSTAGE) & 1)) {
+                fail();
+                break;
+            }
+            const int slot = si[s].slot;
+            const bool valid = slot >= 0;
             if (valid) {
-                if (!wait(cbar + s, (v / NSTAGE) & 1)) return false;
                 const uint16_t* rows = reinterpret_cast<const uint16_t*>(smem + L::CONV + s * L::CSTAGE);
                 const uint16_t* wts = reinterpret_cast<const uint16_t*>(smem + L::CONV + s * L::CSTAGE +
                                                                          round_up(W * nch * 2, 16));
@@ -241,7 +276,10 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 if (valid) mbar_arrive_expect_tx(qkbar + q, 2 * DK * 4);
                 else mbar_arrive(qkbar + q);
             }
-            if (!wait(qkbar + q, (v / QB) & 1)) return false;
+            if (!wait(qkbar + q, (v / QB) & 1)) {
+                fail();
+                break;
+            }
             if (valid) {
                 const float* qr = qkb + q * 2 * DK;
                 float sq = 0.f, sk = 0.f, dot = 0.f;
@@ -262,59 +300,19 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                     st.nq = rsqrtf(sq + p.sh.l2_eps) * p.sh.q_scale;
                     st.nk = rsqrtf(sk + p.sh.l2_eps);
                     st.kq = dot * st.nq * st.nk;
-                    gate_and_beta(ga, gb, gA, gdt, st.alpha, st.beta);
-                    st.slot = slot;
+                    const uint16_t* ab = reinterpret_cast<const uint16_t*>(smem + L::AB + s * 32);
+                    gate_and_beta(ab[h & 7], ab[8 + (h & 7)], gparams[h], gparams[L::MAX_HV + h], st.alpha,
+                                  st.beta);
                 }
-            } else if (lane == 0) {
-                si[s].slot = -1;
-                if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
+            } else if (lane == 0 && p.err_flag) {
+                atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(full + s);
-            return true;
-        };
-        // unit v's copies go out, then unit v-1 is finished: the conv inputs of a unit
-        // have a whole iteration to land before they are needed
-        int sl_prev = -1, sl0 = slot_of(0), sl1 = slot_of(1);
-        uint16_t na = 0, nb = 0;
-        float nA = 0.f, ndt = 0.f;
-        for (int v = 0; v <= n; ++v) {
-            if (v < n) {
-                if (v >= NSTAGE && !wait(empty + v % NSTAGE, ((v / NSTAGE) - 1) & 1)) {
-                    fail();
-                    break;
-                }
-                issue(v, sl0);
-            }
-            const uint16_t a_v = (v < n && lane == 0) ? p.a[(size_t)group_seq(v) * Hv + group_hk(v) * G + rank] : 0;
-            const uint16_t b_v = (v < n && lane == 0) ? p.b[(size_t)group_seq(v) * Hv + group_hk(v) * G + rank] : 0;
-            const float A_v = (v < n && lane == 0) ? p.A_log[group_hk(v) * G + rank] : 0.f;
-            const float dt_v = (v < n && lane == 0) ? p.dt_bias[group_hk(v) * G + rank] : 0.f;
-            const int sl2 = slot_of(v + 2);
-            if (v >= 1) {
-                ga = na;
-                gb = nb;
-                gA = nA;
-                gdt = ndt;
-                if (!finish(v - 1, sl_prev)) {
-                    fail();
-                    break;
-                }
-            }
-            na = a_v;
-            nb = b_v;
-            nA = A_v;
-            ndt = dt_v;
-            sl_prev = sl0;
-            sl0 = sl1;
-            sl1 = sl2;
-        }
-        if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
-            for (int i = 0; i < 1024; ++i) __nanosleep(64);
         }
     } else {
         // ============================== consumers ==============================
-        const int cw = warp - 1, team = cw / L::TEAM_WARPS, wt = cw - team * L::TEAM_WARPS;
+        const int cw = warp - L::PRODUCER_WARPS, team = cw / L::TEAM_WARPS, wt = cw - team * L::TEAM_WARPS;
         const int rg = lane / L::CG, cg = lane - rg * L::CG;
         const int col = wt * L::CPW + 4 * cg;
         int parity_part = 0;
@@ -455,8 +453,7 @@ cudaError_t ws_dispatch(const DecodeArgs& a, int G, cudaStream_t stream, bool qu
 
 cudaError_t ws_call(const DecodeArgs& a, cudaStream_t stream, bool query_only, int* cap) {
     const int G = a.sh.Hv / a.sh.Hk;
-    if (a.T != 1 || a.sh.W > kMaxConvWidthPersistent || G > 8 || (2 * a.sh.dk) % (8 * G) != 0)
-        return cudaErrorInvalidValue;
+    if (!persistent_supported(a)) return cudaErrorInvalidValue;
     switch (a.sh.dk) {
         case 16: return ws_dispatch<16>(a, G, stream, query_only, cap);
         case 32: return ws_dispatch<32>(a, G, stream, query_only, cap);
@@ -472,7 +469,8 @@ bool persistent_supported(const DecodeArgs& a) {
     // the q/k share of each CTA must be a whole number of 16-byte bf16 runs for the
     // bulk copies of the conv inputs
     const int G = a.sh.Hv / a.sh.Hk;
-    return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && G <= 8 && (2 * a.sh.dk) % (8 * G) == 0;
+    return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && G <= 8 && (2 * a.sh.dk) % (8 * G) == 0 &&
+           a.sh.Hv % 8 == 0 && a.sh.Hv <= 128;
 }
 
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters) {

@@ -70,10 +70,10 @@ def test_fused_matches_oracle(spec):
 PERSISTENT_SHAPES = [
     # name              Hk Hv   dk   dv  W    B  T    P  steps
     ("p_d128_g2", 4, 8, 128, 128, 4, 40, 1, 48, 3),
-    ("p_d128_g1_w2", 2, 2, 128, 128, 2, 160, 1, 170, 2),
+    ("p_d128_g1_w2", 8, 8, 128, 128, 2, 40, 1, 44, 2),
     ("p_dk128_dv64_g4", 2, 8, 128, 64, 4, 80, 1, 80, 2),
     ("p_dk64_dv128_g8_w3", 1, 8, 64, 128, 3, 100, 1, 101, 2),
-    ("p_d32_g2_many", 2, 4, 32, 32, 3, 800, 1, 800, 3),
+    ("p_d32_g2_many", 4, 8, 32, 32, 3, 400, 1, 400, 3),
 ]
 
 

@@ -9,7 +9,7 @@
 
 #include <vector>
 
-#include "../../include/gdn.h"
+#include "gdn.h"
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
 

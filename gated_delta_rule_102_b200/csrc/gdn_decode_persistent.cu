@@ -54,7 +54,8 @@ struct StageInfo {  // what the producer publishes for a staged unit
 template <int DK, int DV>
 struct WS {
     static constexpr int CONSUMER_WARPS = 8;
-    static constexpr int PRODUCER_WARPS = 2;  // a copy-issuing warp and a conv/gate warp
+    static constexpr int FINISHER_WARPS = 4;
+    static constexpr int PRODUCER_WARPS = 1 + FINISHER_WARPS;  // the copy-issuing warp, then the conv/gate warps
     static constexpr int NT = 32 * (PRODUCER_WARPS + CONSUMER_WARPS);
     static constexpr int MAX_HV = 128;        // A_log, dt_bias held in shared memory
     static constexpr int TEAM_WARPS = DV >= 128 ? 4 : (DV >= 64 ? 2 : 1);
@@ -71,8 +72,8 @@ struct WS {
     static constexpr int CSTAGE = round_up(CROWS, 16) + round_up(MAXNCH * kMaxConvWidthPersistent * 2, 16);
     // as many stages as fit: each costs its tile, conv inputs, z, v, info and a q/k buffer
     static constexpr int PER_STAGE = TILE_BYTES + CSTAGE + DV * 6 + 32 + 2 * DK * 4 + 24 + 32;
-    static constexpr int NSTAGE = clampi((232448 - 3072 - 2 * DK * 4) / PER_STAGE, 2, 8);
-    static constexpr int QB = NSTAGE + 1;        // q/k buffers: one more than stages (see the producer)
+    static constexpr int NSTAGE = clampi((232448 - 3072 - 4 * DK * 4) / PER_STAGE, 2, 8);
+    static constexpr int QB = NSTAGE + 2;        // q/k buffers: two more than stages (see the finishers)
     // shared-memory byte offsets
     static constexpr int TILES = 0;
     static constexpr int CONV = TILES + NSTAGE * TILE_BYTES;        // [NSTAGE] staged conv inputs
@@ -86,7 +87,7 @@ struct WS {
     static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
     static constexpr int BARS = FLAG + 16;  // full, empty, conv [NSTAGE]; qk [QB]
     static constexpr int TOTAL = BARS + (3 * NSTAGE + QB) * 8;
-    static_assert(CG >= 1 && RG >= 1 && RPL >= 1 && RG * CG == 32, "consumer geometry");
+    static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && RPL % 4 == 0 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
 };
 
@@ -231,15 +232,22 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
             for (int i = 0; i < 1024; ++i) __nanosleep(64);
         }
-    } else if (warp == 1) {
-        // ============================== finisher ==============================
-        // Unit v in order: step 3 from its staged inputs, the q/k exchange, the norms,
-        // k.q and gates; then the stage is published to the consumers.
-        for (int i = lane; i < Hv; i += 32) {
-            gparams[i] = p.A_log[i];
-            gparams[L::MAX_HV + i] = p.dt_bias[i];
+    } else if (warp <= L::FINISHER_WARPS) {
+        // ============================== finishers ==============================
+        // Units in order once their conv inputs have landed. All finisher warps
+        // convolve this CTA's channels two at a time (step 3), send the raw q/k
+        // share to every CTA of the cluster, keep v and roll the history; then the
+        // first finisher warp waits for the other shares and publishes the norms, k.q
+        // and the gates. A finisher warp runs at most one unit ahead of the first.
+        const int fw = warp - 1;
+        constexpr int NFT = 32 * L::FINISHER_WARPS;
+        if (fw == 0) {
+            for (int i = lane; i < Hv; i += 32) {
+                gparams[i] = p.A_log[i];
+                gparams[L::MAX_HV + i] = p.dt_bias[i];
+            }
         }
-        __syncwarp();
+        named_barrier(15, NFT);
         for (int v = 0; v < n; ++v) {
             const int s = v % NSTAGE, q = v % QB, hk = group_hk(v), h = hk * G + rank;
             if (!wait(cbar + s, (v / NSTAGE) & 1)) {
@@ -249,29 +257,36 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             const int slot = si[s].slot;
             const bool valid = slot >= 0;
             if (valid) {
-                const uint16_t* rows = reinterpret_cast<const uint16_t*>(smem + L::CONV + s * L::CSTAGE);
-                const uint16_t* wts = reinterpret_cast<const uint16_t*>(smem + L::CONV + s * L::CSTAGE +
-                                                                         round_up(W * nch * 2, 16));
+                const unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
+                const uint16_t* rows = reinterpret_cast<const uint16_t*>(cst);
+                const uint16_t* wts = reinterpret_cast<const uint16_t*>(cst + round_up(W * nch * 2, 16));
                 uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
                 const uint32_t q_loc = smem_addr(qkb + q * 2 * DK + qk_lo), bar_loc = smem_addr(qkbar + q);
-                for (int c = lane; c < nch; c += 32) {
-                    float acc = 0.f;
-                    for (int j = 0; j < W; ++j)
-                        acc = fmaf(bf16_bits_to_float(wts[c * W + j]), bf16_bits_to_float(rows[j * nch + c]), acc);
-                    const float sv = silu(acc);
+                for (int c = 2 * (fw * 32 + lane); c < nch; c += 2 * NFT) {
+                    float acc0 = 0.f, acc1 = 0.f;
+                    for (int j = 0; j < W; ++j) {
+                        const uint32_t xx = *reinterpret_cast<const uint32_t*>(rows + j * nch + c);
+                        acc0 = fmaf(bf16_bits_to_float(wts[c * W + j]), bf16_bits_to_float(xx & 0xffffu), acc0);
+                        acc1 = fmaf(bf16_bits_to_float(wts[(c + 1) * W + j]), bf16_bits_to_float(xx >> 16), acc1);
+                    }
+                    const float s0 = silu(acc0), s1 = silu(acc1);
                     int lc, ch, cnt;
                     const int sg = G == 1 ? (c < DK ? 0 : (c < 2 * DK ? 1 : 2)) : (c < nqk ? 0 : 1);
                     seg_info(sg, hk, h, lc, ch, cnt);
                     ch += c - lc;
                     if (c < nqk) {
                         for (int r = 0; r < G; ++r)
-                            st_async_f32(cluster_map_u32(q_loc + 4 * c, r), sv, cluster_map_u32(bar_loc, r));
+                            st_async_f32x2(cluster_map_u32(q_loc + 4 * c, r), s0, s1, cluster_map_u32(bar_loc, r));
                     } else {
-                        vsb[s * DV + (c - nqk)] = sv;
+                        *reinterpret_cast<float2*>(vsb + s * DV + (c - nqk)) = make_float2(s0, s1);
                     }
-                    for (int r = 0; r < W - 1; ++r) hist[(size_t)r * C + ch] = rows[(r + 1) * nch + c];
+                    for (int r = 0; r < W - 1; ++r)
+                        *reinterpret_cast<uint32_t*>(hist + (size_t)r * C + ch) =
+                            *reinterpret_cast<const uint32_t*>(rows + (r + 1) * nch + c);
                 }
             }
+            named_barrier(15, NFT);  // every finisher's v values are written
+            if (fw != 0) continue;
             if (lane == 0) {
                 if (valid) mbar_arrive_expect_tx(qkbar + q, 2 * DK * 4);
                 else mbar_arrive(qkbar + q);
@@ -328,16 +343,21 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 const float4* tl = reinterpret_cast<const float4*>(tiles + (size_t)s * (DK * DV)) + col / 4;
                 const float* qr = qkb + q * 2 * DK;
                 const float* kr = qr + DK;
+                const int row0 = rg * L::RPL;  // this lane's rows: row0 .. row0 + RPL - 1
                 float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
-#pragma unroll 8
-                for (int i = 0; i < L::RPL; ++i) {
-                    const int row = rg + L::RG * i;
-                    const float4 x = tl[(size_t)row * (DV / 4)];
-                    const float ki = kr[row], qi = qr[row];
-                    mk.x = fmaf(x.x, ki, mk.x); mk.y = fmaf(x.y, ki, mk.y);
-                    mk.z = fmaf(x.z, ki, mk.z); mk.w = fmaf(x.w, ki, mk.w);
-                    mq.x = fmaf(x.x, qi, mq.x); mq.y = fmaf(x.y, qi, mq.y);
-                    mq.z = fmaf(x.z, qi, mq.z); mq.w = fmaf(x.w, qi, mq.w);
+#pragma unroll 2
+                for (int i = 0; i < L::RPL; i += 4) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(kr + row0 + i);
+                    const float4 q4 = *reinterpret_cast<const float4*>(qr + row0 + i);
+                    const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 x = tl[(size_t)(row0 + i + e) * (DV / 4)];
+                        mk.x = fmaf(x.x, kk[e], mk.x); mk.y = fmaf(x.y, kk[e], mk.y);
+                        mk.z = fmaf(x.z, kk[e], mk.z); mk.w = fmaf(x.w, kk[e], mk.w);
+                        mq.x = fmaf(x.x, qq[e], mq.x); mq.y = fmaf(x.y, qq[e], mq.y);
+                        mq.z = fmaf(x.z, qq[e], mq.z); mq.w = fmaf(x.w, qq[e], mq.w);
+                    }
                 }
 #pragma unroll
                 for (int off = L::CG; off < 32; off <<= 1) {
@@ -356,14 +376,17 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 const float4 dn = make_float4(d.x * st.nk, d.y * st.nk, d.z * st.nk, d.w * st.nk);
                 float4* Sg = reinterpret_cast<float4*>(p.state_pool + ((size_t)st.slot * Hv + h) * (size_t)(DK * DV) +
                                                        col);
-#pragma unroll 8
-                for (int i = 0; i < L::RPL; ++i) {
-                    const int row = rg + L::RG * i;
-                    float4 x = tl[(size_t)row * (DV / 4)];
-                    const float ki = kr[row];
-                    x.x = fmaf(st.alpha, x.x, ki * dn.x); x.y = fmaf(st.alpha, x.y, ki * dn.y);
-                    x.z = fmaf(st.alpha, x.z, ki * dn.z); x.w = fmaf(st.alpha, x.w, ki * dn.w);
-                    __stcs(Sg + (size_t)row * (DV / 4), x);
+#pragma unroll 2
+                for (int i = 0; i < L::RPL; i += 4) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(kr + row0 + i);
+                    const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float4 x = tl[(size_t)(row0 + i + e) * (DV / 4)];
+                        x.x = fmaf(st.alpha, x.x, kk[e] * dn.x); x.y = fmaf(st.alpha, x.y, kk[e] * dn.y);
+                        x.z = fmaf(st.alpha, x.z, kk[e] * dn.z); x.w = fmaf(st.alpha, x.w, kk[e] * dn.w);
+                        __stcs(Sg + (size_t)(row0 + i + e) * (DV / 4), x);
+                    }
                 }
                 // ---- step 8 over the whole head: the team's warps pool their sums of o^2
                 float ss = rg == 0 ? o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w : 0.f;
@@ -443,7 +466,9 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
 template <int DK>
 cudaError_t ws_dispatch(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap) {
     switch (a.sh.dv) {
-        case 16: return launch_ws_tile<DK, 16>(a, G, stream, query_only, cap);
+        case 16:
+            if constexpr (DK >= 32) return launch_ws_tile<DK, 16>(a, G, stream, query_only, cap);
+            return cudaErrorInvalidValue;
         case 32: return launch_ws_tile<DK, 32>(a, G, stream, query_only, cap);
         case 64: return launch_ws_tile<DK, 64>(a, G, stream, query_only, cap);
         case 128: return launch_ws_tile<DK, 128>(a, G, stream, query_only, cap);
@@ -470,7 +495,7 @@ bool persistent_supported(const DecodeArgs& a) {
     // bulk copies of the conv inputs
     const int G = a.sh.Hv / a.sh.Hk;
     return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && G <= 8 && (2 * a.sh.dk) % (8 * G) == 0 &&
-           a.sh.Hv % 8 == 0 && a.sh.Hv <= 128;
+           a.sh.Hv % 8 == 0 && a.sh.Hv <= 128 && (a.sh.dv >= 32 || a.sh.dk >= 32);
 }
 
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters) {

@@ -409,3 +409,14 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 }
 
 }  // namespace gdn
+
+namespace gdn {
+// Two floats into another cluster CTA's shared memory (8-byte aligned), counted as
+// 8 bytes on that CTA's mbarrier.
+__device__ __forceinline__ void st_async_f32x2(uint32_t remote_addr, float a, float b, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];\n" ::"r"(
+                     remote_addr),
+                 "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(remote_bar)
+                 : "memory");
+}
+}  // namespace gdn

@@ -203,30 +203,31 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h) * (size_t)(DK * DV));
             char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
             unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
+            // the small conv inputs first: the finishers need them long before the
+            // consumers need the tile
+            if (lane == 30 || lane == 31) {  // the 8-aligned group of a (lane 30) or b (lane 31) holding h
+                const uint16_t* srcab = (lane == 30 ? p.a : p.b) + (size_t)seq * Hv + (h & ~7);
+                tma_load_1d(smem + L::AB + s * 32 + (lane - 30) * 16, srcab, 16, cbar + s);
+            } else if (lane < nseg * (W + 1)) {
+                const int sg = lane / (W + 1), kind = lane - sg * (W + 1);
+                int lc, ch, cnt;
+                seg_info(sg, hk, h, lc, ch, cnt);
+                if (kind < W - 1) {
+                    tma_load_1d(cst + (kind * nch + lc) * 2, p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch,
+                                cnt * 2, cbar + s);
+                } else if (kind == W - 1) {
+                    tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
+                } else {
+                    tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W, cnt * W * 2,
+                                cbar + s);
+                }
+            }
+            __syncwarp();
             if (lane < nchunk) {
                 const int c = lane * kTileChunk;
                 tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
             } else if (lane == nchunk) {
                 tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
-            } else if (lane == 6 || lane == 7) {  // the 8-aligned group of a (lane 6) or b (lane 7) holding h
-                const uint16_t* srcab = (lane == 6 ? p.a : p.b) + (size_t)seq * Hv + (h & ~7);
-                tma_load_1d(smem + L::AB + s * 32 + (lane - 6) * 16, srcab, 16, cbar + s);
-            } else {
-                const int k = lane - 8;
-                if (k >= 0 && k < nseg * (W + 1)) {
-                    const int sg = k / (W + 1), kind = k - sg * (W + 1);
-                    int lc, ch, cnt;
-                    seg_info(sg, hk, h, lc, ch, cnt);
-                    if (kind < W - 1) {
-                        tma_load_1d(cst + (kind * nch + lc) * 2,
-                                    p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch, cnt * 2, cbar + s);
-                    } else if (kind == W - 1) {
-                        tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
-                    } else {
-                        tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W,
-                                    cnt * W * 2, cbar + s);
-                    }
-                }
             }
         }
         if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land

@@ -255,3 +255,36 @@ def test_deterministic():
     ob, ob32 = b.step(x)
     torch.cuda.synchronize()
     assert torch.equal(oa, ob) and torch.equal(oa32, ob32) and torch.equal(a.state, b.state)
+
+
+@pytest.mark.parametrize("name", ["batch64_small", "tiny_d16", "multitoken"])
+def test_step_replays_from_a_cuda_graph(name):
+    # a decode engine captures the step once and replays it: the replay must give the
+    # same bits as eager launches (both the persistent and the per-tile kernels)
+    base = {"batch64_small": synth.WORKLOADS["batch64"].replace(batch=40, pool_slots=40, num_k_heads=4,
+                                                                 num_v_heads=8),
+            "tiny_d16": synth.WORKLOADS["tiny_d16"],
+            "multitoken": synth.WORKLOADS["multitoken_b32_t16"].replace(batch=4, pool_slots=4)}[name]
+    eager, graphed = GpuRun(base), GpuRun(base)
+    xs = [eager.inputs(s) for s in range(3)]
+    outs_e = [eager.step(x)[1].clone() for x in xs]
+    graphed.step(xs[0])  # first call on the device outside the capture (one-time set-up)
+    graphed.state.copy_(GpuRun(base).state)
+    graphed.conv.copy_(GpuRun(base).conv)
+    shape = (base.batch, base.tokens, base.num_v_heads, base.head_v_dim)
+    outs = [torch.empty(shape, device="cuda") for _ in xs]
+    outb = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        for x, o in zip(xs, outs):
+            gdn.gdn_decode_step(graphed.cfg, x["qkv"], x["a"], x["b"], x["z"], graphed.conv_w, graphed.A_log,
+                                graphed.dt_bias, graphed.norm_w, graphed.conv, graphed.state, graphed.slots, outb, o,
+                                graphed.err)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(outs_e, outs):
+        assert torch.equal(a, b)
+    assert torch.equal(eager.state, graphed.state) and torch.equal(eager.conv, graphed.conv)
+    assert int(graphed.err.item()) == 0

@@ -87,7 +87,7 @@ struct WS {
     static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
     static constexpr int BARS = FLAG + 16;  // full, empty, conv [NSTAGE]; qk [QB]
     static constexpr int TOTAL = BARS + (3 * NSTAGE + QB) * 8;
-    static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && RPL % 4 == 0 && RG * CG == 32, "consumer geometry");
+    static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && (RPL & (RPL - 1)) == 0 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
 };
 
@@ -264,11 +264,34 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
                 const uint32_t q_loc = smem_addr(qkb + q * 2 * DK + qk_lo), bar_loc = smem_addr(qkbar + q);
                 for (int c = 2 * (fw * 32 + lane); c < nch; c += 2 * NFT) {
+                    // the two channels' weights are 2W consecutive bf16 values (W words):
+                    // taps of channel c, then taps of channel c+1
+                    float w0[kMaxConvWidthPersistent] = {0.f, 0.f, 0.f, 0.f};
+                    float w1[kMaxConvWidthPersistent] = {0.f, 0.f, 0.f, 0.f};
+                    auto lo = [](uint32_t x) { return bf16_bits_to_float(x & 0xffffu); };
+                    auto hi = [](uint32_t x) { return bf16_bits_to_float(x >> 16); };
+                    const uint32_t* wq = reinterpret_cast<const uint32_t*>(wts) + (c * W) / 2;
+                    if (W == 4) {
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(wq);
+                        w0[0] = lo(w4.x); w0[1] = hi(w4.x); w0[2] = lo(w4.y); w0[3] = hi(w4.y);
+                        w1[0] = lo(w4.z); w1[1] = hi(w4.z); w1[2] = lo(w4.w); w1[3] = hi(w4.w);
+                    } else if (W == 3) {
+                        const uint32_t a0 = wq[0], a1 = wq[1], a2 = wq[2];
+                        w0[0] = lo(a0); w0[1] = hi(a0); w0[2] = lo(a1);
+                        w1[0] = hi(a1); w1[1] = lo(a2); w1[2] = hi(a2);
+                    } else {
+                        const uint32_t a0 = wq[0], a1 = wq[1];
+                        w0[0] = lo(a0); w0[1] = hi(a0);
+                        w1[0] = lo(a1); w1[1] = hi(a1);
+                    }
                     float acc0 = 0.f, acc1 = 0.f;
-                    for (int j = 0; j < W; ++j) {
-                        const uint32_t xx = *reinterpret_cast<const uint32_t*>(rows + j * nch + c);
-                        acc0 = fmaf(bf16_bits_to_float(wts[c * W + j]), bf16_bits_to_float(xx & 0xffffu), acc0);
-                        acc1 = fmaf(bf16_bits_to_float(wts[(c + 1) * W + j]), bf16_bits_to_float(xx >> 16), acc1);
+#pragma unroll
+                    for (int j = 0; j < kMaxConvWidthPersistent; ++j) {
+                        if (j < W) {
+                            const uint32_t xx = *reinterpret_cast<const uint32_t*>(rows + j * nch + c);
+                            acc0 = fmaf(w0[j], lo(xx), acc0);
+                            acc1 = fmaf(w1[j], hi(xx), acc1);
+                        }
                     }
                     const float s0 = silu(acc0), s1 = silu(acc1);
                     int lc, ch, cnt;
@@ -346,14 +369,18 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 const float* kr = qr + DK;
                 const int row0 = rg * L::RPL;  // this lane's rows: row0 .. row0 + RPL - 1
                 float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
+                // each row group starts its rows at a different offset, so the four
+                // groups read k and q from different banks
+                const int rot = 4 * rg;
 #pragma unroll 2
                 for (int i = 0; i < L::RPL; i += 4) {
-                    const float4 k4 = *reinterpret_cast<const float4*>(kr + row0 + i);
-                    const float4 q4 = *reinterpret_cast<const float4*>(qr + row0 + i);
+                    const int r = row0 + ((i + rot) & (L::RPL - 1));
+                    const float4 k4 = *reinterpret_cast<const float4*>(kr + r);
+                    const float4 q4 = *reinterpret_cast<const float4*>(qr + r);
                     const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float4 x = tl[(size_t)(row0 + i + e) * (DV / 4)];
+                        const float4 x = tl[(size_t)(r + e) * (DV / 4)];
                         mk.x = fmaf(x.x, kk[e], mk.x); mk.y = fmaf(x.y, kk[e], mk.y);
                         mk.z = fmaf(x.z, kk[e], mk.z); mk.w = fmaf(x.w, kk[e], mk.w);
                         mq.x = fmaf(x.x, qq[e], mq.x); mq.y = fmaf(x.y, qq[e], mq.y);
@@ -379,14 +406,15 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                                                        col);
 #pragma unroll 2
                 for (int i = 0; i < L::RPL; i += 4) {
-                    const float4 k4 = *reinterpret_cast<const float4*>(kr + row0 + i);
+                    const int r = row0 + ((i + rot) & (L::RPL - 1));
+                    const float4 k4 = *reinterpret_cast<const float4*>(kr + r);
                     const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        float4 x = tl[(size_t)(row0 + i + e) * (DV / 4)];
+                        float4 x = tl[(size_t)(r + e) * (DV / 4)];
                         x.x = fmaf(st.alpha, x.x, kk[e] * dn.x); x.y = fmaf(st.alpha, x.y, kk[e] * dn.y);
                         x.z = fmaf(st.alpha, x.z, kk[e] * dn.z); x.w = fmaf(st.alpha, x.w, kk[e] * dn.w);
-                        __stcs(Sg + (size_t)(row0 + i + e) * (DV / 4), x);
+                        __stcs(Sg + (size_t)(r + e) * (DV / 4), x);
                     }
                 }
                 // ---- step 8 over the whole head: the team's warps pool their sums of o^2

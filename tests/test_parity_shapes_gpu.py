@@ -73,7 +73,8 @@ PERSISTENT_SHAPES = [
     ("p_d128_g1_w2", 8, 8, 128, 128, 2, 40, 1, 44, 2),
     ("p_dk128_dv64_g4", 2, 8, 128, 64, 4, 80, 1, 80, 2),
     ("p_dk64_dv128_g8_w3", 1, 8, 64, 128, 3, 100, 1, 101, 2),
-    ("p_d32_g2_many", 4, 8, 32, 32, 3, 400, 1, 400, 3),
+    ("p_dk128_dv32_g2_w3", 4, 8, 128, 32, 3, 48, 1, 50, 3),
+    ("p_dk32_dv128_g4", 2, 8, 32, 128, 4, 80, 1, 90, 2),
 ]
 
 

@@ -17,14 +17,13 @@
 //    its v-head's v channels), sends the raw q/k share to every CTA of the cluster
 //    with st.async (completed on the receiver's mbarrier), rolls the conv history,
 //    waits for the other shares, and publishes the q/k norms, k.q and the gates.
-//  * The remaining eight warps, the consumers, take each unit together. Each warp
-//    holds a band of 32 columns (the columns of S are independent under the update)
-//    and a part of the rows. Pass 1 copies the lane's rows of the tile into registers
-//    while accumulating S^T k and S^T q; as soon as k, v, the gates and z are copied
-//    out too, the stage goes back to the loader. The reductions over dk (two shuffle
-//    stages, then the row parts through shared memory), the update (from registers,
-//    streamed to HBM), the RMSNorm, the norm weight and SiLU(z) follow while the next
-//    tiles are already landing.
+//  * The remaining eight warps form teams that take units in turn. A team owns a
+//    unit: each warp holds a band of columns (the columns of S are independent under
+//    the update), reads the tile from shared memory twice (S^T k and S^T q, then the
+//    update, written back in place), reduces over dk with two shuffle stages; one
+//    lane then hands the updated tile to the TMA engine as bulk stores and frees the
+//    stage once they have read it, and the team applies the RMSNorm, the norm weight
+//    and SiLU(z).
 // Every channel's conv history is therefore read and rolled by exactly one CTA, the
 // state is read once and written once, and HBM sees a steady stream of TMA loads and
 // row stores instead of alternating load, compute and store phases.
@@ -61,11 +60,12 @@ struct WS {
     static constexpr int PRODUCER_WARPS = 1 + FINISHER_WARPS;  // the copy-issuing warp, then the conv/gate warps
     static constexpr int NT = 32 * (PRODUCER_WARPS + CONSUMER_WARPS);
     static constexpr int MAX_HV = 128;        // A_log, dt_bias held in shared memory
-    // The consumer warps share each unit: warp w holds column block w % CB (32
-    // columns) and row part w / CB; a lane holds RPL consecutive rows of 4 columns.
-    static constexpr int CB = DV / 32;             // column blocks
-    static constexpr int RP = CONSUMER_WARPS / CB;  // row parts
-    static constexpr int RPL = DK / (RP * 4);       // rows per lane (4 row groups per warp)
+    static constexpr int TEAM_WARPS = DV >= 128 ? 4 : (DV >= 64 ? 2 : 1);
+    static constexpr int NTEAMS = CONSUMER_WARPS / TEAM_WARPS;
+    static constexpr int CPW = DV / TEAM_WARPS;  // columns per consumer warp (32, or 16 when dv = 16)
+    static constexpr int CG = CPW / 4;           // float4 column groups per warp
+    static constexpr int RG = 32 / CG;           // row groups per warp
+    static constexpr int RPL = DK / RG;          // rows per lane
     static constexpr int TILE_BYTES = DK * DV * 4;
     static constexpr int MAXNCH = 2 * DK + DV;   // most conv channels one CTA owns (G = 1)
     // staged conv inputs of one unit: W rows (W-1 history rows, then x) of the CTA's
@@ -85,12 +85,11 @@ struct WS {
     static constexpr int VS = ZB + round_up(NSTAGE * DV * 2, 16);    // [NSTAGE][DV] f32
     static constexpr int SI = VS + NSTAGE * DV * 4;                  // [NSTAGE] StageInfo
     static constexpr int QK = SI + NSTAGE * (int)sizeof(StageInfo);  // [QB][2*DK] f32
-    static constexpr int RED = QK + QB * 2 * DK * 4;                 // [2][RP][CB][2][32] f32 partial sums
-    static constexpr int PART = RED + 2 * RP * CB * 2 * 32 * 4;      // [2][CB] f32 sums of o^2
-    static constexpr int FLAG = PART + round_up(2 * CB * 4, 16);
+    static constexpr int PART = QK + QB * 2 * DK * 4;                // [NTEAMS][2][TEAM_WARPS] f32
+    static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
     static constexpr int BARS = FLAG + 16;  // full, empty, conv [NSTAGE]; qk [QB]
     static constexpr int TOTAL = BARS + (3 * NSTAGE + QB) * 8;
-    static_assert(DV >= 32 && RP >= 1 && RPL >= 4 && (RPL & (RPL - 1)) == 0, "consumer geometry");
+    static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && (RPL & (RPL - 1)) == 0 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
 };
 
@@ -125,7 +124,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     if (tid == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(full + s, 2);                // the producer's copy arrival and its publish arrival
-            mbar_init(empty + s, L::CONSUMER_WARPS);  // one arrival per consumer warp
+            mbar_init(empty + s, L::TEAM_WARPS);   // one arrival per warp of the consuming team
             mbar_init(cbar + s, 1);                // the staged conv inputs
         }
         for (int q = 0; q < QB; ++q) mbar_init(qkbar + q, 1);
@@ -354,131 +353,116 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         }
     } else {
         // ============================== consumers ==============================
-        // All consumer warps take each unit together. Pass 1 pulls the lane's rows of
-        // the tile into registers while accumulating S^T k and S^T q; with k, v, the
-        // gates and z also copied out, the stage goes back to the loader at once, and
-        // the reductions, the update (from registers) and the output follow while the
-        // next tiles stream in.
-        const int cw = warp - L::PRODUCER_WARPS, cb = cw % L::CB, rpart = cw / L::CB;
-        const int rg = lane >> 3, cg = lane & 7;
-        const int col = cb * 32 + 4 * cg;
-        const int row0 = rpart * (DK / L::RP) + rg * L::RPL;  // this lane's rows: row0 .. row0 + RPL - 1
-        const int rot = 4 * rg;  // row groups start at different offsets: k, q reads hit distinct banks
-        const float4 wn4 = make_float4(bf16_bits_to_float(p.norm_w[col]), bf16_bits_to_float(p.norm_w[col + 1]),
-                                       bf16_bits_to_float(p.norm_w[col + 2]), bf16_bits_to_float(p.norm_w[col + 3]));
-        constexpr int NCW = 32 * L::CONSUMER_WARPS;
-        for (int u = 0; u < n; ++u) {
-            const int s = u % NSTAGE, q = u % QB, par = u & 1;
+        const int cw = warp - L::PRODUCER_WARPS, team = cw / L::TEAM_WARPS, wt = cw - team * L::TEAM_WARPS;
+        const int rg = lane / L::CG, cg = lane - rg * L::CG;
+        const int col = wt * L::CPW + 4 * cg;
+        int parity_part = 0;
+        for (int u = team; u < n; u += L::NTEAMS) {
+            const int s = u % NSTAGE, q = u % QB;
             if (!wait(full + s, (u / NSTAGE) & 1)) {
                 fail();
                 break;
             }
             const StageInfo st = si[s];
-            if (st.slot < 0) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty + s);
-                continue;
-            }
-            const int seq = group_seq(u), h = group_hk(u) * G + rank;
-            const float4* tl = reinterpret_cast<const float4*>(tiles + (size_t)s * (DK * DV)) + col / 4;
-            const float* qr = qkb + q * 2 * DK;
-            const float* kr = qr + DK;
-            float4 S[L::RPL];
-            float kreg[L::RPL];
-            float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
+            if (st.slot >= 0) {
+                const int seq = group_seq(u), h = group_hk(u) * G + rank;
+                const uint2 zz = rg == 0 ? *reinterpret_cast<const uint2*>(zb + s * DV + col) : make_uint2(0u, 0u);
+                const float4* tl = reinterpret_cast<const float4*>(tiles + (size_t)s * (DK * DV)) + col / 4;
+                const float* qr = qkb + q * 2 * DK;
+                const float* kr = qr + DK;
+                const int row0 = rg * L::RPL;  // this lane's rows: row0 .. row0 + RPL - 1
+                float4 mk = make_float4(0.f, 0.f, 0.f, 0.f), mq = mk;
+                // each row group starts its rows at a different offset, so the four
+                // groups read k and q from different banks
+                const int rot = 4 * rg;
+#pragma unroll 2
+                for (int i = 0; i < L::RPL; i += 4) {
+                    const int r = row0 + ((i + rot) & (L::RPL - 1));
+                    const float4 k4 = *reinterpret_cast<const float4*>(kr + r);
+                    const float4 q4 = *reinterpret_cast<const float4*>(qr + r);
+                    const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-            for (int i = 0; i < L::RPL; i += 4) {
-                const int r = (i + rot) & (L::RPL - 1);
-                const float4 k4 = *reinterpret_cast<const float4*>(kr + row0 + r);
-                const float4 q4 = *reinterpret_cast<const float4*>(qr + row0 + r);
-                const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 x = tl[(size_t)(row0 + r + e) * (DV / 4)];
-                    S[i + e] = x;
-                    kreg[i + e] = kk[e];
-                    mk.x = fmaf(x.x, kk[e], mk.x); mk.y = fmaf(x.y, kk[e], mk.y);
-                    mk.z = fmaf(x.z, kk[e], mk.z); mk.w = fmaf(x.w, kk[e], mk.w);
-                    mq.x = fmaf(x.x, qq[e], mq.x); mq.y = fmaf(x.y, qq[e], mq.y);
-                    mq.z = fmaf(x.z, qq[e], mq.z); mq.w = fmaf(x.w, qq[e], mq.w);
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 x = tl[(size_t)(r + e) * (DV / 4)];
+                        mk.x = fmaf(x.x, kk[e], mk.x); mk.y = fmaf(x.y, kk[e], mk.y);
+                        mk.z = fmaf(x.z, kk[e], mk.z); mk.w = fmaf(x.w, kk[e], mk.w);
+                        mq.x = fmaf(x.x, qq[e], mq.x); mq.y = fmaf(x.y, qq[e], mq.y);
+                        mq.z = fmaf(x.z, qq[e], mq.z); mq.w = fmaf(x.w, qq[e], mq.w);
+                    }
                 }
-            }
-            const float4 vv = *reinterpret_cast<const float4*>(vsb + s * DV + col);
-            const uint2 zz = *reinterpret_cast<const uint2*>(zb + s * DV + col);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty + s);  // this warp is done with the stage
-            // ---- S^T k, S^T q over dk: the warp's four row groups, then the row parts
 #pragma unroll
-            for (int off = 8; off < 32; off <<= 1) {
-                mk.x += __shfl_xor_sync(0xffffffffu, mk.x, off); mk.y += __shfl_xor_sync(0xffffffffu, mk.y, off);
-                mk.z += __shfl_xor_sync(0xffffffffu, mk.z, off); mk.w += __shfl_xor_sync(0xffffffffu, mk.w, off);
-                mq.x += __shfl_xor_sync(0xffffffffu, mq.x, off); mq.y += __shfl_xor_sync(0xffffffffu, mq.y, off);
-                mq.z += __shfl_xor_sync(0xffffffffu, mq.z, off); mq.w += __shfl_xor_sync(0xffffffffu, mq.w, off);
-            }
-            if (L::RP > 1) {
-                float* rb = reinterpret_cast<float*>(smem + L::RED) + par * (L::RP * L::CB * 2 * 32);
-                if (rg == 0) {
-                    reinterpret_cast<float4*>(rb + ((rpart * L::CB + cb) * 2 + 0) * 32)[cg] = mk;
-                    reinterpret_cast<float4*>(rb + ((rpart * L::CB + cb) * 2 + 1) * 32)[cg] = mq;
+                for (int off = L::CG; off < 32; off <<= 1) {
+                    mk.x += __shfl_xor_sync(0xffffffffu, mk.x, off); mk.y += __shfl_xor_sync(0xffffffffu, mk.y, off);
+                    mk.z += __shfl_xor_sync(0xffffffffu, mk.z, off); mk.w += __shfl_xor_sync(0xffffffffu, mk.w, off);
+                    mq.x += __shfl_xor_sync(0xffffffffu, mq.x, off); mq.y += __shfl_xor_sync(0xffffffffu, mq.y, off);
+                    mq.z += __shfl_xor_sync(0xffffffffu, mq.z, off); mq.w += __shfl_xor_sync(0xffffffffu, mq.w, off);
                 }
-                named_barrier(1, NCW);
-                mk = make_float4(0.f, 0.f, 0.f, 0.f);
-                mq = mk;
+                const float4 vv = *reinterpret_cast<const float4*>(vsb + s * DV + col);
+                const float am = st.alpha * st.nk, aq = st.alpha * st.nq;
+                float4 d, o;
+                d.x = st.beta * fmaf(-am, mk.x, vv.x); d.y = st.beta * fmaf(-am, mk.y, vv.y);
+                d.z = st.beta * fmaf(-am, mk.z, vv.z); d.w = st.beta * fmaf(-am, mk.w, vv.w);
+                o.x = fmaf(aq, mq.x, d.x * st.kq); o.y = fmaf(aq, mq.y, d.y * st.kq);
+                o.z = fmaf(aq, mq.z, d.z * st.kq); o.w = fmaf(aq, mq.w, d.w * st.kq);
+                const float4 dn = make_float4(d.x * st.nk, d.y * st.nk, d.z * st.nk, d.w * st.nk);
+                // the updated rows go back into the stage; the TMA engine stores the tile
+                float4* tw = const_cast<float4*>(tl);
+#pragma unroll 2
+                for (int i = 0; i < L::RPL; i += 4) {
+                    const int r = row0 + ((i + rot) & (L::RPL - 1));
+                    const float4 k4 = *reinterpret_cast<const float4*>(kr + r);
+                    const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-                for (int r2 = 0; r2 < L::RP; ++r2) {
-                    const float4 a = reinterpret_cast<const float4*>(rb + ((r2 * L::CB + cb) * 2 + 0) * 32)[cg];
-                    const float4 b = reinterpret_cast<const float4*>(rb + ((r2 * L::CB + cb) * 2 + 1) * 32)[cg];
-                    mk.x += a.x; mk.y += a.y; mk.z += a.z; mk.w += a.w;
-                    mq.x += b.x; mq.y += b.y; mq.z += b.z; mq.w += b.w;
+                    for (int e = 0; e < 4; ++e) {
+                        float4 x = tl[(size_t)(r + e) * (DV / 4)];
+                        x.x = fmaf(st.alpha, x.x, kk[e] * dn.x); x.y = fmaf(st.alpha, x.y, kk[e] * dn.y);
+                        x.z = fmaf(st.alpha, x.z, kk[e] * dn.z); x.w = fmaf(st.alpha, x.w, kk[e] * dn.w);
+                        tw[(size_t)(r + e) * (DV / 4)] = x;
+                    }
                 }
-            }
-            const float am = st.alpha * st.nk, aq = st.alpha * st.nq;
-            float4 d, o;
-            d.x = st.beta * fmaf(-am, mk.x, vv.x); d.y = st.beta * fmaf(-am, mk.y, vv.y);
-            d.z = st.beta * fmaf(-am, mk.z, vv.z); d.w = st.beta * fmaf(-am, mk.w, vv.w);
-            o.x = fmaf(aq, mq.x, d.x * st.kq); o.y = fmaf(aq, mq.y, d.y * st.kq);
-            o.z = fmaf(aq, mq.z, d.z * st.kq); o.w = fmaf(aq, mq.w, d.w * st.kq);
-            const float4 dn = make_float4(d.x * st.nk, d.y * st.nk, d.z * st.nk, d.w * st.nk);
-            // ---- the update, from registers, streamed to HBM
-            float4* Sg = reinterpret_cast<float4*>(p.state_pool + ((size_t)st.slot * Hv + h) * (size_t)(DK * DV) + col);
-#pragma unroll
-            for (int i = 0; i < L::RPL; i += 4) {
-                const int r = (i + rot) & (L::RPL - 1);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float4 x = S[i + e];
-                    const float ki = kreg[i + e];
-                    x.x = fmaf(st.alpha, x.x, ki * dn.x); x.y = fmaf(st.alpha, x.y, ki * dn.y);
-                    x.z = fmaf(st.alpha, x.z, ki * dn.z); x.w = fmaf(st.alpha, x.w, ki * dn.w);
-                    __stcs(Sg + (size_t)(row0 + r + e) * (DV / 4), x);
-                }
-            }
-            // ---- step 8 over the whole head (the row-part-0 warps hold every column once)
-            float* pt = reinterpret_cast<float*>(smem + L::PART) + par * L::CB;
-            if (rpart == 0) {
+                fence_proxy_async_smem();  // the bulk store (async proxy) must see these writes
+                // ---- step 8 over the whole head: the team's warps pool their sums of o^2
                 float ss = rg == 0 ? o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w : 0.f;
 #pragma unroll
-                for (int off = 1; off < 8; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                if (lane == 0) pt[cb] = ss;
-            }
-            named_barrier(1, NCW);
-            if (rpart == 0 && rg == 0) {
+                for (int off = 1; off < L::CG; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                float* pt = part + (team * 2 + parity_part) * L::TEAM_WARPS;
+                if (lane == 0) pt[wt] = ss;
+                if (L::TEAM_WARPS > 1) named_barrier(1 + team, 32 * L::TEAM_WARPS);
+                else __syncwarp();
+                if (wt == 0 && lane == 0) {  // the whole updated tile back to the pool, then free the stage
+                    char* dstg = reinterpret_cast<char*>(p.state_pool + ((size_t)st.slot * Hv + h) * (size_t)(DK * DV));
+                    const char* srcs = reinterpret_cast<const char*>(tiles + (size_t)s * (DK * DV));
+                    for (int c = 0; c < L::TILE_BYTES; c += kTileChunk)
+                        tma_store_1d(dstg + c, srcs + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c));
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
                 float tot = 0.f;
 #pragma unroll
-                for (int w = 0; w < L::CB; ++w) tot += pt[w];
-                const float inv = rsqrtf(tot / (float)DV + p.sh.rms_eps);
-                const float y0 = o.x * inv * wn4.x * silu(bf16_bits_to_float(zz.x & 0xffffu));
-                const float y1 = o.y * inv * wn4.y * silu(bf16_bits_to_float(zz.x >> 16));
-                const float y2 = o.z * inv * wn4.z * silu(bf16_bits_to_float(zz.y & 0xffffu));
-                const float y3 = o.w * inv * wn4.w * silu(bf16_bits_to_float(zz.y >> 16));
-                const size_t oi = ((size_t)seq * Hv + h) * DV + col;
-                uint2 packed;
-                packed.x = (uint32_t)float_to_bf16_bits(y0) | ((uint32_t)float_to_bf16_bits(y1) << 16);
-                packed.y = (uint32_t)float_to_bf16_bits(y2) | ((uint32_t)float_to_bf16_bits(y3) << 16);
-                *reinterpret_cast<uint2*>(p.out + oi) = packed;
-                if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + oi) = make_float4(y0, y1, y2, y3);
+                for (int w = 0; w < L::TEAM_WARPS; ++w) tot += pt[w];
+                if (rg == 0) {
+                    const float inv = rsqrtf(tot / (float)DV + p.sh.rms_eps);
+                    const uint2 ww = *reinterpret_cast<const uint2*>(p.norm_w + col);
+                    const float y0 = o.x * inv * bf16_bits_to_float(ww.x & 0xffffu) * silu(bf16_bits_to_float(zz.x & 0xffffu));
+                    const float y1 = o.y * inv * bf16_bits_to_float(ww.x >> 16) * silu(bf16_bits_to_float(zz.x >> 16));
+                    const float y2 = o.z * inv * bf16_bits_to_float(ww.y & 0xffffu) * silu(bf16_bits_to_float(zz.y & 0xffffu));
+                    const float y3 = o.w * inv * bf16_bits_to_float(ww.y >> 16) * silu(bf16_bits_to_float(zz.y >> 16));
+                    const size_t oi = ((size_t)seq * Hv + h) * DV + col;
+                    uint2 packed;
+                    packed.x = (uint32_t)float_to_bf16_bits(y0) | ((uint32_t)float_to_bf16_bits(y1) << 16);
+                    packed.y = (uint32_t)float_to_bf16_bits(y2) | ((uint32_t)float_to_bf16_bits(y3) << 16);
+                    *reinterpret_cast<uint2*>(p.out + oi) = packed;
+                    if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + oi) = make_float4(y0, y1, y2, y3);
+                }
+                parity_part ^= 1;
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
             }
         }
+        if (wt == 0 && lane == 0) bulk_wait_all();  // this lane's tile stores have completed
     }
     __syncthreads();
     cluster_arrive_release();  // no CTA leaves while a peer may still send to it
@@ -523,18 +507,15 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
     return cudaLaunchKernelEx(&cfg, kern, a, ncl);
 }
 
-template <int DK, int DV>
-cudaError_t ws_if_geometry(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap) {
-    if constexpr (DV >= 32 && DK * DV >= 4096) return launch_ws_tile<DK, DV>(a, G, stream, query_only, cap);
-    return cudaErrorInvalidValue;
-}
-
 template <int DK>
 cudaError_t ws_dispatch(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap) {
     switch (a.sh.dv) {
-        case 32: return ws_if_geometry<DK, 32>(a, G, stream, query_only, cap);
-        case 64: return ws_if_geometry<DK, 64>(a, G, stream, query_only, cap);
-        case 128: return ws_if_geometry<DK, 128>(a, G, stream, query_only, cap);
+        case 16:
+            if constexpr (DK >= 32) return launch_ws_tile<DK, 16>(a, G, stream, query_only, cap);
+            return cudaErrorInvalidValue;
+        case 32: return launch_ws_tile<DK, 32>(a, G, stream, query_only, cap);
+        case 64: return launch_ws_tile<DK, 64>(a, G, stream, query_only, cap);
+        case 128: return launch_ws_tile<DK, 128>(a, G, stream, query_only, cap);
     }
     return cudaErrorInvalidValue;
 }
@@ -557,9 +538,8 @@ bool persistent_supported(const DecodeArgs& a) {
     // the q/k share of each CTA must be a whole number of 16-byte bf16 runs for the
     // bulk copies of the conv inputs
     const int G = a.sh.Hv / a.sh.Hk;
-    // consumer geometry: at least 4 rows per lane (dk * dv >= 4096 with dv >= 32)
     return a.T == 1 && a.sh.W <= kMaxConvWidthPersistent && G <= 8 && (2 * a.sh.dk) % (8 * G) == 0 &&
-           a.sh.Hv % 8 == 0 && a.sh.Hv <= 128 && a.sh.dv >= 32 && a.sh.dk * a.sh.dv >= 4096;
+           a.sh.Hv % 8 == 0 && a.sh.Hv <= 128 && (a.sh.dv >= 32 || a.sh.dk >= 32);
 }
 
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters) {

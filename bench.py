@@ -269,9 +269,10 @@ def main():
     xs = [{k: bf16(v) for k, v in synth.step_inputs(wlr, s).items()} for s in range(n_inputs)]
     out = torch.empty(wl.batch, wl.tokens, wl.num_v_heads, wl.head_v_dim, dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = gdn.decode_workspace(dev)  # dynamic spread of the sequences over the SMs
     stream = torch.cuda.current_stream(dev)
     plans = [gdn.DecodePlan(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
-                            convs[i % args.pools], states[i % args.pools], slots, out, None, err, stream)
+                            convs[i % args.pools], states[i % args.pools], slots, out, None, err, ws, stream)
              for i, x in enumerate(xs)]
 
     def barrier():
@@ -305,7 +306,7 @@ def main():
             for i in range(count):
                 x = xs[i]
                 gdn.gdn_decode_step(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
-                                    convs[i % args.pools], states[i % args.pools], slots, out, None, err)
+                                    convs[i % args.pools], states[i % args.pools], slots, out, None, err, ws)
         graphs.append(g)
     for _ in range(max(1, args.warmup // n_inputs)):
         graphs[0].replay()
@@ -345,7 +346,7 @@ def main():
         dx = {k: torch.empty_like(v) for k, v in xs[0].items()}
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         eplans = [gdn.DecodePlan(cfg, dx["qkv"], dx["a"], dx["b"], dx["z"], conv_w, A_log, dt_bias, norm_w,
-                                 convs[p], states[p], slots, out, None, err, stream) for p in range(args.pools)]
+                                 convs[p], states[p], slots, out, None, err, ws, stream) for p in range(args.pools)]
         h2d = sum(v.numel() * v.element_size() for v in hx[0].values())
         d2h = hout.numel() * hout.element_size()
 

@@ -27,7 +27,7 @@ GDN_DEVICE_ERR_SLOT_RANGE = 1
 GDN_DEVICE_ERR_TIMEOUT = 2
 
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
-           "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
+           "gdn_decode_workspace_bytes", "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
 
 
 class GdnConfig(ctypes.Structure):
@@ -68,7 +68,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_conv_update.argtypes = [cfgp, i32, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
         L.gdn_recurrent_step.argtypes = [cfgp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
         L.gdn_gated_rmsnorm.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp]
-        L.gdn_decode_step.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp]
+        L.gdn_decode_step.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_decode_workspace_bytes.argtypes = []
+        L.gdn_decode_workspace_bytes.restype = ctypes.c_size_t
         L.gdn_check_slots_host.argtypes = [vp, i32, i32]
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -106,6 +108,7 @@ def _ptr(t: Optional[torch.Tensor], dtypes, name: str):
 _BF16 = (torch.bfloat16, torch.int16, torch.uint16)
 _F32 = (torch.float32,)
 _I32 = (torch.int32,)
+_WS = (torch.int32, torch.uint8, torch.int64)
 
 
 def _stream(stream, ref: torch.Tensor):
@@ -145,7 +148,7 @@ def gdn_gated_rmsnorm(cfg: GdnConfig, o, z, norm_w, out, out_f32=None, stream=No
 
 
 def gdn_decode_step(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
-                    slots, out, out_f32=None, err_flag=None, stream=None) -> None:
+                    slots, out, out_f32=None, err_flag=None, workspace=None, stream=None) -> None:
     B, T = qkv.shape[0], qkv.shape[1]
     _check(lib().gdn_decode_step(ctypes.byref(cfg), B, T, _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"),
                                  _ptr(b, _BF16, "b"), _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"),
@@ -154,7 +157,16 @@ def gdn_decode_step(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w
                                  _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0],
                                  _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
                                  _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
-                                 _stream(stream, qkv)), "gdn_decode_step")
+                                 _ptr(workspace, _WS, "workspace"), _stream(stream, qkv)), "gdn_decode_step")
+
+
+def decode_workspace_bytes() -> int:
+    return int(lib().gdn_decode_workspace_bytes())
+
+
+def decode_workspace(device) -> torch.Tensor:
+    """A zeroed workspace for gdn_decode_step on `device` (keep one per stream)."""
+    return torch.zeros(decode_workspace_bytes() // 4, dtype=torch.int32, device=device)
 
 
 def gdn_check_slots_host(slots, pool_slots: int) -> int:
@@ -174,16 +186,17 @@ class DecodePlan:
     (the tensors must stay alive and in place while the plan is used)."""
 
     def __init__(self, cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
-                 slots, out, out_f32=None, err_flag=None, stream=None):
+                 slots, out, out_f32=None, err_flag=None, workspace=None, stream=None):
         self._keep = (cfg, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots, out,
-                      out_f32, err_flag)
+                      out_f32, err_flag, workspace)
         self._fn = lib().gdn_decode_step
         self._args = (ctypes.byref(cfg), qkv.shape[0], qkv.shape[1], _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"),
                       _ptr(b, _BF16, "b"), _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"),
                       _ptr(A_log, _F32, "A_log"), _ptr(dt_bias, _F32, "dt_bias"), _ptr(norm_w, _BF16, "norm_w"),
                       _ptr(conv_pool, _BF16, "conv_pool"), _ptr(state_pool, _F32, "state_pool"),
                       state_pool.shape[0], _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
-                      _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"), _stream(stream, qkv))
+                      _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
+                      _ptr(workspace, _WS, "workspace"), _stream(stream, qkv))
 
     def launch(self) -> None:
         st = self._fn(*self._args)

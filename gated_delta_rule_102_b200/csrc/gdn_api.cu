@@ -116,21 +116,23 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
                            const uint16_t* b, const uint16_t* z, const uint16_t* conv_w, const float* A_log,
                            const float* dt_bias, const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
                            int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16, float* out_f32,
-                           int32_t* err_flag, void* stream) {
+                           int32_t* err_flag, void* workspace, void* stream) {
     gdn::Shape sh;
     gdn_status st = check_config(cfg, &sh);
     if (st != GDN_OK) return st;
     if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
     if (B == 0) return GDN_OK;
     if ((st = check_pointers({qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots, out_bf16},
-                             {out_f32, err_flag})) != GDN_OK)
+                             {out_f32, err_flag, workspace})) != GDN_OK)
         return st;
     const int G = sh.Hv / sh.Hk;
     gdn::DecodeArgs d{sh, B, T, pool_slots, gdn::decode_column_splits(B, sh.Hv, G, sh.dv),
                       qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots,
-                      out_bf16, out_f32, err_flag};
+                      out_bf16, out_f32, err_flag, static_cast<unsigned int*>(workspace)};
     return from_cuda(gdn::launch_decode_fused(d, (cudaStream_t)stream));
 }
+
+size_t gdn_decode_workspace_bytes(void) { return 64; }
 
 gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t pool_slots) {
     if (B < 0 || pool_slots < 0 || (B > 0 && !slots_host)) return GDN_ERR_INVALID_ARGUMENT;

@@ -49,9 +49,12 @@ __host__ __device__ constexpr int clampi(int x, int lo, int hi) { return x < lo 
 
 struct StageInfo {  // what the producer publishes for a staged unit
     float alpha, beta, nq, nk, kq;
-    int slot;  // -1: the unit's slot is out of range
-    int pad[2];
+    int slot;   // -1: the unit's slot is out of range
+    int group;  // (sequence, k-head) group of the unit; kEndOfWork: no more units
+    int pad;
 };
+constexpr int kEndOfWork = -1;
+constexpr int kRing = 16;  // group indices relayed from the cluster's rank 0 (dynamic schedule)
 
 template <int DK, int DV>
 struct WS {
@@ -87,8 +90,9 @@ struct WS {
     static constexpr int QK = SI + NSTAGE * (int)sizeof(StageInfo);  // [QB][2*DK] f32
     static constexpr int PART = QK + QB * 2 * DK * 4;                // [NTEAMS][2][TEAM_WARPS] f32
     static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
-    static constexpr int BARS = FLAG + 16;  // full, empty, conv [NSTAGE]; qk [QB]
-    static constexpr int TOTAL = BARS + (3 * NSTAGE + QB) * 8;
+    static constexpr int RING = FLAG + 16;                           // [kRing] int: relayed group indices
+    static constexpr int BARS = RING + kRing * 4;  // full, empty, conv [NSTAGE]; qk [QB]; ring [kRing]
+    static constexpr int TOTAL = BARS + (3 * NSTAGE + QB + kRing) * 8;
     static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && (RPL & (RPL - 1)) == 0 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
 };
@@ -114,11 +118,12 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     uint64_t* empty = full + NSTAGE;
     uint64_t* cbar = empty + NSTAGE;
     uint64_t* qkbar = cbar + NSTAGE;
+    uint64_t* rbar = qkbar + QB;
+    int* ring = reinterpret_cast<int*>(smem + L::RING);
 
     const int Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk, C = p.sh.C, W = p.sh.W;
     const int rank = (int)cluster_ctarank(), cid = blockIdx.x / G;
     const int ngroups = p.B * Hk;
-    const int n = cid < ngroups ? (ngroups - cid + ncl - 1) / ncl : 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     if (tid == 0) {
@@ -128,6 +133,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             mbar_init(cbar + s, 1);                // the staged conv inputs
         }
         for (int q = 0; q < QB; ++q) mbar_init(qkbar + q, 1);
+        for (int r = 0; r < kRing; ++r) mbar_init(rbar + r, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -144,8 +150,6 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     auto wait = [&](uint64_t* bar, uint32_t parity) {
         return mbar_wait_deadline(bar, parity, kWaitTimeoutNs, [&] { return *abort_flag != 0; });
     };
-    auto group_seq = [&](int u) { return (cid + u * ncl) / Hk; };
-    auto group_hk = [&](int u) { return (cid + u * ncl) % Hk; };
     auto slot_ok = [&](int s) { return s >= 0 && s < p.P; };
 
     // This CTA's conv channels, in local order: its share of the k-head's q/k
@@ -174,22 +178,79 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         // ============================== loader ==============================
         // Unit v's copies into stage v % NSTAGE as soon as the stage is free: the
         // state tile and z row (completing on full), the conv inputs and the a/b
-        // groups (completing on cbar). The slot goes along in the stage info.
+        // groups (completing on cbar). The group and slot go along in the stage info.
+        //
+        // Which group unit v is: with a static schedule cid + v * ncl; with the
+        // dynamic schedule, the cluster's rank 0 takes groups from the shared counter
+        // one unit ahead and relays each index to every CTA of the cluster with
+        // st.async (ring of kRing entries), so the CTAs of a cluster walk the same
+        // groups and faster clusters simply take more of them.
         const int conv_bytes = 2 * W * nch * 2 + 32;
-        int slots32 = -1;
-        for (int v = 0; v < n; ++v) {
-            const int s = v % NSTAGE, seq = group_seq(v), hk = group_hk(v), h = hk * G + rank;
-            if ((v & 31) == 0) {  // the next 32 units' slots, one per lane
-                const int u = v + lane;
-                slots32 = u < n ? __ldg(p.slots + group_seq(u)) : -1;
+        const bool dyn = p.sched != nullptr;
+        unsigned int pending = 0;  // rank 0, lane 0: the index to relay next
+        auto relay = [&](int v, unsigned int val) {  // rank 0, lane 0
+            const uint32_t a_loc = smem_addr(ring + (v % kRing)), b_loc = smem_addr(rbar + (v % kRing));
+            for (int r = 0; r < G; ++r)
+                st_async_f32(cluster_map_u32(a_loc, r), __uint_as_float(val), cluster_map_u32(b_loc, r));
+        };
+        auto fetch = [&]() { return atomicAdd(p.sched, 1u); };
+        auto receive = [&](int v) {  // lane-uniform group index of unit v (kEndOfWork past the end)
+            int g;
+            if (!dyn) {
+                g = cid + v * ncl;
+            } else {
+                bool ok = true;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(rbar + (v % kRing), 4);
+                    ok = wait(rbar + (v % kRing), (v / kRing) & 1);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) return -2;
+                g = ring[v % kRing];
             }
-            const int slot = __shfl_sync(0xffffffffu, slots32, v & 31);
+            return g < ngroups ? g : kEndOfWork;
+        };
+        if (dyn && rank == 0 && lane == 0) {
+            const unsigned int f0 = fetch();
+            relay(0, f0);
+            pending = f0 < (unsigned)ngroups ? fetch() : f0;
+        }
+        int g_next = receive(0);
+        int slot_next = g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1;
+        for (int v = 0;; ++v) {
+            const int g = g_next, slot = slot_next;
+            if (g == -2) {
+                fail();
+                break;
+            }
+            if (g != kEndOfWork && dyn && rank == 0 && lane == 0) {  // the index of unit v+1, then fetch for v+2
+                relay(v + 1, pending);
+                if (pending < (unsigned)ngroups) pending = fetch();
+            }
+            if (g == kEndOfWork) {  // one end marker per consumer team
+                bool ok = true;
+                for (int e = 0; e < L::NTEAMS && ok; ++e) {
+                    const int ve = v + e, s = ve % NSTAGE;
+                    if (ve >= NSTAGE && !wait(empty + s, ((ve / NSTAGE) - 1) & 1)) ok = false;
+                    if (ok && lane == 0) {
+                        si[s].group = kEndOfWork;
+                        mbar_arrive(cbar + s);
+                        mbar_arrive(full + s);
+                        mbar_arrive(full + s);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) fail();
+                break;
+            }
+            const int s = v % NSTAGE, seq = g / Hk, hk = g - seq * Hk, h = hk * G + rank;
             if (v >= NSTAGE && !wait(empty + s, ((v / NSTAGE) - 1) & 1)) {
                 fail();
                 break;
             }
             const bool valid = slot_ok(slot);
             if (lane == 0) {
+                si[s].group = g;
                 si[s].slot = valid ? slot : -1;
                 if (valid) {
                     mbar_arrive_expect_tx(full + s, L::TILE_BYTES + DV * 2);
@@ -200,37 +261,42 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 }
             }
             __syncwarp();
-            if (!valid) continue;
-            constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
-            const char* src = reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h) * (size_t)(DK * DV));
-            char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
-            unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
-            // the small conv inputs first: the finishers need them long before the
-            // consumers need the tile
-            if (lane == 30 || lane == 31) {  // the 8-aligned group of a (lane 30) or b (lane 31) holding h
-                const uint16_t* srcab = (lane == 30 ? p.a : p.b) + (size_t)seq * Hv + (h & ~7);
-                tma_load_1d(smem + L::AB + s * 32 + (lane - 30) * 16, srcab, 16, cbar + s);
-            } else if (lane < nseg * (W + 1)) {
-                const int sg = lane / (W + 1), kind = lane - sg * (W + 1);
-                int lc, ch, cnt;
-                seg_info(sg, hk, h, lc, ch, cnt);
-                if (kind < W - 1) {
-                    tma_load_1d(cst + (kind * nch + lc) * 2, p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch,
-                                cnt * 2, cbar + s);
-                } else if (kind == W - 1) {
-                    tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
-                } else {
-                    tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W, cnt * W * 2,
-                                cbar + s);
+            if (valid) {
+                constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
+                const char* src =
+                    reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h) * (size_t)(DK * DV));
+                char* dst = reinterpret_cast<char*>(tiles) + (size_t)s * L::TILE_BYTES;
+                unsigned char* cst = smem + L::CONV + s * L::CSTAGE;
+                // the small conv inputs first: the finishers need them long before the
+                // consumers need the tile
+                if (lane == 30 || lane == 31) {  // the 8-aligned group of a (lane 30) or b (lane 31) holding h
+                    const uint16_t* srcab = (lane == 30 ? p.a : p.b) + (size_t)seq * Hv + (h & ~7);
+                    tma_load_1d(smem + L::AB + s * 32 + (lane - 30) * 16, srcab, 16, cbar + s);
+                } else if (lane < nseg * (W + 1)) {
+                    const int sg = lane / (W + 1), kind = lane - sg * (W + 1);
+                    int lc, ch, cnt;
+                    seg_info(sg, hk, h, lc, ch, cnt);
+                    if (kind < W - 1) {
+                        tma_load_1d(cst + (kind * nch + lc) * 2,
+                                    p.conv_pool + ((size_t)slot * (W - 1) + kind) * C + ch, cnt * 2, cbar + s);
+                    } else if (kind == W - 1) {
+                        tma_load_1d(cst + ((W - 1) * nch + lc) * 2, p.qkv + (size_t)seq * C + ch, cnt * 2, cbar + s);
+                    } else {
+                        tma_load_1d(cst + round_up(W * nch * 2, 16) + lc * W * 2, p.conv_w + (size_t)ch * W,
+                                    cnt * W * 2, cbar + s);
+                    }
+                }
+                __syncwarp();
+                if (lane < nchunk) {
+                    const int c = lane * kTileChunk;
+                    tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
+                } else if (lane == nchunk) {
+                    tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
                 }
             }
-            __syncwarp();
-            if (lane < nchunk) {
-                const int c = lane * kTileChunk;
-                tma_load_1d(dst + c, src + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c), full + s);
-            } else if (lane == nchunk) {
-                tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
-            }
+            // the next unit's group and slot, while this unit's copies are in flight
+            g_next = receive(v + 1);
+            slot_next = g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1;
         }
         if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
             for (int i = 0; i < 1024; ++i) __nanosleep(64);
@@ -251,12 +317,15 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             }
         }
         named_barrier(15, NFT);
-        for (int v = 0; v < n; ++v) {
-            const int s = v % NSTAGE, q = v % QB, hk = group_hk(v), h = hk * G + rank;
+        for (int v = 0;; ++v) {
+            const int s = v % NSTAGE, q = v % QB;
             if (!wait(cbar + s, (v / NSTAGE) & 1)) {
                 fail();
                 break;
             }
+            const int g = si[s].group;
+            if (g == kEndOfWork) break;
+            const int hk = g % Hk, h = hk * G + rank;
             const int slot = si[s].slot;
             const bool valid = slot >= 0;
             if (valid) {
@@ -357,15 +426,16 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         const int rg = lane / L::CG, cg = lane - rg * L::CG;
         const int col = wt * L::CPW + 4 * cg;
         int parity_part = 0;
-        for (int u = team; u < n; u += L::NTEAMS) {
+        for (int u = team;; u += L::NTEAMS) {
             const int s = u % NSTAGE, q = u % QB;
             if (!wait(full + s, (u / NSTAGE) & 1)) {
                 fail();
                 break;
             }
             const StageInfo st = si[s];
+            if (st.group == kEndOfWork) break;
             if (st.slot >= 0) {
-                const int seq = group_seq(u), h = group_hk(u) * G + rank;
+                const int seq = st.group / Hk, h = (st.group - seq * Hk) * G + rank;
                 const uint2 zz = rg == 0 ? *reinterpret_cast<const uint2*>(zb + s * DV + col) : make_uint2(0u, 0u);
                 const float4* tl = reinterpret_cast<const float4*>(tiles + (size_t)s * (DK * DV)) + col / 4;
                 const float* qr = qkb + q * 2 * DK;
@@ -465,6 +535,13 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         if (wt == 0 && lane == 0) bulk_wait_all();  // this lane's tile stores have completed
     }
     __syncthreads();
+    if (p.sched && tid == 0) {  // the last CTA out leaves the counters at zero for the next call
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+        }
+    }
     cluster_arrive_release();  // no CTA leaves while a peer may still send to it
     cluster_wait_acquire();
 }
@@ -501,7 +578,7 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
     if (cap_out) *cap_out = cap;
     if (query_only) return cudaSuccess;
     const int ngroups = a.B * a.sh.Hk;
-    const int ncl = ngroups < cap ? ngroups : cap;
+    const int ncl = ngroups < cap ? ngroups : cap;  // the dynamic schedule needs ncl <= co-resident clusters too
     if (ncl <= 0) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3((unsigned)(ncl * G));
     return cudaLaunchKernelEx(&cfg, kern, a, ncl);

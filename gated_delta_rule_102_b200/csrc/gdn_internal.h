@@ -31,6 +31,7 @@ struct DecodeArgs {
     uint16_t* out;
     float* out_f32;
     int32_t* err_flag;
+    unsigned int* sched;  // nullable: two zeroed counters for the dynamic schedule of the persistent kernel
 };
 
 struct ConvArgs {

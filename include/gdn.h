@@ -136,13 +136,24 @@ gdn_status gdn_gated_rmsnorm(const gdn_config* cfg, int32_t rows, const float* o
  *   out_bf16 [B][T][Hv][dv] bf16
  *   out_f32  [B][T][Hv][dv] fp32, nullable (the unrounded output, for parity checks)
  *   err_flag nullable device int32
+ *   workspace nullable device buffer of gdn_decode_workspace_bytes() bytes, zeroed by
+ *            the caller once before its first use; every call leaves it zeroed again.
+ *            With it, large single-token batches are spread over the SMs dynamically
+ *            (faster SMs take more sequences); without it the split is static. The
+ *            results are the same bits either way. Calls that may run at the same
+ *            time on the GPU need separate workspaces.
+ * The first call on a device (per shape) queries the device once and sets a kernel
+ * attribute; make it before capturing the call into a CUDA graph.
  */
 gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv,
                            const uint16_t* a, const uint16_t* b, const uint16_t* z,
                            const uint16_t* conv_w, const float* A_log, const float* dt_bias,
                            const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
                            int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
-                           float* out_f32, int32_t* err_flag, void* stream);
+                           float* out_f32, int32_t* err_flag, void* workspace, void* stream);
+
+/* Bytes of the optional workspace of gdn_decode_step (a multiple of 16). */
+size_t gdn_decode_workspace_bytes(void);
 
 /*
  * Host-side check of a HOST copy of slots[]: GDN_OK when all B values are distinct

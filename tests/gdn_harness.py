@@ -36,8 +36,10 @@ def cfg_of(wl: synth.Workload) -> gdn.GdnConfig:
 class GpuRun:
     """The workload on the GPU: weights, pools and slots resident on the device."""
 
-    def __init__(self, wl: synth.Workload, device="cuda", state0: Optional[np.ndarray] = None):
+    def __init__(self, wl: synth.Workload, device="cuda", state0: Optional[np.ndarray] = None,
+                 dynamic: bool = True):
         self.wl, self.device = wl, device
+        self.workspace = gdn.decode_workspace(device) if dynamic else None
         self.cfg = cfg_of(wl)
         w = synth.weights(wl)
         self.conv_w = bf16_dev(w["conv_w"], device)
@@ -61,7 +63,7 @@ class GpuRun:
         out = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
         out32 = torch.empty(shape, dtype=torch.float32, device=self.device) if want_f32 else None
         gdn.gdn_decode_step(self.cfg, x["qkv"], x["a"], x["b"], x["z"], self.conv_w, self.A_log, self.dt_bias,
-                            self.norm_w, self.conv, self.state, self.slots, out, out32, self.err)
+                            self.norm_w, self.conv, self.state, self.slots, out, out32, self.err, self.workspace)
         return out, out32
 
 

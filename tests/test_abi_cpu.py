@@ -78,10 +78,10 @@ def good_cfg(**kw):
     return gdn.GdnConfig.make(**base)
 
 
-def decode(L, cfg, B=4, T=1, ptrs=None, pool=8, out_f32=None, err=None):
+def decode(L, cfg, B=4, T=1, ptrs=None, pool=8, out_f32=None, err=None, ws=None):
     p = [FAKE] * 10 if ptrs is None else ptrs
     return L.gdn_decode_step(ctypes.byref(cfg) if cfg is not None else None, B, T, *p, pool, FAKE, FAKE,
-                             out_f32, err, None)
+                             out_f32, err, ws, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -117,6 +117,8 @@ def test_decode_rejects_bad_sizes_and_pointers(L):
         assert decode(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
     assert decode(L, cfg, out_f32=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
     assert decode(L, cfg, err=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    assert decode(L, cfg, ws=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    assert gdn.decode_workspace_bytes() % 16 == 0 and gdn.decode_workspace_bytes() >= 8
 
 
 def test_empty_batch_is_a_no_op(L):

@@ -95,10 +95,11 @@ def test_persistent_path_bad_slot():
     out = torch.full(shape, 3.0, dtype=torch.bfloat16, device="cuda")
     out32 = torch.full(shape, 3.0, device="cuda")
     gdn.gdn_decode_step(g.cfg, x["qkv"], x["a"], x["b"], x["z"], g.conv_w, g.A_log, g.dt_bias, g.norm_w,
-                        g.conv, g.state, g.slots, out, out32, g.err)
+                        g.conv, g.state, g.slots, out, out32, g.err, g.workspace)
     torch.cuda.synchronize()
     assert int(g.err.item()) == gdn.GDN_DEVICE_ERR_SLOT_RANGE
     assert torch.all(out32[17] == 3.0)
+    assert int(g.workspace.abs().sum().item()) == 0
     skipped = int(g.slots_np[17])  # the slot sequence 17 would have used: nobody touched it
     assert torch.equal(g.state[skipped], state0[skipped]) and torch.equal(g.conv[skipped], conv0[skipped])
     rows = [0, 16, 18, 39]
@@ -282,10 +283,27 @@ def test_step_replays_from_a_cuda_graph(name):
         for x, o in zip(xs, outs):
             gdn.gdn_decode_step(graphed.cfg, x["qkv"], x["a"], x["b"], x["z"], graphed.conv_w, graphed.A_log,
                                 graphed.dt_bias, graphed.norm_w, graphed.conv, graphed.state, graphed.slots, outb, o,
-                                graphed.err)
+                                graphed.err, graphed.workspace)
     g.replay()
     torch.cuda.synchronize()
     for a, b in zip(outs_e, outs):
         assert torch.equal(a, b)
     assert torch.equal(eager.state, graphed.state) and torch.equal(eager.conv, graphed.conv)
     assert int(graphed.err.item()) == 0
+
+
+@pytest.mark.parametrize("spec", [PERSISTENT_SHAPES[0], PERSISTENT_SHAPES[2]], ids=["g2", "g4"])
+def test_dynamic_and_static_schedules_agree(spec):
+    # the workspace only changes which SM takes which sequence: the same bits come out,
+    # and the workspace is left zeroed for the next call
+    name, Hk, Hv, dk, dv, W, B, T, P, steps = spec
+    wl = wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed=77)
+    dyn, sta = GpuRun(wl, dynamic=True), GpuRun(wl, dynamic=False)
+    for s in range(steps):
+        x = dyn.inputs(s)
+        od, od32 = dyn.step(x)
+        os_, os32 = sta.step(x)
+        torch.cuda.synchronize()
+        assert torch.equal(od32, os32) and torch.equal(od, os_)
+        assert int(dyn.workspace.abs().sum().item()) == 0
+    assert torch.equal(dyn.state, sta.state) and torch.equal(dyn.conv, sta.conv)

@@ -100,6 +100,17 @@ struct WS {
 __device__ __forceinline__ void named_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
 }
+// Named barrier that also returns whether `pred` held in every participating thread:
+// warps sharing later named barriers leave a loop together or not at all.
+__device__ __forceinline__ bool named_barrier_and(int id, int threads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(WS<DK, DV>::NT, 1)
@@ -319,10 +330,9 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         named_barrier(15, NFT);
         for (int v = 0;; ++v) {
             const int s = v % NSTAGE, q = v % QB;
-            if (!wait(cbar + s, (v / NSTAGE) & 1)) {
-                fail();
-                break;
-            }
+            bool ok = wait(cbar + s, (v / NSTAGE) & 1);
+            if (!ok) fail();
+            if (!named_barrier_and(15, NFT, ok && !*abort_flag)) break;  // every finisher warp leaves together
             const int g = si[s].group;
             if (g == kEndOfWork) break;
             const int hk = g % Hk, h = hk * G + rank;
@@ -387,8 +397,8 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 else mbar_arrive(qkbar + q);
             }
             if (!wait(qkbar + q, (v / QB) & 1)) {
-                fail();
-                break;
+                fail();  // the other finisher warps see the abort at the next agreement
+                continue;
             }
             if (valid) {
                 const float* qr = qkb + q * 2 * DK;
@@ -428,10 +438,11 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         int parity_part = 0;
         for (int u = team;; u += L::NTEAMS) {
             const int s = u % NSTAGE, q = u % QB;
-            if (!wait(full + s, (u / NSTAGE) & 1)) {
-                fail();
-                break;
-            }
+            bool ok = wait(full + s, (u / NSTAGE) & 1);
+            if (!ok) fail();
+            if (L::TEAM_WARPS > 1) ok = named_barrier_and(1 + team, 32 * L::TEAM_WARPS, ok && !*abort_flag);
+            else ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+            if (!ok) break;  // the team's warps leave together
             const StageInfo st = si[s];
             if (st.group == kEndOfWork) break;
             if (st.slot >= 0) {

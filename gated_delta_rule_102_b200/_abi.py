@@ -27,7 +27,8 @@ GDN_DEVICE_ERR_SLOT_RANGE = 1
 GDN_DEVICE_ERR_TIMEOUT = 2
 
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
-           "gdn_decode_workspace_bytes", "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
+           "gdn_decode_workspace_bytes", "gdn_decode_step_static_scratch", "gdn_decode_static_scratch_bytes",
+           "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
 
 
 class GdnConfig(ctypes.Structure):
@@ -71,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_step.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp, vp]
         L.gdn_decode_workspace_bytes.argtypes = []
         L.gdn_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.gdn_decode_step_static_scratch.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp]
+        L.gdn_decode_step_static_scratch.restype = ctypes.c_int32
+        L.gdn_decode_static_scratch_bytes.argtypes = []
+        L.gdn_decode_static_scratch_bytes.restype = ctypes.c_size_t
         L.gdn_check_slots_host.argtypes = [vp, i32, i32]
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -158,6 +163,24 @@ def gdn_decode_step(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w
                                  _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
                                  _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
                                  _ptr(workspace, _WS, "workspace"), _stream(stream, qkv)), "gdn_decode_step")
+
+
+def gdn_decode_step_static_scratch(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool,
+                                   state_pool, slots, out, out_f32=None, err_flag=None, stream=None) -> None:
+    """gdn_decode_step for callers that cannot allocate: the library's own fixed device
+    scratch replaces the workspace (calls that overlap on the GPU race on it)."""
+    B, T = qkv.shape[0], qkv.shape[1]
+    _check(lib().gdn_decode_step_static_scratch(
+        ctypes.byref(cfg), B, T, _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"), _ptr(b, _BF16, "b"),
+        _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"), _ptr(A_log, _F32, "A_log"),
+        _ptr(dt_bias, _F32, "dt_bias"), _ptr(norm_w, _BF16, "norm_w"), _ptr(conv_pool, _BF16, "conv_pool"),
+        _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0], _ptr(slots, _I32, "slots"),
+        _ptr(out, _BF16, "out"), _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
+        _stream(stream, qkv)), "gdn_decode_step_static_scratch")
+
+
+def decode_static_scratch_bytes() -> int:
+    return int(lib().gdn_decode_static_scratch_bytes())
 
 
 def decode_workspace_bytes() -> int:

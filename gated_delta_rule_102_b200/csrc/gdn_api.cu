@@ -7,6 +7,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <vector>
 
 #include "gdn.h"
@@ -133,6 +134,63 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
 }
 
 size_t gdn_decode_workspace_bytes(void) { return 64; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Scratch for gdn_decode_step_static_scratch: the workspace of gdn_decode_step kept
+// in this library's own device memory, so callers that cannot allocate still get the
+// dynamic spread of sequences over the SMs. Every GPU that loads the library holds
+// this array until the process exits; all calls on a device share it.
+namespace {
+constexpr size_t kStaticScratchBytes = 256;  // fixed maximum
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxScratchDevices];  // device address of g_decode_scratch, per device
+
+// Once per device, with that device current: the array's device address (in host
+// code the symbol itself only names a host-side stand-in).
+gdn_status static_scratch_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxScratchDevices) return GDN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return GDN_ERR_CUDA;
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return GDN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_decode_step_static_scratch(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv,
+                                          const uint16_t* a, const uint16_t* b, const uint16_t* z,
+                                          const uint16_t* conv_w, const float* A_log, const float* dt_bias,
+                                          const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                                          int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
+                                          float* out_f32, int32_t* err_flag, void* stream) {
+    const size_t need = gdn_decode_workspace_bytes();
+    if (need > kStaticScratchBytes) return GDN_ERR_UNSUPPORTED;  // the fixed array is too small for this build
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    void* scratch = nullptr;
+    if ((st = static_scratch_address(&scratch)) != GDN_OK) return st;
+    // the counters must start at zero; clear them in stream order before the launch
+    if (cudaMemsetAsync(scratch, 0, need, (cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
+    return gdn_decode_step(cfg, B, T, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
+                           pool_slots, slots, out_bf16, out_f32, err_flag, scratch, stream);
+}
+
+size_t gdn_decode_static_scratch_bytes(void) { return kStaticScratchBytes; }
 
 gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t pool_slots) {
     if (B < 0 || pool_slots < 0 || (B > 0 && !slots_host)) return GDN_ERR_INVALID_ARGUMENT;

@@ -156,6 +156,41 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
 size_t gdn_decode_workspace_bytes(void);
 
 /*
+ * gdn_decode_step for callers that cannot allocate device memory. The pages have
+ * no counterpart of this entry point; it exists for the library's users.
+ *
+ * Some callers cannot provide even the small workspace of gdn_decode_step: code
+ * that runs inside a host framework which owns the device allocator, plugins with a
+ * fixed memory budget, or latency-critical paths that must not call cudaMalloc
+ * (which can synchronize the device). This entry point takes the same arguments as
+ * gdn_decode_step without `workspace`, allocates nothing (no cudaMalloc, cudaFree
+ * or allocating library call) and uses a fixed scratch array that the library
+ * itself places in device memory instead: gdn_decode_static_scratch_bytes() bytes
+ * on every GPU that loads the library, held until the process exits.
+ *   - The first call on a device looks up that array's device address once (with
+ *     the device current); make that first call before any stream capture.
+ *   - Each call clears the part of the array it needs with an asynchronous memset
+ *     on `stream`, then launches as gdn_decode_step does. The results are the same.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents: calls that overlap on the GPU (other streams, other threads) race
+ *     on it. Serialize them, or use gdn_decode_step with one workspace each.
+ *   - If the scratch this build needs exceeds the array, the call returns
+ *     GDN_ERR_UNSUPPORTED before doing anything.
+ */
+gdn_status gdn_decode_step_static_scratch(const gdn_config* cfg, int32_t B, int32_t T,
+                                          const uint16_t* qkv, const uint16_t* a,
+                                          const uint16_t* b, const uint16_t* z,
+                                          const uint16_t* conv_w, const float* A_log,
+                                          const float* dt_bias, const uint16_t* norm_w,
+                                          uint16_t* conv_pool, float* state_pool,
+                                          int32_t pool_slots, const int32_t* slots,
+                                          uint16_t* out_bf16, float* out_f32, int32_t* err_flag,
+                                          void* stream);
+
+/* Size in bytes of the fixed scratch array of gdn_decode_step_static_scratch. */
+size_t gdn_decode_static_scratch_bytes(void);
+
+/*
  * Host-side check of a HOST copy of slots[]: GDN_OK when all B values are distinct
  * and in [0, pool_slots), GDN_ERR_SLOT_RANGE otherwise, GDN_ERR_INVALID_ARGUMENT for
  * a null pointer or negative size. Touches no device.

@@ -213,6 +213,23 @@ def run_reference(args, wl, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def rank_workload(wl, rank: int):
+    """Rank `rank`'s own sequences: the same shapes and distributions under its own seed
+    (the ranks share no sequence, so no data moves between them)."""
+    return wl.replace(seed=wl.seed + 7919 * rank)
+
+
+def max_over_ranks(v: float, device, world: int) -> float:
+    """The largest value over all ranks (timings are reported as the slowest rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_config(wl, args, world):
     return {"workload": f"{wl.name}: B={wl.batch} sequences x T={wl.tokens} token, Hk={wl.num_k_heads}, "
                         f"Hv={wl.num_v_heads}, dk={wl.head_k_dim}, dv={wl.head_v_dim}, conv width {wl.conv_width}, "
@@ -252,7 +269,7 @@ def main():
     if world > 1:
         dist.barrier()
     gdn.lib()
-    wlr = wl.replace(seed=wl.seed + 7919 * rank)  # each rank owns different sequences
+    wlr = rank_workload(wl, rank)  # each rank owns different sequences
 
     def bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -278,13 +295,6 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     sampler = ClockSampler(local) if rank == 0 else None
     for i in range(args.warmup):
@@ -324,7 +334,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
-    elapsed_ms = max_over_ranks(start.elapsed_time(end))
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev, world)
     # per-launch kernel time from events around eager launches of the same plans
     Ke = min(K, 2000)
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
@@ -334,7 +344,7 @@ def main():
         plans[i % n_inputs].launch()
         ev_e[i].record(stream)
     torch.cuda.synchronize()
-    kernel_ms_eager = max_over_ranks(statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(Ke)))
+    kernel_ms_eager = max_over_ranks(statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(Ke)), dev, world)
     if int(err.item()) != 0:
         raise RuntimeError("device reported an error flag %d" % int(err.item()))
     del graphs
@@ -368,7 +378,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
         e2e = {"value": world * wl.batch * wl.tokens * K / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 

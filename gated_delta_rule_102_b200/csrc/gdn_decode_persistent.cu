@@ -199,8 +199,9 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         const int conv_bytes = 2 * W * nch * 2 + 32;
         const bool dyn = p.sched != nullptr;
         unsigned int pending = 0;  // rank 0, lane 0: the index to relay next
-        auto relay = [&](int v, unsigned int val) {  // rank 0, lane 0
-            const uint32_t a_loc = smem_addr(ring + (v % kRing)), b_loc = smem_addr(rbar + (v % kRing));
+        auto relay = [&](int v, unsigned int val) {  // rank 0, lane 0: the group of unit v >= 1 (ring entry v - 1)
+            const int e = v - 1;
+            const uint32_t a_loc = smem_addr(ring + (e % kRing)), b_loc = smem_addr(rbar + (e % kRing));
             for (int r = 0; r < G; ++r)
                 st_async_f32(cluster_map_u32(a_loc, r), __uint_as_float(val), cluster_map_u32(b_loc, r));
         };
@@ -209,23 +210,23 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             int g;
             if (!dyn) {
                 g = cid + v * ncl;
-            } else {
+            } else if (v == 0) {
+                g = cid;  // the first ncl groups go out one per cluster, without waiting for the counter
+            } else {  // unit v >= 1 travels as ring entry v - 1
+                const int e = v - 1;
                 bool ok = true;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(rbar + (v % kRing), 4);
-                    ok = wait(rbar + (v % kRing), (v / kRing) & 1);
+                    mbar_arrive_expect_tx(rbar + (e % kRing), 4);
+                    ok = wait(rbar + (e % kRing), (e / kRing) & 1);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) return -2;
-                g = ring[v % kRing];
+                g = ring[e % kRing];
             }
             return g < ngroups ? g : kEndOfWork;
         };
-        if (dyn && rank == 0 && lane == 0) {
-            const unsigned int f0 = fetch();
-            relay(0, f0);
-            pending = f0 < (unsigned)ngroups ? fetch() : f0;
-        }
+        // with the dynamic schedule the counter numbers the groups after the first ncl
+        if (dyn && rank == 0 && lane == 0) pending = (unsigned)ncl + fetch();
         int g_next = receive(0);
         int slot_next = g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1;
         for (int v = 0;; ++v) {
@@ -236,7 +237,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             }
             if (g != kEndOfWork && dyn && rank == 0 && lane == 0) {  // the index of unit v+1, then fetch for v+2
                 relay(v + 1, pending);
-                if (pending < (unsigned)ngroups) pending = fetch();
+                if (pending < (unsigned)ngroups) pending = (unsigned)ncl + fetch();
             }
             if (g == kEndOfWork) {  // one end marker per consumer team
                 bool ok = true;
@@ -311,6 +312,13 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         }
         if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
             for (int i = 0; i < 1024; ++i) __nanosleep(64);
+        }
+        // The last loader through leaves the counters at zero for the next call: every
+        // fetch of every cluster has returned (its value was relayed) before its CTA
+        // counts itself here, and nothing else in this launch reads the counters.
+        if (dyn && lane == 0 && atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
         }
     } else if (warp <= L::FINISHER_WARPS) {
         // ============================== finishers ==============================
@@ -546,14 +554,9 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         if (wt == 0 && lane == 0) bulk_wait_all();  // this lane's tile stores have completed
     }
     __syncthreads();
-    if (p.sched && tid == 0) {  // the last CTA out leaves the counters at zero for the next call
-        __threadfence();
-        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-            atomicExch(p.sched, 0u);
-            atomicExch(p.sched + 1, 0u);
-        }
-    }
-    cluster_arrive_release();  // no CTA leaves while a peer may still send to it
+    // No CTA leaves while a peer may still send to it. Every message a CTA expects has
+    // been waited for, so the arrival needs no release ordering of this CTA's stores.
+    cluster_arrive_relaxed();
     cluster_wait_acquire();
 }
 

@@ -12,18 +12,20 @@
 //    free it starts the copies of unit v's state tile and z row (completing on the
 //    stage's `full` barrier) and of its conv inputs (history rows, x, weights) and
 //    a/b values (completing on `cbar`).
-//  * Warp 1, the finisher, takes units in order once their conv inputs have landed:
-//    it convolves this CTA's channels (its share of the k-head's q/k channels plus
-//    its v-head's v channels), sends the raw q/k share to every CTA of the cluster
-//    with st.async (completed on the receiver's mbarrier), rolls the conv history,
-//    waits for the other shares, and publishes the q/k norms, k.q and the gates.
-//  * The remaining eight warps form teams that take units in turn. A team owns a
-//    unit: each warp holds a band of columns (the columns of S are independent under
-//    the update), reads the tile from shared memory twice (S^T k and S^T q, then the
-//    update, written back in place), reduces over dk with two shuffle stages; one
-//    lane then hands the updated tile to the TMA engine as bulk stores and frees the
-//    stage once they have read it, and the team applies the RMSNorm, the norm weight
-//    and SiLU(z).
+//  * Warps 1-4, the finishers, take units in order once their conv inputs have
+//    landed: they convolve this CTA's channels (its share of the k-head's q/k
+//    channels plus its v-head's v channels), send the raw q/k share to every CTA of
+//    the cluster with st.async (completed on the receiver's mbarrier) and roll the
+//    conv history. The first finisher warp then waits for the other shares, tells
+//    the consumers that q/k and v are in (the stage's `full` barrier), and
+//    publishes the q/k norms, k.q and the gates on the stage's `pub` barrier.
+//  * The remaining eight warps form two teams that take units in turn. A team owns
+//    a unit: each warp holds a band of columns (the columns of S are independent
+//    under the update), reads the tile from shared memory for S^T k and S^T q and
+//    reduces over dk with shuffles, then (once `pub` has completed) reads it again
+//    for the update and streams the new rows straight to the pool; each warp frees
+//    its part of the stage after that, and the team applies the RMSNorm, the norm
+//    weight and SiLU(z).
 // Every channel's conv history is therefore read and rolled by exactly one CTA, the
 // state is read once and written once, and HBM sees a steady stream of TMA loads and
 // row stores instead of alternating load, compute and store phases.
@@ -91,8 +93,8 @@ struct WS {
     static constexpr int PART = QK + QB * 2 * DK * 4;                // [NTEAMS][2][TEAM_WARPS] f32
     static constexpr int FLAG = PART + round_up(NTEAMS * 2 * TEAM_WARPS * 4, 16);
     static constexpr int RING = FLAG + 16;                           // [kRing] int: relayed group indices
-    static constexpr int BARS = RING + kRing * 4;  // full, empty, conv [NSTAGE]; qk [QB]; ring [kRing]
-    static constexpr int TOTAL = BARS + (3 * NSTAGE + QB + kRing) * 8;
+    static constexpr int BARS = RING + kRing * 4;  // full, empty, conv, pub [NSTAGE]; qk [QB]; ring [kRing]
+    static constexpr int TOTAL = BARS + (4 * NSTAGE + QB + kRing) * 8;
     static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && (RPL & (RPL - 1)) == 0 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
 };
@@ -128,7 +130,8 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
     uint64_t* empty = full + NSTAGE;
     uint64_t* cbar = empty + NSTAGE;
-    uint64_t* qkbar = cbar + NSTAGE;
+    uint64_t* pub = cbar + NSTAGE;
+    uint64_t* qkbar = pub + NSTAGE;
     uint64_t* rbar = qkbar + QB;
     int* ring = reinterpret_cast<int*>(smem + L::RING);
 
@@ -139,7 +142,8 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
 
     if (tid == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(full + s, 2);                // the producer's copy arrival and its publish arrival
+            mbar_init(full + s, 2);  // the loader's copies (tile, z) and the finisher's "q/k are in" arrival
+            mbar_init(pub + s, 1);   // the finisher's norms, k.q and gates
             mbar_init(empty + s, L::TEAM_WARPS);   // one arrival per warp of the consuming team
             mbar_init(cbar + s, 1);                // the staged conv inputs
         }
@@ -149,6 +153,12 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         mbar_init_fence();
     }
     __syncthreads();
+    // With programmatic dependent launch this grid may start while the previous one
+    // drains; nothing it reads is touched before that grid has completed.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    // unit 0 of every CTA is group cid: its slot load overlaps the cluster barrier
+    const int slot_first = warp == 0 ? __ldg(p.slots + cid / Hk) : -1;
     cluster_arrive_relaxed();  // every CTA of the cluster runs before any st.async targets it
     cluster_wait_acquire();
 
@@ -192,13 +202,12 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         // groups (completing on cbar). The group and slot go along in the stage info.
         //
         // Which group unit v is: with a static schedule cid + v * ncl; with the
-        // dynamic schedule, the cluster's rank 0 takes groups from the shared counter
-        // one unit ahead and relays each index to every CTA of the cluster with
-        // st.async (ring of kRing entries), so the CTAs of a cluster walk the same
-        // groups and faster clusters simply take more of them.
+        // dynamic schedule, the cluster's rank 0 takes the group of unit v + 1 from the
+        // shared counter once unit v's copies are out and relays it to every CTA of the
+        // cluster with st.async (ring of kRing entries), so the CTAs of a cluster walk
+        // the same groups and faster clusters simply take more of them.
         const int conv_bytes = 2 * W * nch * 2 + 32;
         const bool dyn = p.sched != nullptr;
-        unsigned int pending = 0;  // rank 0, lane 0: the index to relay next
         auto relay = [&](int v, unsigned int val) {  // rank 0, lane 0: the group of unit v >= 1 (ring entry v - 1)
             const int e = v - 1;
             const uint32_t a_loc = smem_addr(ring + (e % kRing)), b_loc = smem_addr(rbar + (e % kRing));
@@ -225,19 +234,13 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             }
             return g < ngroups ? g : kEndOfWork;
         };
-        // with the dynamic schedule the counter numbers the groups after the first ncl
-        if (dyn && rank == 0 && lane == 0) pending = (unsigned)ncl + fetch();
         int g_next = receive(0);
-        int slot_next = g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1;
+        int slot_next = slot_first;
         for (int v = 0;; ++v) {
             const int g = g_next, slot = slot_next;
             if (g == -2) {
                 fail();
                 break;
-            }
-            if (g != kEndOfWork && dyn && rank == 0 && lane == 0) {  // the index of unit v+1, then fetch for v+2
-                relay(v + 1, pending);
-                if (pending < (unsigned)ngroups) pending = (unsigned)ncl + fetch();
             }
             if (g == kEndOfWork) {  // one end marker per consumer team
                 bool ok = true;
@@ -306,7 +309,11 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                     tma_load_1d(zb + s * DV, p.z + ((size_t)seq * Hv + h) * DV, DV * 2, full + s);
                 }
             }
-            // the next unit's group and slot, while this unit's copies are in flight
+            // The next unit's group and slot, while this unit's copies are in flight. With
+            // the dynamic schedule the counter numbers the groups after the first ncl; a
+            // group is taken only once this unit's copies are out, so no cluster holds
+            // more than the units its stages can take when the counter runs out.
+            if (dyn && rank == 0 && lane == 0) relay(v + 1, (unsigned)ncl + fetch());
             g_next = receive(v + 1);
             slot_next = g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1;
         }
@@ -408,6 +415,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 fail();  // the other finisher warps see the abort at the next agreement
                 continue;
             }
+            if (lane == 0) mbar_arrive(full + s);  // the raw q/k and v are in: pass 1 may start
             if (valid) {
                 const float* qr = qkb + q * 2 * DK;
                 float sq = 0.f, sk = 0.f, dot = 0.f;
@@ -436,7 +444,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(full + s);
+            if (lane == 0) mbar_arrive(pub + s);
         }
     } else {
         // ============================== consumers ==============================
@@ -451,10 +459,10 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             if (L::TEAM_WARPS > 1) ok = named_barrier_and(1 + team, 32 * L::TEAM_WARPS, ok && !*abort_flag);
             else ok = __all_sync(0xffffffffu, ok && !*abort_flag);
             if (!ok) break;  // the team's warps leave together
-            const StageInfo st = si[s];
-            if (st.group == kEndOfWork) break;
-            if (st.slot >= 0) {
-                const int seq = st.group / Hk, h = (st.group - seq * Hk) * G + rank;
+            const int st_group = si[s].group, st_slot = si[s].slot;
+            if (st_group == kEndOfWork) break;
+            if (st_slot >= 0) {
+                const int seq = st_group / Hk, h = (st_group - seq * Hk) * G + rank;
                 const uint2 zz = rg == 0 ? *reinterpret_cast<const uint2*>(zb + s * DV + col) : make_uint2(0u, 0u);
                 const float4* tl = reinterpret_cast<const float4*>(tiles + (size_t)s * (DK * DV)) + col / 4;
                 const float* qr = qkb + q * 2 * DK;
@@ -487,6 +495,13 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                     mq.z += __shfl_xor_sync(0xffffffffu, mq.z, off); mq.w += __shfl_xor_sync(0xffffffffu, mq.w, off);
                 }
                 const float4 vv = *reinterpret_cast<const float4*>(vsb + s * DV + col);
+                // the norms, k.q and gates of this unit (published after the q/k exchange)
+                bool okp = wait(pub + s, (u / NSTAGE) & 1);
+                if (!okp) fail();
+                if (L::TEAM_WARPS > 1) okp = named_barrier_and(1 + team, 32 * L::TEAM_WARPS, okp && !*abort_flag);
+                else okp = __all_sync(0xffffffffu, okp && !*abort_flag);
+                if (!okp) break;
+                const StageInfo st = si[s];
                 const float am = st.alpha * st.nk, aq = st.alpha * st.nq;
                 float4 d, o;
                 d.x = st.beta * fmaf(-am, mk.x, vv.x); d.y = st.beta * fmaf(-am, mk.y, vv.y);
@@ -494,8 +509,9 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 o.x = fmaf(aq, mq.x, d.x * st.kq); o.y = fmaf(aq, mq.y, d.y * st.kq);
                 o.z = fmaf(aq, mq.z, d.z * st.kq); o.w = fmaf(aq, mq.w, d.w * st.kq);
                 const float4 dn = make_float4(d.x * st.nk, d.y * st.nk, d.z * st.nk, d.w * st.nk);
-                // the updated rows go back into the stage; the TMA engine stores the tile
-                float4* tw = const_cast<float4*>(tl);
+                // the updated rows go straight to the pool (streaming stores: nothing here reads them again)
+                float4* sg = reinterpret_cast<float4*>(p.state_pool + ((size_t)st_slot * Hv + h) * (size_t)(DK * DV)) +
+                             col / 4;
 #pragma unroll 2
                 for (int i = 0; i < L::RPL; i += 4) {
                     const int r = row0 + ((i + rot) & (L::RPL - 1));
@@ -506,10 +522,11 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                         float4 x = tl[(size_t)(r + e) * (DV / 4)];
                         x.x = fmaf(st.alpha, x.x, kk[e] * dn.x); x.y = fmaf(st.alpha, x.y, kk[e] * dn.y);
                         x.z = fmaf(st.alpha, x.z, kk[e] * dn.z); x.w = fmaf(st.alpha, x.w, kk[e] * dn.w);
-                        tw[(size_t)(r + e) * (DV / 4)] = x;
+                        __stcs(sg + (size_t)(r + e) * (DV / 4), x);
                     }
                 }
-                fence_proxy_async_smem();  // the bulk store (async proxy) must see these writes
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
                 // ---- step 8 over the whole head: the team's warps pool their sums of o^2
                 float ss = rg == 0 ? o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w : 0.f;
 #pragma unroll
@@ -518,16 +535,6 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 if (lane == 0) pt[wt] = ss;
                 if (L::TEAM_WARPS > 1) named_barrier(1 + team, 32 * L::TEAM_WARPS);
                 else __syncwarp();
-                if (wt == 0 && lane == 0) {  // the whole updated tile back to the pool, then free the stage
-                    char* dstg = reinterpret_cast<char*>(p.state_pool + ((size_t)st.slot * Hv + h) * (size_t)(DK * DV));
-                    const char* srcs = reinterpret_cast<const char*>(tiles + (size_t)s * (DK * DV));
-                    for (int c = 0; c < L::TILE_BYTES; c += kTileChunk)
-                        tma_store_1d(dstg + c, srcs + c, (uint32_t)min(kTileChunk, L::TILE_BYTES - c));
-                    bulk_commit();
-                    bulk_wait_read_all();
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty + s);
                 float tot = 0.f;
 #pragma unroll
                 for (int w = 0; w < L::TEAM_WARPS; ++w) tot += pt[w];
@@ -551,7 +558,6 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 if (lane == 0) mbar_arrive(empty + s);
             }
         }
-        if (wt == 0 && lane == 0) bulk_wait_all();  // this lane's tile stores have completed
     }
     __syncthreads();
     // No CTA leaves while a peer may still send to it. Every message a CTA expects has
@@ -572,13 +578,15 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
     cfg.blockDim = dim3(L::NT);
     cfg.dynamicSmemBytes = L::TOTAL;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)G;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;  // the occupancy query takes the cluster shape only
     int& cap = cap_cache[dev & 15][G];
     if (cap <= 0) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
@@ -595,6 +603,7 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
     const int ncl = ngroups < cap ? ngroups : cap;  // the dynamic schedule needs ncl <= co-resident clusters too
     if (ncl <= 0) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3((unsigned)(ncl * G));
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, a, ncl);
 }
 

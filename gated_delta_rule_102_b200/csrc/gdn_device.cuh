@@ -305,6 +305,12 @@ __device__ __forceinline__ void tma_load_1d(void* dst_smem, const void* src_gmem
         : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (a hint: no completion, no ordering).
+// src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src_gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src_gmem), "r"(bytes) : "memory");
+}
+
 // The gated delta rule on a DK x DVS tile held in shared memory, for tokens 0..T-1.
 // Same arithmetic as delta_rule_tile; S lives in shared memory between tokens and
 // each thread reads it twice per token (reductions, then update), so registers stay

@@ -57,6 +57,10 @@ struct StageInfo {  // what the producer publishes for a staged unit
 };
 constexpr int kEndOfWork = -1;
 constexpr int kRing = 16;  // group indices relayed from the cluster's rank 0 (dynamic schedule)
+// Units 0 .. kFixedUnits - 1 of every CTA are groups cid + u * ncl under either
+// schedule; their state tiles are prefetched into L2 before the grid dependency wait.
+constexpr int kFixedUnits = 2;
+static_assert(kFixedUnits >= 1 && kFixedUnits <= 8, "fixed units: four prefetch lanes each");
 
 template <int DK, int DV>
 struct WS {
@@ -153,31 +157,6 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         mbar_init_fence();
     }
     __syncthreads();
-    // Units 0 and 1 of every CTA are fixed: groups cid and cid + ncl. With
-    // programmatic dependent launch this grid may start while the previous one
-    // drains, so their state tiles are prefetched into L2 now. The slot read here
-    // may be stale (the previous grid may still write the slot list): it only steers
-    // the hint, and L2 stays coherent with whatever that grid still writes. Nothing
-    // is read for use before that grid has completed.
-    if (warp == 0 && lane < 8) {
-        const int g = cid + (lane >> 2) * ncl;
-        if (g < ngroups) {
-            const int sl = __ldcg(p.slots + g / Hk);
-            if (sl >= 0 && sl < p.P) {
-                const char* t = reinterpret_cast<const char*>(
-                    p.state_pool + ((size_t)sl * Hv + (g % Hk) * G + rank) * (size_t)(DK * DV));
-                bulk_prefetch_l2(t + (lane & 3) * (L::TILE_BYTES / 4), L::TILE_BYTES / 4);
-            }
-        }
-    }
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-    // the slots of units 0 and 1, loaded while the cluster barrier completes
-    const int slot_first = warp == 0 ? __ldg(p.slots + cid / Hk) : -1;
-    const int slot_second = warp == 0 && cid + ncl < ngroups ? __ldg(p.slots + (cid + ncl) / Hk) : -1;
-    cluster_arrive_relaxed();  // every CTA of the cluster runs before any st.async targets it
-    cluster_wait_acquire();
-
     auto fail = [&]() {
         if (lane == 0) {
             *abort_flag = 1;
@@ -211,6 +190,31 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     };
     float* gparams = reinterpret_cast<float*>(smem + L::GP);  // A_log then dt_bias
 
+    // With programmatic dependent launch this grid may start while the previous one
+    // drains, so the state tiles of the fixed units are prefetched into L2 now (the
+    // small conv inputs gain nothing from it). The slot read here may be stale (the
+    // previous grid may still write the slot list): it only steers the hint, and L2
+    // stays coherent with whatever that grid still writes. Nothing is read for use
+    // before that grid has completed.
+    if (warp == 0 && lane < 4 * kFixedUnits) {
+        const int g = cid + (lane >> 2) * ncl;
+        if (g < ngroups) {
+            const int sl = __ldcg(p.slots + g / Hk);
+            if (sl >= 0 && sl < p.P) {
+                const char* t = reinterpret_cast<const char*>(
+                    p.state_pool + ((size_t)sl * Hv + (g % Hk) * G + rank) * (size_t)(DK * DV));
+                bulk_prefetch_l2(t + (lane & 3) * (L::TILE_BYTES / 4), L::TILE_BYTES / 4);
+            }
+        }
+    }
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    // lane u of the loader: the slot of fixed unit u, loaded while the cluster barrier completes
+    const int slot_fixed =
+        warp == 0 && lane < kFixedUnits && cid + lane * ncl < ngroups ? __ldg(p.slots + (cid + lane * ncl) / Hk) : -1;
+    cluster_arrive_relaxed();  // every CTA of the cluster runs before any st.async targets it
+    cluster_wait_acquire();
+
     if (warp == 0) {
         // ============================== loader ==============================
         // Unit v's copies into stage v % NSTAGE as soon as the stage is free: the
@@ -218,15 +222,15 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         // groups (completing on cbar). The group and slot go along in the stage info.
         //
         // Which group unit v is: with a static schedule cid + v * ncl; with the
-        // dynamic schedule units 0 and 1 are the same, and from unit 2 on the cluster's
+        // dynamic schedule the fixed units are the same, and after them the cluster's
         // rank 0 takes the group of unit v + 1 from the shared counter once unit v's
         // copies are out and relays it to every CTA of the cluster with st.async (ring
         // of kRing entries), so the CTAs of a cluster walk the same groups and faster
         // clusters simply take more of them.
         const int conv_bytes = 2 * W * nch * 2 + 32;
         const bool dyn = p.sched != nullptr;
-        auto relay = [&](int v, unsigned int val) {  // rank 0, lane 0: the group of unit v >= 2 (ring entry v - 2)
-            const int e = v - 2;
+        auto relay = [&](int v, unsigned int val) {  // rank 0, lane 0: the group of unit v >= kFixedUnits
+            const int e = v - kFixedUnits;
             const uint32_t a_loc = smem_addr(ring + (e % kRing)), b_loc = smem_addr(rbar + (e % kRing));
             for (int r = 0; r < G; ++r)
                 st_async_f32(cluster_map_u32(a_loc, r), __uint_as_float(val), cluster_map_u32(b_loc, r));
@@ -234,10 +238,10 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         auto fetch = [&]() { return atomicAdd(p.sched, 1u); };
         auto receive = [&](int v) {  // lane-uniform group index of unit v (kEndOfWork past the end)
             int g;
-            if (!dyn || v < 2) {
-                g = cid + v * ncl;  // with the dynamic schedule too, the first 2 ncl groups go out two per cluster
-            } else {  // unit v >= 2 travels as ring entry v - 2
-                const int e = v - 2;
+            if (!dyn || v < kFixedUnits) {
+                g = cid + v * ncl;
+            } else {  // later units travel as ring entry v - kFixedUnits
+                const int e = v - kFixedUnits;
                 bool ok = true;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(rbar + (e % kRing), 4);
@@ -250,7 +254,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             return g < ngroups ? g : kEndOfWork;
         };
         int g_next = receive(0);
-        int slot_next = slot_first;
+        int slot_next = __shfl_sync(0xffffffffu, slot_fixed, 0);
         for (int v = 0;; ++v) {
             const int g = g_next, slot = slot_next;
             if (g == -2) {
@@ -325,12 +329,14 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 }
             }
             // The next unit's group and slot, while this unit's copies are in flight. With
-            // the dynamic schedule the counter numbers the groups after the first 2 ncl; a
+            // the dynamic schedule the counter numbers the groups after the fixed ones; a
             // group is taken only once this unit's copies are out, so no cluster holds
             // more than the units its stages can take when the counter runs out.
-            if (dyn && v >= 1 && rank == 0 && lane == 0) relay(v + 1, 2u * (unsigned)ncl + fetch());
+            if (dyn && v + 1 >= kFixedUnits && rank == 0 && lane == 0)
+                relay(v + 1, (unsigned)(kFixedUnits * ncl) + fetch());
             g_next = receive(v + 1);
-            slot_next = v == 0 ? slot_second : (g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1);
+            slot_next = v + 1 < kFixedUnits ? __shfl_sync(0xffffffffu, slot_fixed, v + 1)
+                                            : (g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1);
         }
         if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
             for (int i = 0; i < 1024; ++i) __nanosleep(64);

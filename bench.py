@@ -33,7 +33,7 @@ METRIC = "GDN decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s) at B=6
 UNIT = "tokens/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_NAME = "decode_ws_kernel"
+FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (4 partitions x 32)
 
 
 def parse_args():
@@ -61,6 +61,22 @@ def algorithmic_bytes(wl) -> int:
     return wl.batch * per_seq + per_launch
 
 
+def kernel_for(wl, num_sms: int) -> str:
+    """The kernel the launcher picks for the workload (the rule of launch_decode_fused):
+    the persistent kernel for one token over at least two waves of co-resident clusters
+    (one CTA per SM, G CTAs per cluster), else the cluster-per-group kernels."""
+    G = wl.num_v_heads // wl.num_k_heads
+    if wl.tokens == 1 and wl.batch * wl.num_k_heads >= 2 * (num_sms // G):
+        return "decode_ws_kernel"
+    return "decode_fused_tma_kernel" if wl.tokens == 1 else "decode_mt_kernel"
+
+
+def algorithmic_flops(wl) -> int:
+    """FP32 flops of the delta rule per launch: per state element and token the decay,
+    S^T k, the rank-1 update and S^T q (7 flops); the conv and norms are negligible."""
+    return 7 * wl.batch * wl.tokens * wl.num_v_heads * wl.head_k_dim * wl.head_v_dim
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_102_b200", "csrc")
@@ -71,10 +87,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(wl_name: str):
+def profiled_traffic(kernel: str, wl_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"{KERNEL_NAME}_{wl_name}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{wl_name}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
@@ -230,13 +246,23 @@ def max_over_ranks(v: float, device, world: int) -> float:
     return float(t.item())
 
 
+L2_BYTES = 126 << 20
+
+
+def l2_note(wl, pools: int) -> str:
+    pool = wl.pool_slots * wl.num_v_heads * wl.head_k_dim * wl.head_v_dim * 4
+    if pools * pool > L2_BYTES:
+        return f"inputs larger than L2: {pools} state pools x {pool >> 20} MiB cycled"
+    return (f"state L2-resident: {pools} state pools x {pool / 2**20:.1f} MiB cycled, below the 126 MB L2 "
+            f"(a latency workload; no flush)")
+
+
 def workload_config(wl, args, world):
     return {"workload": f"{wl.name}: B={wl.batch} sequences x T={wl.tokens} token, Hk={wl.num_k_heads}, "
                         f"Hv={wl.num_v_heads}, dk={wl.head_k_dim}, dv={wl.head_v_dim}, conv width {wl.conv_width}, "
                         f"{wl.pool_slots}-slot fp32 state pool per layer",
             "batch_per_gpu": wl.batch, "tokens_per_sequence": wl.tokens, "state_pools_cycled": args.pools,
-            "l2": f"inputs larger than L2: {args.pools} state pools x "
-                  f"{wl.pool_slots * wl.num_v_heads * wl.head_k_dim * wl.head_v_dim * 4 >> 20} MiB cycled",
+            "l2": l2_note(wl, args.pools),
             "parallelism": f"dp{world} (independent sequence shards, no collective)"}
 
 
@@ -395,6 +421,20 @@ def main():
     peak, peak_kind = hbm_peak()
     kernel_ms = elapsed_ms / K  # graph-replayed launches back to back: includes the gaps between them
     achieved = nbytes / (kernel_ms / 1e3) / 1e9
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    kernel = kernel_for(wl, num_sms)
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": profiled_traffic(kernel, wl.name), "peak_source": f"{peak_kind} copy bandwidth"}
+    flops = algorithmic_flops(wl)
+    sm_mhz = (clocks or {}).get("sm_mhz")
+    if sm_mhz and flops / (kernel_ms / 1e3) / 1e12 / (num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6) > roof["frac"]:
+        # closer to the FP32 FMA peak (SMs x 128 lanes x 2 flops x the median SM clock
+        # sampled in the timed region) than to the copy bandwidth: ALU-bound
+        alu_peak = num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6
+        alu = flops / (kernel_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": alu, "peak": alu_peak, "unit": "TFLOP/s", "frac": alu / alu_peak,
+                "traffic": roof["traffic"], "peak_source": "FP32 FMA lanes x measured SM clock",
+                "hbm_gbs_achieved": achieved, "hbm_frac": achieved / peak}
     tokens = world * wl.batch * wl.tokens * K
     value = tokens / (elapsed_ms / 1e3)
     job_gbs = world * nbytes * K / (elapsed_ms / 1e3) / 1e9
@@ -404,11 +444,10 @@ def main():
         "dtype": "f32", "data": "synthetic (seeded SplitMix64 draws; bf16 inputs, fp32 state)",
         "config": workload_config(wl, args, world),
         "hbm_gbs": job_gbs / world, "frac_of_8tbs": job_gbs / world / NOMINAL_HBM_GBS,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic(wl.name), "peak_source": f"{peak_kind} copy bandwidth",
-                     "kernel": KERNEL_NAME, "kernel_us": kernel_ms * 1e3, "algorithmic_bytes": nbytes,
-                     "timing": "CUDA events around K graph-replayed launches (per launch incl. inter-launch gaps)",
-                     "eager_kernel_us": kernel_ms_eager * 1e3},
+        "roofline": dict(roof, kernel=kernel, kernel_us=kernel_ms * 1e3, algorithmic_bytes=nbytes,
+                         algorithmic_flops=flops,
+                         timing="CUDA events around K graph-replayed launches (per launch incl. inter-launch gaps)",
+                         eager_kernel_us=kernel_ms_eager * 1e3),
         "e2e": e2e, "clocks": clocks, "gpu_launches": K,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -2,13 +2,20 @@
 // in one launch (steps 3 to 8 and the SiLU(z) gate of steps 9+10+11 on the page
 // "spark_model/forward/qwen3_5/linear_attention.rs").
 //
-// Work decomposition. One thread-block cluster per (sequence, k-head). Its G*NS CTAs
+// This file holds the launcher that picks the kernel for a launch, and the kernel
+// for single-token launches over few sequences:
+//  * one token, enough (sequence, k-head) groups to fill the GPU twice: the
+//    persistent pipelined kernel (gdn_decode_persistent.cu);
+//  * several tokens: the multi-token kernel (gdn_decode_mt.cu);
+//  * otherwise the cluster kernel below.
+//
+// Cluster kernel. One thread-block cluster per (sequence, k-head). Its G*NS CTAs
 // are the G v-heads that share the k-head (v-head h reads k-head h / G) times NS
 // column slices of dv. CTA (v-head h, slice sl) owns state columns
-// [sl*DVS, (sl+1)*DVS) of head h: it streams that DK x DVS fp32 tile from HBM into
-// registers once, runs every token of the launch on it, and writes it back in place.
-// The columns of S are independent under the update (column j needs only S[:, j],
-// k, q and v_j), so the slices never exchange state.
+// [sl*DVS, (sl+1)*DVS) of head h: it stages that DK x DVS fp32 tile from HBM into
+// shared memory by TMA, runs the token on it, and writes it back in place. The
+// columns of S are independent under the update (column j needs only S[:, j], k, q
+// and v_j), so the slices never exchange state.
 //
 // Conv ownership. Every channel's conv history is read and rolled by exactly one CTA
 // of the grid: the CTA's own v columns, plus a 1/(G*NS) share of its k-head's q and k
@@ -26,7 +33,8 @@ namespace {
 
 constexpr int kMaxCluster = 8;
 // Launches with at most this many tokens stage the state tile in shared memory
-// (bandwidth-bound); longer ones keep it in registers across tokens (ALU-bound).
+// (bandwidth-bound); longer ones run the multi-token kernel, which keeps it in
+// registers across tokens (ALU-bound).
 #ifndef GDN_MAX_TOKENS_STAGED
 #define GDN_MAX_TOKENS_STAGED 1
 #endif
@@ -51,136 +59,6 @@ struct FusedSmem {
     static __host__ __device__ int part(int T) { return sc(T) + round4(T * (int)(sizeof(TokenScalars) / 4)); }
     static __host__ __device__ int total_floats(int T, int NS) { return part(T) + round4(T * NS); }
 };
-
-template <int DK, int DVS>
-__global__ void __launch_bounds__(Tile<DK, DVS>::NT)
-decode_fused_kernel(const DecodeArgs p) {
-    using Geo = Tile<DK, DVS>;
-    using L = FusedSmem<DK, DVS>;
-    constexpr int RPT = Geo::RPT, NT = Geo::NT;
-    extern __shared__ __align__(128) float4 smem4[];
-    float* smem = reinterpret_cast<float*>(smem4);
-
-    const int T = p.T, G = p.sh.Hv / p.sh.Hk, NS = p.NS, CS = G * NS;
-    const int dv = p.sh.dv, C = p.sh.C;
-    const int cid = blockIdx.x / CS, rank = blockIdx.x - cid * CS;
-    const int seq = cid / p.sh.Hk, hk = cid - seq * p.sh.Hk;
-    const int gi = rank / NS, sl = rank - gi * NS;
-    const int h = hk * G + gi, col0 = sl * DVS;
-    const int tid = threadIdx.x;
-
-    if (CS > 1) cluster_arrive_relaxed();  // B0: peers' shared memory becomes addressable
-    const int slot = __ldg(p.slots + seq);
-    if (slot < 0 || slot >= p.P) {  // the whole cluster sees the same slot and leaves together
-        if (tid == 0 && rank == 0 && p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
-        return;
-    }
-
-    // ---- stream the state tile in: issued first, consumed after the conv
-    float4 S[RPT];
-    const int cg = tid % Geo::TPR, rp = tid / Geo::TPR;
-    float4* Sg = reinterpret_cast<float4*>(p.state_pool + ((size_t)slot * p.sh.Hv + h) * (size_t)DK * dv + col0) +
-                 (size_t)(rp * RPT) * (dv / 4) + cg;
-#pragma unroll
-    for (int s = 0; s < RPT; ++s) S[s] = __ldcs(Sg + (size_t)s * (dv / 4));
-
-    float* qk = smem + L::qk(T);
-    float* vs = smem + L::vs(T);
-    float* os = smem + L::os(T);
-    float* red = smem + L::red(T);
-    TokenScalars* sc = reinterpret_cast<TokenScalars*>(smem + L::sc(T));
-    float* part = smem + L::part(T);
-
-    // ---- steps 4, 5: gate and beta of v-head h, per token
-    if (tid < T) {
-        const size_t i = ((size_t)seq * T + tid) * p.sh.Hv + h;
-        gate_and_beta(p.a[i], p.b[i], p.A_log[h], p.dt_bias[h], sc[tid].alpha, sc[tid].beta);
-    }
-
-    // ---- step 3: this CTA's conv channels
-    if (CS > 1) cluster_wait_acquire();
-    const int qk_lo = (rank * 2 * DK) / CS, qk_hi = ((rank + 1) * 2 * DK) / CS;
-    const int nqk = qk_hi - qk_lo;
-    uint16_t* hist_base = p.conv_pool + (size_t)slot * (p.sh.W - 1) * C;
-    const uint16_t* x_base = p.qkv + (size_t)seq * T * C;
-    for (int c = tid; c < nqk + DVS; c += NT) {
-        int ch;
-        if (c < nqk) {
-            const int j = qk_lo + c;  // 0..2DK-1 within this k-head: q then k
-            ch = j < DK ? hk * DK + j : p.sh.Hk * DK + hk * DK + (j - DK);
-            conv_channel(hist_base + ch, x_base + ch, p.conv_w + (size_t)ch * p.sh.W, p.sh.W, T, (size_t)C,
-                         [&](int t, float s) {
-                             float* dst = qk + t * 2 * DK + j;
-                             if (CS > 1) {
-                                 for (int r = 0; r < CS; ++r) *cluster_map(dst, r) = s;
-                             } else {
-                                 *dst = s;
-                             }
-                         });
-        } else {
-            const int jj = c - nqk;
-            ch = 2 * p.sh.Hk * DK + h * dv + col0 + jj;
-            conv_channel(hist_base + ch, x_base + ch, p.conv_w + (size_t)ch * p.sh.W, p.sh.W, T, (size_t)C,
-                         [&](int t, float s) { vs[t * DVS + jj] = s; });
-        }
-    }
-    if (CS > 1) {  // B1: every CTA now holds the k-head's whole raw q and k
-        cluster_arrive_release();
-        cluster_wait_acquire();
-    } else {
-        __syncthreads();
-    }
-
-    // ---- L2 norms of q and k (step 3) as factors on the raw values
-    qk_norms<DK>(qk, sc, T, p.sh.l2_eps, p.sh.q_scale, Geo::NW);
-    __syncthreads();
-
-    // ---- step 7 on the register tile, all tokens
-    delta_rule_tile<DK, DVS>(S, qk, vs, sc, os, red, T);
-
-#pragma unroll
-    for (int s = 0; s < RPT; ++s) __stcs(Sg + (size_t)s * (dv / 4), S[s]);
-
-    // ---- step 8: per-token sum of o^2 over this slice, shared with the v-head's other slices
-    __syncthreads();
-    {
-        const int lane = tid & 31, warp = tid >> 5;
-        for (int t = warp; t < T; t += Geo::NW) {
-            float acc = 0.f;
-            for (int j = lane; j < DVS; j += 32) acc = fmaf(os[t * DVS + j], os[t * DVS + j], acc);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) {
-                float* dst = part + t * NS + sl;
-                if (NS > 1) {
-                    for (int u = 0; u < NS; ++u) *cluster_map(dst, gi * NS + u) = acc;
-                } else {
-                    *dst = acc;
-                }
-            }
-        }
-    }
-    if (CS > 1 && NS > 1) {  // B2
-        cluster_arrive_release();
-        cluster_wait_acquire();
-    } else {
-        __syncthreads();
-    }
-
-    // ---- RMSNorm x norm weight x SiLU(z), bf16 out
-    const float inv_dv = 1.0f / (float)dv;
-    for (int idx = tid; idx < T * DVS; idx += NT) {
-        const int t = idx / DVS, j = idx - t * DVS;
-        float ss = 0.f;
-        for (int u = 0; u < NS; ++u) ss += part[t * NS + u];
-        const float inv = rsqrtf(ss * inv_dv + p.sh.rms_eps);
-        const size_t o_i = (((size_t)seq * T + t) * p.sh.Hv + h) * dv + col0 + j;
-        const float y = os[t * DVS + j] * inv * bf16_bits_to_float(p.norm_w[col0 + j]) *
-                        silu(bf16_bits_to_float(p.z[o_i]));
-        p.out[o_i] = float_to_bf16_bits(y);
-        if (p.out_f32) p.out_f32[o_i] = y;
-    }
-}
 
 template <int DK, int DVS>
 struct TmaSmem {
@@ -358,39 +236,13 @@ cudaError_t launch_tma(const DecodeArgs& a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int DK, int DVS>
-cudaError_t launch_tile(const DecodeArgs& a, cudaStream_t stream) {
-    using Geo = Tile<DK, DVS>;
-    const int G = a.sh.Hv / a.sh.Hk, CS = G * a.NS;
-    const size_t smem = (size_t)FusedSmem<DK, DVS>::total_floats(a.T, a.NS) * sizeof(float);
-    auto kern = decode_fused_kernel<DK, DVS>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.B * a.sh.Hk * CS));
-    cfg.blockDim = dim3(Geo::NT);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)CS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
-}
-
 template <int DK>
 cudaError_t dispatch_dvs(const DecodeArgs& a, int dvs, cudaStream_t stream) {
-    const bool staged = a.T <= kMaxTokensStaged;
     switch (dvs) {
-        case 16: return staged ? launch_tma<DK, 16>(a, stream) : launch_tile<DK, 16>(a, stream);
-        case 32: return staged ? launch_tma<DK, 32>(a, stream) : launch_tile<DK, 32>(a, stream);
-        case 64: return staged ? launch_tma<DK, 64>(a, stream) : launch_tile<DK, 64>(a, stream);
-        case 128: return staged ? launch_tma<DK, 128>(a, stream) : launch_tile<DK, 128>(a, stream);
+        case 16: return launch_tma<DK, 16>(a, stream);
+        case 32: return launch_tma<DK, 32>(a, stream);
+        case 64: return launch_tma<DK, 64>(a, stream);
+        case 128: return launch_tma<DK, 128>(a, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -418,6 +270,10 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream) {
         cudaError_t e = persistent_capacity(a, &cap);
         if (e != cudaSuccess) return e;
         if (cap > 0 && (long)a.B * a.sh.Hk >= (long)kPersistentMinWaves * cap) return launch_decode_persistent(a, stream);
+    }
+    if (a.T > kMaxTokensStaged) {  // several tokens: the state stays in registers across them
+        if (!multitoken_supported(a)) return cudaErrorInvalidValue;
+        return launch_decode_multitoken(a, stream);
     }
     const int dvs = a.sh.dv / a.NS;
     switch (a.sh.dk) {

@@ -86,6 +86,9 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
 bool persistent_supported(const DecodeArgs& a);
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters);
 cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream);
+// Multi-token kernel (state in registers across the launch's tokens).
+bool multitoken_supported(const DecodeArgs& a);
+cudaError_t launch_decode_multitoken(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_conv_update(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_recurrent(const RecurrentArgs& a, cudaStream_t stream);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);

@@ -103,7 +103,9 @@ class Workload:
     seeded permutation of the pool) or ``sample`` (``batch`` distinct slots
     drawn without replacement from a larger pool).
     ``gate_mode``: ``normal`` (a ~ N(0,1) like the other projections) or
-    ``decay_half_to_one`` (a chosen so that exp(g) is spread over [0.5, 1)).
+    ``decay_half_to_one`` (a chosen so that exp(g) is spread over [0.5, 1)) or
+    ``decay_wide`` (exp(g) = 2^-u with u ~ U(0, 48), and 2^-200 for about one entry
+    in eight: decays far below 1, down to values that underflow in fp32).
     """
 
     name: str
@@ -184,7 +186,7 @@ def step_inputs(wl: Workload, step: int, rows: Optional[Sequence[int]] = None) -
     T, C, Hv, dv = wl.tokens, wl.channels, wl.num_v_heads, wl.head_v_dim
     rows = list(_seq_rows(wl, rows))
     out = {k: [] for k in ("qkv", "a", "b", "z")}
-    w = weights(wl) if wl.gate_mode == "decay_half_to_one" else None
+    w = weights(wl) if wl.gate_mode != "normal" else None
     for r in rows:
         out["qkv"].append(normal(stream_key(wl.seed, "qkv", step, r), T * C))
         out["b"].append(normal(stream_key(wl.seed, "b", step, r), T * Hv))
@@ -192,11 +194,17 @@ def step_inputs(wl: Workload, step: int, rows: Optional[Sequence[int]] = None) -
         if wl.gate_mode == "normal":
             out["a"].append(normal(stream_key(wl.seed, "a", step, r), T * Hv))
         else:
-            # Choose the decay d = exp(g) ~ U(0.5, 1 - 2^-8) and invert the gate's
-            # parameterisation for the raw projection a (input construction only).
-            d = uniform(stream_key(wl.seed, "decay", step, r), T * Hv, 0.5, 1.0 - 2.0 ** -8)
+            # Choose the decay d = exp(g) and invert the gate's parameterisation for
+            # the raw projection a (input construction only): -ln d = exp(A_log)
+            # softplus(a + dt_bias).
+            if wl.gate_mode == "decay_half_to_one":
+                neg_ln_d = -np.log(uniform(stream_key(wl.seed, "decay", step, r), T * Hv, 0.5, 1.0 - 2.0 ** -8))
+            else:
+                u = uniform(stream_key(wl.seed, "decay", step, r), T * Hv, 0.0, 48.0)
+                tiny = uniform(stream_key(wl.seed, "decay_tiny", step, r), T * Hv, 0.0, 1.0) < 0.125
+                neg_ln_d = np.where(tiny, 200.0, u) * np.log(2.0)
             A = np.tile(w["A_log"].astype(np.float64), T)
-            y = -np.log(d) / np.exp(A)
+            y = neg_ln_d / np.exp(A)
             out["a"].append(np.log(np.expm1(y)) - np.tile(w["dt_bias"].astype(np.float64), T))
     n = len(rows)
     return {

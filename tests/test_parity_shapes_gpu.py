@@ -19,12 +19,12 @@ pytestmark = pytest.mark.gpu
 BASE = synth.WORKLOADS["tiny_d16"]
 
 
-def wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed, slot_mode="sample", std=0.02):
+def wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed, slot_mode="sample", std=0.02, gate_mode="normal"):
     if slot_mode == "permutation":
         P = B
     return BASE.replace(name=name, num_k_heads=Hk, num_v_heads=Hv, head_k_dim=dk, head_v_dim=dv, conv_width=W,
                         batch=B, tokens=T, pool_slots=P, steps=steps, seed=seed, slot_mode=slot_mode,
-                        state_std=std)
+                        state_std=std, gate_mode=gate_mode)
 
 
 SHAPES = [
@@ -44,9 +44,10 @@ SHAPES = [
 
 
 @pytest.mark.parametrize("spec", SHAPES, ids=[s[0] for s in SHAPES])
-def test_fused_matches_oracle(spec):
+def test_fused_matches_oracle(spec, gate_mode="normal"):
     name, Hk, Hv, dk, dv, W, B, T, P, steps = spec
-    wl = wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed=zlib.crc32(name.encode()) % 10000)
+    wl = wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed=zlib.crc32(name.encode()) % 10000,
+               gate_mode=gate_mode)
     g = GpuRun(wl)
     rows = list(range(B))
     o = OracleRun(wl, rows)
@@ -63,6 +64,23 @@ def test_fused_matches_oracle(spec):
     if idle:
         idx = torch.tensor(idle, device="cuda")
         assert torch.equal(g.state[idx], pool0[idx])
+
+
+# Decays from 1 down to fp32 underflow (exp(g) = 2^-u, u up to 48, and 2^-200): the
+# multi-token kernel carries the decay as a running scale and must fold it into the
+# state before it underflows; the single-token kernels multiply directly.
+WIDE_DECAY_SHAPES = [
+    # name               Hk Hv  dk   dv  W   B  T   P  steps
+    ("wide_t16", 2, 4, 128, 128, 4, 3, 16, 4, 2),
+    ("wide_t5_dk16_dv32", 1, 2, 16, 32, 3, 2, 5, 3, 2),
+    ("wide_t1", 2, 4, 64, 64, 4, 3, 1, 5, 2),
+    ("wide_t1_persistent", 4, 8, 128, 128, 4, 40, 1, 48, 2),
+]
+
+
+@pytest.mark.parametrize("spec", WIDE_DECAY_SHAPES, ids=[s[0] for s in WIDE_DECAY_SHAPES])
+def test_wide_decay_matches_oracle(spec):
+    test_fused_matches_oracle(spec, gate_mode="decay_wide")
 
 
 # Single-token launches with many (sequence, k-head) groups take the persistent

@@ -69,3 +69,18 @@ def test_decay_workload_gate_range():
     al, _ = oracle.gate(oracle.Shape.of(wl), x["a"], x["b"], w["A_log"], w["dt_bias"])
     assert al.min() > 0.47 and al.max() < 1.0
     assert al.min() < 0.55 and al.max() > 0.95
+
+
+def test_wide_decay_gate_range():
+    # decay_wide: exp(g) = 2^-u, u ~ U(0, 48), and about one entry in eight at 2^-200
+    import oracle
+    wl = synth.WORKLOADS["batch64"].replace(num_k_heads=2, num_v_heads=4, head_k_dim=16, head_v_dim=16,
+                                             batch=8, tokens=16, pool_slots=8, gate_mode="decay_wide")
+    w = synth.weights(wl)
+    x = synth.step_inputs(wl, 0)
+    al, _ = oracle.gate(oracle.Shape.of(wl), x["a"], x["b"], w["A_log"], w["dt_bias"])
+    log2a = np.log2(np.maximum(al, 1e-300))
+    assert al.max() <= 1.0 and log2a.max() > -2.0          # some decays near 1
+    assert 0.3 < np.mean(log2a < -24.0) < 0.7                # many far below fp32 epsilon
+    tiny = np.mean(log2a < -150.0)
+    assert 0.05 < tiny < 0.25                                # the 2^-200 entries (fp32 underflow)

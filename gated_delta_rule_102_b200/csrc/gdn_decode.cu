@@ -96,28 +96,39 @@ decode_fused_tma_kernel(const DecodeArgs p) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     if (tid == 0) {
-        mbar_init(bar, 1);
+        // a contiguous tile comes by bulk copies (one arrival with the bytes); a strided
+        // one by 16-byte asynchronous copies from every thread (one arrival each)
+        mbar_init(bar, DVS == dv ? 1 : NT);
         mbar_init_fence();
     }
     __syncthreads();
     if (CS > 1) cluster_arrive_relaxed();  // B0
+    // With programmatic dependent launch this grid may start while the previous one
+    // drains: nothing is read before that grid has completed.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const int slot = __ldg(p.slots + seq);
     if (slot < 0 || slot >= p.P) {
         if (tid == 0 && rank == 0 && p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
         return;
     }
     const float* Sbase = p.state_pool + ((size_t)slot * p.sh.Hv + h) * (size_t)DK * dv + col0;
-    if (warp == 0) {  // ---- stage the DK x DVS state tile in with bulk copies
-        if (lane == 0) mbar_arrive_expect_tx(bar, DK * DVS * 4);
-        __syncwarp();
-        if (DVS == dv) {  // contiguous tile: DK/32 rows per copy
+    // ---- stage the DK x DVS state tile in
+    if (DVS == dv) {  // contiguous tile: bulk copies of DK/32 rows each
+        if (warp == 0) {
+            if (lane == 0) mbar_arrive_expect_tx(bar, DK * DVS * 4);
+            __syncwarp();
             constexpr int rows = DK >= 32 ? DK / 32 : 1;
             for (int r = lane * rows; r < DK; r += 32 * rows)
                 tma_load_1d(tile + (size_t)r * DVS, Sbase + (size_t)r * dv, rows * DVS * 4, bar);
-        } else {
-            for (int r = lane; r < DK; r += 32)
-                tma_load_1d(tile + (size_t)r * DVS, Sbase + (size_t)r * dv, DVS * 4, bar);
         }
+    } else {  // rows of DVS columns at the pool's row stride: 16-byte copies from every thread
+        constexpr int VPR = DVS / 4;
+        for (int i = tid; i < DK * VPR; i += NT) {
+            const int r = i / VPR, c = (i - r * VPR) * 4;
+            cp_async_16(tile + (size_t)r * DVS + c, Sbase + (size_t)r * dv + c);
+        }
+        cp_async_arrive(bar);
     }
 
     float* qk = smem + L::qk(T);
@@ -226,13 +237,15 @@ cudaError_t launch_tma(const DecodeArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(Geo::NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)CS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 

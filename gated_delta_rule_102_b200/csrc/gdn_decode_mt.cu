@@ -65,18 +65,8 @@ __device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-// 16-byte asynchronous copy global -> shared (both 16-byte aligned), and the arrival
-// on `bar` once all of this thread's earlier such copies have landed (the arrival
-// counts toward the barrier's expected count: it does not add to it).
-__device__ __forceinline__ void cp_async_16(void* dst_smem, const void* src_gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(dst_smem)), "l"(src_gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_addr(bar)) : "memory");
-}
-
 // SiLU with the hardware exponential and an approximate division (relative error a
-// few ulp; the multi-token conv evaluates it for every channel of every token).
+// few ulp; evaluated for every conv channel and every output element of every token).
 __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 template <int DK, int DV>
@@ -91,15 +81,15 @@ struct MtGeo {
     static constexpr int TILE = DK * DV * 4;
     static_assert(DV % 16 == 0 && RPL >= 2 && (RPL == 2 || RPL % 4 == 0), "multi-token geometry");
     // Shared memory (bytes, every block 16-byte aligned): the stage (NHC state tiles,
-    // the staged raw rows and the weights), then the raw q and k per token, v and o per
-    // v-head and token, the z rows of the pass, the per-token scalars, the stage's slot
-    // and the abort flag, and the stage and z barriers.
+    // the staged raw rows and the weights), then the raw q and k per token, v per v-head
+    // and token (replaced by o: the warp that reads v_t of a column writes o_t of it),
+    // the z rows of the pass, the per-token scalars, the stage's slot and the abort
+    // flag, and the stage and z barriers.
     static __host__ __device__ int rows_off() { return NHC * TILE; }
     static __host__ __device__ int wts_off(int W, int T) { return rows_off() + ((W - 1 + T) * NCHC * 2 + 15) / 16 * 16; }
     static __host__ __device__ int qk_off(int W, int T) { return wts_off(W, T) + (NCHC * W * 2 + 15) / 16 * 16; }
     static __host__ __device__ int vs_off(int W, int T) { return qk_off(W, T) + T * 2 * DK * 4; }
-    static __host__ __device__ int os_off(int W, int T) { return vs_off(W, T) + T * NHC * DV * 4; }
-    static __host__ __device__ int zb_off(int W, int T) { return os_off(W, T) + T * NHC * DV * 4; }
+    static __host__ __device__ int zb_off(int W, int T) { return vs_off(W, T) + T * NHC * DV * 4; }
     static __host__ __device__ int sc_off(int W, int T) { return zb_off(W, T) + T * NHC * DV * 2; }
     static __host__ __device__ int ctl_off(int W, int T) {
         return (sc_off(W, T) + T * NHC * (int)sizeof(TokenScalars) + 15) / 16 * 16;
@@ -128,7 +118,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     uint16_t* wts = reinterpret_cast<uint16_t*>(smem + Geo::wts_off(W, T));
     float* qk = reinterpret_cast<float*>(smem + Geo::qk_off(W, T));
     float* vs = reinterpret_cast<float*>(smem + Geo::vs_off(W, T));
-    float* os = reinterpret_cast<float*>(smem + Geo::os_off(W, T));
+    float* os = vs;  // o_t of a column replaces v_t once the warp owning the column has read it
     uint16_t* zb = reinterpret_cast<uint16_t*>(smem + Geo::zb_off(W, T));
     TokenScalars* sc = reinterpret_cast<TokenScalars*>(smem + Geo::sc_off(W, T));
     volatile int* stage_slot = reinterpret_cast<volatile int*>(smem + Geo::ctl_off(W, T));
@@ -196,6 +186,22 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         mbar_init_fence();
     }
     __syncthreads();
+    // With programmatic dependent launch this grid may start while the previous one
+    // drains (on the SMs its early finishers have left), so the first pass's state
+    // tiles are prefetched into L2 now. The slot read here may be stale: it only steers
+    // the hint, and L2 stays coherent with whatever that grid still writes. Nothing is
+    // read for use before that grid has completed.
+    if (warp == 0 && blockIdx.x < ngroups) {
+        const int seq0 = (int)blockIdx.x / Hk, h00 = ((int)blockIdx.x - seq0 * Hk) * G;
+        const int sl = __ldcg(p.slots + seq0);
+        if (sl >= 0 && sl < p.P) {
+            const char* t0 = reinterpret_cast<const char*>(p.state_pool + ((size_t)sl * Hv + h00) * (size_t)(DK * DV));
+            for (int c = lane * kMtChunk; c < NH * Geo::TILE; c += 32 * kMtChunk)
+                bulk_prefetch_l2(t0 + c, (uint32_t)min(kMtChunk, NH * Geo::TILE - c));
+        }
+    }
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     prefetch(0, slot_of(0));
 
     const int rg = lane >> 2, cg = lane & 3;
@@ -274,6 +280,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                 // before token 0's shift position m holds staged row j - 1 (history rows only)
                 win[m] = j >= 1 ? bf16_bits_to_float(rows[(j - 1) * NCH + lc]) : 0.f;
             }
+#pragma unroll 4
             for (int t = 0; t < T; ++t) {
 #pragma unroll
                 for (int m = 0; m < kMaxConvWidth - 1; ++m) win[m] = win[m + 1];
@@ -392,6 +399,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                     d[cc] = st.beta * fmaf(-am, mk[cc], vv[cc]);
                     o[cc] = fmaf(aqs, mq[cc], d[cc] * st.kq);
                 }
+                __syncwarp();  // every lane has read v_t of these columns before o_t replaces it
                 if (rg == 0) *reinterpret_cast<float4*>(os + (hh * T + t) * DV + col) = make_float4(o[0], o[1], o[2], o[3]);
                 float f;  // the update's factor on the raw k: nk delta / c, with c the new scale
                 if (c1 < 0x1p-64f) {  // fold the scale into the registers before it underflows
@@ -466,10 +474,10 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
             const float inv = rsqrtf(ss / (float)DV + p.sh.rms_eps);
             const size_t base = (((size_t)seq * T + t) * Hv + h0 + k) * DV + 4 * lane;
             const uint2 zz = *reinterpret_cast<const uint2*>(zb + (t * NH + k) * DV + 4 * lane);
-            const float y0 = o.x * inv * bf16_bits_to_float(nw.x & 0xffffu) * silu(bf16_bits_to_float(zz.x & 0xffffu));
-            const float y1 = o.y * inv * bf16_bits_to_float(nw.x >> 16) * silu(bf16_bits_to_float(zz.x >> 16));
-            const float y2 = o.z * inv * bf16_bits_to_float(nw.y & 0xffffu) * silu(bf16_bits_to_float(zz.y & 0xffffu));
-            const float y3 = o.w * inv * bf16_bits_to_float(nw.y >> 16) * silu(bf16_bits_to_float(zz.y >> 16));
+            const float y0 = o.x * inv * bf16_bits_to_float(nw.x & 0xffffu) * silu_fast(bf16_bits_to_float(zz.x & 0xffffu));
+            const float y1 = o.y * inv * bf16_bits_to_float(nw.x >> 16) * silu_fast(bf16_bits_to_float(zz.x >> 16));
+            const float y2 = o.z * inv * bf16_bits_to_float(nw.y & 0xffffu) * silu_fast(bf16_bits_to_float(zz.y & 0xffffu));
+            const float y3 = o.w * inv * bf16_bits_to_float(nw.y >> 16) * silu_fast(bf16_bits_to_float(zz.y >> 16));
             uint2 packed;
             packed.x = (uint32_t)float_to_bf16_bits(y0) | ((uint32_t)float_to_bf16_bits(y1) << 16);
             packed.y = (uint32_t)float_to_bf16_bits(y2) | ((uint32_t)float_to_bf16_bits(y3) << 16);
@@ -506,8 +514,17 @@ cudaError_t launch_mt(const DecodeArgs& a, cudaStream_t stream) {
     const int ngroups = a.B * a.sh.Hk;
     const int grid = ngroups < sms * per_sm ? ngroups : sms * per_sm;
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, Geo::NT, smem, stream>>>(a, heads_per_pass<DK, DV>(a.sh.Hv / a.sh.Hk));
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(Geo::NT);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, heads_per_pass<DK, DV>(a.sh.Hv / a.sh.Hk));
 }
 
 template <int DK>

@@ -77,13 +77,24 @@ def algorithmic_flops(wl) -> int:
     return 7 * wl.batch * wl.tokens * wl.num_v_heads * wl.head_k_dim * wl.head_v_dim
 
 
-def kernel_source_hash() -> str:
+# The sources each decode kernel is compiled from (its own file and the shared headers).
+KERNEL_SOURCES = {
+    "decode_ws_kernel": ("gdn_decode_persistent.cu",),
+    "decode_mt_kernel": ("gdn_decode_mt.cu",),
+    "decode_fused_tma_kernel": ("gdn_decode.cu",),
+}
+SHARED_SOURCES = ("gdn_device.cuh", "gdn_internal.h")
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources `kernel` is built from: a profile taken on other sources of
+    this kernel no longer describes it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_102_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(f.encode())
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in sorted(KERNEL_SOURCES.get(kernel, ()) + SHARED_SOURCES):
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "gdn.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -96,7 +107,7 @@ def profiled_traffic(kernel: str, wl_name: str):
     txt = open(path).read()
     m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
     m_bytes = re.search(r"dram bytes per launch:\s*`?([0-9]+)", txt)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(kernel):
         return None
     return int(m_bytes.group(1))
 

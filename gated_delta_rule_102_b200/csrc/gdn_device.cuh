@@ -436,19 +436,3 @@ __device__ __forceinline__ void st_async_f32x2(uint32_t remote_addr, float a, fl
                  : "memory");
 }
 }  // namespace gdn
-
-namespace gdn {
-// Bulk copy of `bytes` from this CTA's shared memory to global memory (both 16-byte
-// aligned, size a multiple of 16), tracked in this thread's bulk async-group.
-__device__ __forceinline__ void tma_store_1d(void* dst_gmem, const void* src_smem, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst_gmem),
-                 "r"(smem_addr(src_smem)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
-// Waits until every committed bulk group of this thread has finished reading its
-// shared-memory source (the writes to global memory may still be in flight).
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
-// Waits until every committed bulk group of this thread has completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
-}  // namespace gdn

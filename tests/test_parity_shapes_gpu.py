@@ -325,3 +325,46 @@ def test_dynamic_and_static_schedules_agree(spec):
         assert torch.equal(od32, os32) and torch.equal(od, os_)
         assert int(dyn.workspace.abs().sum().item()) == 0
     assert torch.equal(dyn.state, sta.state) and torch.equal(dyn.conv, sta.conv)
+
+
+# Launches of different token counts on the same pools (a chunk of several tokens, then
+# single tokens, and so on) must act like the same tokens run in order. The kernels
+# for one token and for several differ, and a launch may begin while the previous one
+# drains (programmatic dependent launch): every read of a pool waits for that grid.
+MIXED = [
+    # name          Hk Hv   dk   dv  W   B   P   token counts of the launches
+    ("mixed_small", 2, 4, 128, 128, 4, 3, 5, [5, 1, 16, 1, 1, 3, 2]),        # cluster kernel for T = 1
+    ("mixed_persist", 4, 8, 128, 128, 4, 40, 43, [1, 4, 1, 1, 16, 1]),      # persistent kernel for T = 1
+    ("mixed_w3_dv64", 2, 8, 64, 64, 3, 5, 6, [2, 1, 7, 1]),
+]
+
+
+@pytest.mark.parametrize("spec", MIXED, ids=[m[0] for m in MIXED])
+def test_mixed_token_counts_share_pools(spec):
+    name, Hk, Hv, dk, dv, W, B, P, counts = spec
+    wl1 = wl_of(name, Hk, Hv, dk, dv, W, B, 1, P, len(counts), seed=zlib.crc32(name.encode()) % 10000)
+    g = GpuRun(wl1)
+    rows = sorted({0, B // 2, B - 1})
+    o = OracleRun(wl1, rows)
+    pool0 = g.state.clone()
+    for i, T in enumerate(counts):
+        wl = wl1.replace(tokens=T)
+        x = {k: bf16_dev(v) for k, v in synth.step_inputs(wl, i).items()}
+        shape = (B, T, Hv, dv)
+        out = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        out32 = torch.empty(shape, dtype=torch.float32, device="cuda")
+        gdn.gdn_decode_step(g.cfg, x["qkv"], x["a"], x["b"], x["z"], g.conv_w, g.A_log, g.dt_bias, g.norm_w, g.conv,
+                            g.state, g.slots, out, out32, g.err, g.workspace)
+        xr = synth.step_inputs(wl, i, rows=rows)
+        w = o.w
+        r = oracle.decode_step(o.shape, xr["qkv"], xr["a"], xr["b"], xr["z"], w["conv_w"], w["A_log"], w["dt_bias"],
+                               w["norm_w"], o.conv, o.state, o.local)
+        compare_out(out, out32, r["out"], rows, f"{name} launch {i} (T={T})")
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == 0
+    compare_state(g.state, o.state, o.slot_ids, name)
+    np.testing.assert_array_equal(bf16_host(g.conv)[o.slot_ids], o.conv)
+    idle = sorted(set(range(P)) - set(g.slots_np.tolist()))
+    if idle:
+        idx = torch.tensor(idle, device="cuda")
+        assert torch.equal(g.state[idx], pool0[idx])

@@ -33,7 +33,7 @@ def cfg_of(wl: synth.Workload) -> gdn.GdnConfig:
     return gdn.GdnConfig.make(wl.num_k_heads, wl.num_v_heads, wl.head_k_dim, wl.head_v_dim, wl.conv_width)
 
 
-class GpuRun:
+class DeviceRun:
     """The workload on the GPU: weights, pools and slots resident on the device."""
 
     def __init__(self, wl: synth.Workload, device="cuda", state0: Optional[np.ndarray] = None,

@@ -12,13 +12,13 @@ import pytest
 import torch
 
 from gated_delta_rule_102_b200 import synth
-from gdn_harness import (GpuRun, OracleRun, bf16_host, compare_out, compare_state, conv_pool_reference)
+from gdn_harness import (DeviceRun, OracleRun, bf16_host, compare_out, compare_state, conv_pool_reference)
 
 pytestmark = pytest.mark.gpu
 
 
 def _run(wl, rows, check_every=1):
-    g = GpuRun(wl)
+    g = DeviceRun(wl)
     o = OracleRun(wl, rows)
     pool0 = g.state.clone() if wl.pool_slots > wl.batch else None
     worst_out = 0.0

@@ -11,7 +11,7 @@ import torch
 import gated_delta_rule_102_b200 as gdn
 import oracle
 from gated_delta_rule_102_b200 import synth
-from gdn_harness import (GpuRun, OracleRun, bf16_dev, bf16_host, compare_out, compare_state, conv_pool_reference,
+from gdn_harness import (DeviceRun, OracleRun, bf16_dev, bf16_host, compare_out, compare_state, conv_pool_reference,
                          f32_dev)
 
 pytestmark = pytest.mark.gpu
@@ -48,7 +48,7 @@ def test_fused_matches_oracle(spec, gate_mode="normal"):
     name, Hk, Hv, dk, dv, W, B, T, P, steps = spec
     wl = wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed=zlib.crc32(name.encode()) % 10000,
                gate_mode=gate_mode)
-    g = GpuRun(wl)
+    g = DeviceRun(wl)
     rows = list(range(B))
     o = OracleRun(wl, rows)
     pool0 = g.state.clone()
@@ -103,7 +103,7 @@ def test_persistent_path_matches_oracle(spec):
 
 def test_persistent_path_bad_slot():
     wl = wl_of("p_badslot", 4, 8, 128, 128, 4, 40, 1, 40, 1, seed=21, slot_mode="permutation")
-    g = GpuRun(wl)
+    g = DeviceRun(wl)
     slots = g.slots_np.copy()
     slots[17] = 40  # outside the 40-slot pool
     g.slots = torch.from_numpy(slots).cuda()
@@ -129,7 +129,7 @@ def test_persistent_path_bad_slot():
 
 def _stage_problem(seed=5, Hk=2, Hv=4, dk=64, dv=128, W=4, B=3, T=3, P=4):
     wl = wl_of("stages", Hk, Hv, dk, dv, W, B, T, P, 1, seed)
-    return wl, GpuRun(wl), synth.step_inputs(wl, 0)
+    return wl, DeviceRun(wl), synth.step_inputs(wl, 0)
 
 
 def test_conv_stage_matches_oracle():
@@ -185,7 +185,7 @@ def test_gated_rmsnorm_stage_matches_oracle():
 
 def test_fused_equals_stage_chain():
     wl, g, x = _stage_problem(seed=8, T=2)
-    g2 = GpuRun(wl)
+    g2 = DeviceRun(wl)
     B, T = wl.batch, wl.tokens
     out, out32 = g.step({k: bf16_dev(v) for k, v in x.items()})
     q = torch.empty(B, T, wl.num_k_heads, wl.head_k_dim, device="cuda")
@@ -206,7 +206,7 @@ def test_fused_equals_stage_chain():
 
 def test_out_of_range_slot_is_skipped_and_flagged():
     wl = wl_of("badslot", 2, 4, 32, 32, 4, 3, 1, 4, 1, seed=9)
-    g = GpuRun(wl)
+    g = DeviceRun(wl)
     g.slots = torch.tensor([1, 7, 3], dtype=torch.int32, device="cuda")  # 7 is outside the 4-slot pool
     g.slots_np = g.slots.cpu().numpy()
     state0, conv0 = g.state.clone(), g.conv.clone()
@@ -238,7 +238,7 @@ def test_out_of_range_slot_is_skipped_and_flagged():
 
 def test_empty_batch_is_a_no_op_on_device():
     wl = wl_of("empty", 2, 4, 32, 32, 4, 2, 1, 2, 1, seed=10)
-    g = GpuRun(wl)
+    g = DeviceRun(wl)
     st, cv = g.state.clone(), g.conv.clone()
     e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device="cuda")  # noqa: E731
     gdn.gdn_decode_step(g.cfg, e(0, 1, wl.channels), e(0, 1, 4), e(0, 1, 4), e(0, 1, 4, 32), g.conv_w, g.A_log,
@@ -251,14 +251,14 @@ def test_split_run_resumes_bit_identically():
     # N steps, pools copied to the host and back into fresh buffers, M more steps:
     # the same bits as N + M steps in one go (the pools are the whole resumable state).
     wl = wl_of("resume", 2, 4, 64, 64, 4, 4, 2, 6, 6, seed=11)
-    a = GpuRun(wl)
+    a = DeviceRun(wl)
     for s in range(6):
         out_a, _ = a.step(a.inputs(s))
-    b = GpuRun(wl)
+    b = DeviceRun(wl)
     for s in range(3):
         b.step(b.inputs(s))
     state_host, conv_host = b.state.cpu(), b.conv.cpu()
-    c = GpuRun(wl)
+    c = DeviceRun(wl)
     c.state.copy_(state_host.cuda())
     c.conv.copy_(conv_host.cuda())
     for s in range(3, 6):
@@ -269,7 +269,7 @@ def test_split_run_resumes_bit_identically():
 
 def test_deterministic():
     wl = wl_of("det", 2, 4, 128, 128, 4, 8, 1, 8, 1, seed=12, slot_mode="permutation")
-    a, b = GpuRun(wl), GpuRun(wl)
+    a, b = DeviceRun(wl), DeviceRun(wl)
     x = a.inputs(0)
     oa, oa32 = a.step(x)
     ob, ob32 = b.step(x)
@@ -285,12 +285,12 @@ def test_step_replays_from_a_cuda_graph(name):
                                                                  num_v_heads=8),
             "tiny_d16": synth.WORKLOADS["tiny_d16"],
             "multitoken": synth.WORKLOADS["multitoken_b32_t16"].replace(batch=4, pool_slots=4)}[name]
-    eager, graphed = GpuRun(base), GpuRun(base)
+    eager, graphed = DeviceRun(base), DeviceRun(base)
     xs = [eager.inputs(s) for s in range(3)]
     outs_e = [eager.step(x)[1].clone() for x in xs]
     graphed.step(xs[0])  # first call on the device outside the capture (one-time set-up)
-    graphed.state.copy_(GpuRun(base).state)
-    graphed.conv.copy_(GpuRun(base).conv)
+    graphed.state.copy_(DeviceRun(base).state)
+    graphed.conv.copy_(DeviceRun(base).conv)
     shape = (base.batch, base.tokens, base.num_v_heads, base.head_v_dim)
     outs = [torch.empty(shape, device="cuda") for _ in xs]
     outb = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
@@ -316,7 +316,7 @@ def test_dynamic_and_static_schedules_agree(spec):
     # and the workspace is left zeroed for the next call
     name, Hk, Hv, dk, dv, W, B, T, P, steps = spec
     wl = wl_of(name, Hk, Hv, dk, dv, W, B, T, P, steps, seed=77)
-    dyn, sta = GpuRun(wl, dynamic=True), GpuRun(wl, dynamic=False)
+    dyn, sta = DeviceRun(wl, dynamic=True), DeviceRun(wl, dynamic=False)
     for s in range(steps):
         x = dyn.inputs(s)
         od, od32 = dyn.step(x)
@@ -343,7 +343,7 @@ MIXED = [
 def test_mixed_token_counts_share_pools(spec):
     name, Hk, Hv, dk, dv, W, B, P, counts = spec
     wl1 = wl_of(name, Hk, Hv, dk, dv, W, B, 1, P, len(counts), seed=zlib.crc32(name.encode()) % 10000)
-    g = GpuRun(wl1)
+    g = DeviceRun(wl1)
     rows = sorted({0, B // 2, B - 1})
     o = OracleRun(wl1, rows)
     pool0 = g.state.clone()

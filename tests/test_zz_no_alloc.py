@@ -12,7 +12,7 @@ import torch
 
 import gated_delta_rule_102_b200 as gdn
 from gated_delta_rule_102_b200 import synth
-from gdn_harness import OUT_ABS_TOL, STATE_REL_TOL, GpuRun, bf16_host
+from gdn_harness import OUT_ABS_TOL, STATE_REL_TOL, DeviceRun, bf16_host
 
 pytestmark = pytest.mark.gpu
 
@@ -21,8 +21,8 @@ def test_static_scratch_matches_the_workspace_entry_point_on_two_calls_in_a_row(
     # batch64 shape: the single-token kernel that uses the scratch runs here
     wl = synth.WORKLOADS["batch64"].replace(steps=2)
     assert gdn.decode_static_scratch_bytes() >= gdn.decode_workspace_bytes()
-    ref = GpuRun(wl, dynamic=True)     # gdn_decode_step with a caller-allocated workspace
-    nal = GpuRun(wl, dynamic=False)    # same weights, pools and slots; no workspace at all
+    ref = DeviceRun(wl, dynamic=True)     # gdn_decode_step with a caller-allocated workspace
+    nal = DeviceRun(wl, dynamic=False)    # same weights, pools and slots; no workspace at all
     shape = (wl.batch, wl.tokens, wl.num_v_heads, wl.head_v_dim)
     for step in range(2):
         x = ref.inputs(step)

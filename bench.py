@@ -86,15 +86,24 @@ KERNEL_SOURCES = {
 SHARED_SOURCES = ("gdn_device.cuh", "gdn_internal.h")
 
 
+def _code_only(text: str) -> bytes:
+    """C/C++ source without its comments and blank space: edits to comments do not
+    change the kernel a profile describes."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split()).encode()
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources `kernel` is built from: a profile taken on other sources of
-    this kernel no longer describes it."""
+    """Hash of the code `kernel` is built from (its own file, the shared headers and the
+    C-ABI header, comments left out): a profile taken on other code of this kernel no
+    longer describes it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_102_b200", "csrc")
     for f in sorted(KERNEL_SOURCES.get(kernel, ()) + SHARED_SOURCES):
         h.update(f.encode())
-        h.update(open(os.path.join(csrc, f), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "gdn.h"), "rb").read())
+        h.update(_code_only(open(os.path.join(csrc, f)).read()))
+    h.update(_code_only(open(os.path.join(ROOT, "include", "gdn.h")).read()))
     return h.hexdigest()[:16]
 
 

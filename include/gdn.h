@@ -144,6 +144,10 @@ gdn_status gdn_gated_rmsnorm(const gdn_config* cfg, int32_t rows, const float* o
  *            time on the GPU need separate workspaces.
  * The first call on a device (per shape) queries the device once and sets a kernel
  * attribute; make it before capturing the call into a CUDA graph.
+ * The launch allows programmatic stream serialization: the kernel may begin while the
+ * kernel before it in the stream drains, but it reads nothing (inputs, pools, slots,
+ * workspace) before that kernel has completed; until then it only issues L2 prefetch
+ * hints for the first state tiles it will read.
  */
 gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv,
                            const uint16_t* a, const uint16_t* b, const uint16_t* z,

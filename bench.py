@@ -115,7 +115,7 @@ def profiled_traffic(kernel: str, wl_name: str):
         return None
     txt = open(path).read()
     m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
-    m_bytes = re.search(r"dram bytes per launch:\s*`?([0-9]+)", txt)
+    m_bytes = re.search(r"dram bytes per launch:\s*\|?\s*`?([0-9]+)", txt)
     if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(kernel):
         return None
     return int(m_bytes.group(1))

@@ -25,9 +25,10 @@ GDN_ERR_SLOT_RANGE = 4
 GDN_ERR_CUDA = 5
 GDN_DEVICE_ERR_SLOT_RANGE = 1
 GDN_DEVICE_ERR_TIMEOUT = 2
+GDN_DEVICE_ERR_SEQLEN = 4
 
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
-           "gdn_decode_workspace_bytes", "gdn_decode_step_static_scratch", "gdn_decode_static_scratch_bytes",
+           "gdn_decode_workspace_bytes", "gdn_decode_step_varlen", "gdn_decode_step_static_scratch", "gdn_decode_static_scratch_bytes",
            "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
 
 
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_recurrent_step.argtypes = [cfgp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
         L.gdn_gated_rmsnorm.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp]
         L.gdn_decode_step.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_decode_step_varlen.argtypes = [cfgp, i32, vp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp]
         L.gdn_decode_workspace_bytes.argtypes = []
         L.gdn_decode_workspace_bytes.restype = ctypes.c_size_t
         L.gdn_decode_step_static_scratch.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp]
@@ -81,7 +83,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_abi_version.argtypes = []
         for f in ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
-                  "gdn_check_slots_host", "gdn_abi_version"):
+                  "gdn_decode_step_varlen", "gdn_check_slots_host", "gdn_abi_version"):
             getattr(L, f).restype = ctypes.c_int32
         _lib = L
     return _lib
@@ -163,6 +165,22 @@ def gdn_decode_step(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w
                                  _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
                                  _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
                                  _ptr(workspace, _WS, "workspace"), _stream(stream, qkv)), "gdn_decode_step")
+
+
+def gdn_decode_step_varlen(cfg: GdnConfig, cu_seqlens, T_max: int, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w,
+                           conv_pool, state_pool, slots, out, out_f32=None, err_flag=None, stream=None) -> None:
+    """The decode step for sequences with their own token counts, packed row after row:
+    sequence i owns rows cu_seqlens[i] .. cu_seqlens[i+1]-1 of qkv [total][C], a, b
+    [total][Hv], z and out [total][Hv][dv]; T_max bounds every count."""
+    B = cu_seqlens.shape[0] - 1
+    total = qkv.shape[0]
+    _check(lib().gdn_decode_step_varlen(
+        ctypes.byref(cfg), B, _ptr(cu_seqlens, _I32, "cu_seqlens"), int(T_max), total, _ptr(qkv, _BF16, "qkv"),
+        _ptr(a, _BF16, "a"), _ptr(b, _BF16, "b"), _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"),
+        _ptr(A_log, _F32, "A_log"), _ptr(dt_bias, _F32, "dt_bias"), _ptr(norm_w, _BF16, "norm_w"),
+        _ptr(conv_pool, _BF16, "conv_pool"), _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0],
+        _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"), _ptr(out_f32, _F32, "out_f32"),
+        _ptr(err_flag, _I32, "err_flag"), _stream(stream, qkv)), "gdn_decode_step_varlen")
 
 
 def gdn_decode_step_static_scratch(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool,

@@ -135,6 +135,30 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
 
 size_t gdn_decode_workspace_bytes(void) { return 64; }
 
+gdn_status gdn_decode_step_varlen(const gdn_config* cfg, int32_t B, const int32_t* cu_seqlens, int32_t T_max,
+                                  int32_t total_tokens, const uint16_t* qkv, const uint16_t* a, const uint16_t* b,
+                                  const uint16_t* z, const uint16_t* conv_w, const float* A_log,
+                                  const float* dt_bias, const uint16_t* norm_w, uint16_t* conv_pool,
+                                  float* state_pool, int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
+                                  float* out_f32, int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if (total_tokens < 0) return GDN_ERR_INVALID_ARGUMENT;
+    if ((st = check_batch(B, T_max, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0 || total_tokens == 0) return GDN_OK;  // no sequence has a token: nothing to do
+    if (!cu_seqlens) return GDN_ERR_INVALID_ARGUMENT;
+    if (((uintptr_t)cu_seqlens & 3u) != 0) return GDN_ERR_MISALIGNED;
+    if ((st = check_pointers({conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots}, {out_f32, err_flag})) !=
+        GDN_OK)
+        return st;
+    if ((st = check_pointers({qkv, a, b, z, out_bf16}, {})) != GDN_OK) return st;
+    gdn::DecodeArgs d{sh, B, T_max, pool_slots, 1, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool,
+                      state_pool, slots, out_bf16, out_f32, err_flag, nullptr, cu_seqlens, total_tokens};
+    if (!gdn::multitoken_supported(d)) return GDN_ERR_UNSUPPORTED;
+    return from_cuda(gdn::launch_decode_multitoken(d, (cudaStream_t)stream));
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------

@@ -1,8 +1,10 @@
-// Fused GDN decode step for launches of several tokens per sequence (T = 2..16):
+// Fused GDN decode step for launches of several tokens per sequence (up to 16):
 // steps 3 to 8 and the SiLU(z) gate of steps 9+10+11 on the page
 // "spark_model/forward/qwen3_5/linear_attention.rs", applied to the tokens of the
 // launch in order with the state kept on chip in between (the tokens of one launch
-// behave exactly like T single-token calls).
+// behave exactly like single-token calls, one per token). Every sequence has T tokens,
+// or, with per-sequence offsets into packed rows, its own count up to T (none: the
+// sequence is left as it is).
 //
 // Work. Persistent CTAs, one per SM, walk the (sequence, k-head) groups cid,
 // cid + grid, ... A group's G v-heads are taken NH at a time (a "pass"); a pass
@@ -95,6 +97,8 @@ struct MtGeo {
         return (sc_off(W, T) + T * NHC * (int)sizeof(TokenScalars) + 15) / 16 * 16;
     }
     static __host__ __device__ int total(int W, int T) { return ctl_off(W, T) + 32; }
+    // the control block: the stage's slot, the abort flag, the stage and z barriers,
+    // the stage's first packed row and token count
 };
 
 // Row held by lane row group rg in register block j, element e.
@@ -109,8 +113,9 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     using Geo = MtGeo<DK, DV>;
     constexpr int RPL = Geo::RPL, NB = RPL == 2 ? 1 : RPL / 4, EPB = RPL == 2 ? 2 : 4;
     extern __shared__ __align__(128) unsigned char smem[];
+    // T: the most tokens a sequence has in this launch (it sizes the shared buffers)
     const int T = p.T, W = p.sh.W, C = p.sh.C, Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk;
-    const int npass = G / NH, NCH = 2 * DK + NH * DV, nrow = W - 1 + T;
+    const int npass = G / NH, NCH = 2 * DK + NH * DV;
     const int ngroups = p.B * Hk;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float* stage = reinterpret_cast<float*>(smem);
@@ -125,29 +130,38 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     volatile int* abort_flag = stage_slot + 1;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Geo::ctl_off(W, T) + 8);
     uint64_t* zbar = full + 1;
+    volatile int* stage_tok0 = reinterpret_cast<volatile int*>(zbar + 1);  // the stage's first packed row
+    volatile int* stage_ntok = stage_tok0 + 1;                             // and its token count
 
     auto item_group = [&](int u) { return (int)blockIdx.x + (u / npass) * (int)gridDim.x; };
     // Every thread: the copies of pass u into the stage (or, past the last pass,
-    // nothing); `slot` is the pass's pool slot, read beforehand. The barrier expects
-    // one arrival per thread (its asynchronous copies) and the tile bytes' arrival.
-    auto prefetch = [&](int u, int slot) {
+    // nothing); `slot` is the pass's pool slot, `tok0` and `ntok` its sequence's first
+    // packed row and token count, all read beforehand. The barrier expects one arrival
+    // per thread (its asynchronous copies) and the tile bytes' arrival.
+    auto prefetch = [&](int u, int slot, int tok0, int ntok) {
         const int group = item_group(u);
         if (group >= ngroups) return;
         const int seq = group / Hk, hk = group - seq * Hk, h0 = hk * G + (u % npass) * NH;
-        if (slot < 0 || slot >= p.P) {  // skipped and flagged
+        const bool bad_slot = slot < 0 || slot >= p.P;
+        const bool bad_len = ntok < 0 || ntok > T || (p.cu_seqlens && (tok0 < 0 || tok0 + ntok > p.total_rows));
+        if (bad_slot || bad_len || ntok == 0) {  // skipped (flagged unless it simply has no tokens)
             if (tid == 0) {
-                if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
+                if (p.err_flag && bad_slot) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
+                if (p.err_flag && bad_len) atomicOr(p.err_flag, GDN_DEVICE_ERR_SEQLEN_BIT);
                 *stage_slot = -1;
                 mbar_arrive(full);
             }
             mbar_arrive(full);
             return;
         }
+        const int nrow = W - 1 + ntok;
         const int ch_q = hk * DK, ch_k = Hk * DK + hk * DK, ch_v = 2 * Hk * DK + h0 * DV;
         auto run_channel = [&](int lc) { return lc < DK ? ch_q + lc : (lc < 2 * DK ? ch_k + lc - DK : ch_v + lc - 2 * DK); };
         if (warp == 0) {  // the NH state tiles, contiguous in the pool
             if (lane == 0) {
                 *stage_slot = slot;
+                *stage_tok0 = tok0;
+                *stage_ntok = ntok;
                 mbar_arrive_expect_tx(full, (uint32_t)(NH * Geo::TILE));
             }
             __syncwarp();
@@ -161,7 +175,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         // channels' weights ([channel][W], three runs of consecutive channels; a 16-byte
         // group never straddles two runs since every run holds a multiple of 8 channels)
         const uint16_t* hist = p.conv_pool + (size_t)slot * (W - 1) * C;
-        const uint16_t* x = p.qkv + (size_t)seq * T * C;
+        const uint16_t* x = p.qkv + (size_t)tok0 * C;
         const int nv = NCH / 8;
         for (int i = tid; i < nrow * nv; i += Geo::NT) {
             const int r = i / nv, lc = (i - r * nv) * 8, ch = run_channel(lc);
@@ -172,6 +186,20 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
             cp_async_16(wts + i * 8, p.conv_w + (size_t)run_channel(lc) * W + off);
         }
         cp_async_arrive(full);
+    };
+    // the first packed row and the token count of pass u's sequence
+    auto tokens_of = [&](int u, int& tok0, int& ntok) {
+        const int group = item_group(u);
+        if (group >= ngroups) {
+            tok0 = ntok = 0;
+        } else if (p.cu_seqlens) {
+            const int seq = group / Hk;
+            tok0 = __ldg(p.cu_seqlens + seq);
+            ntok = __ldg(p.cu_seqlens + seq + 1) - tok0;
+        } else {
+            tok0 = (group / Hk) * T;
+            ntok = T;
+        }
     };
 
     // the slot of pass u (-1 past the last pass)
@@ -202,7 +230,11 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     }
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-    prefetch(0, slot_of(0));
+    {
+        int tok0 = 0, ntok = 0;
+        tokens_of(0, tok0, ntok);
+        prefetch(0, slot_of(0), tok0, ntok);
+    }
 
     const int rg = lane >> 2, cg = lane & 3;
     const bool active = warp < Geo::NWH * NH;  // warps holding state columns in this launch's passes
@@ -222,29 +254,31 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
             }
             break;
         }
-        const int slot = *stage_slot;
-        // the next pass's slot (the same sequence for the group's next pass): loaded now,
-        // first used when the next copies are issued
-        const int next_slot = (u + 1) % npass != 0 ? slot : slot_of(u + 1);
+        const int slot = *stage_slot, tok0 = *stage_tok0, ntok = *stage_ntok;
+        // the next pass's slot and tokens: loaded now, first used when the next copies
+        // are issued
+        const int next_slot = slot_of(u + 1);
+        int next_tok0 = 0, next_ntok = 0;
+        tokens_of(u + 1, next_tok0, next_ntok);
         if (slot < 0) {
             __syncthreads();  // every thread has read the stage's slot
-            prefetch(u + 1, next_slot);
+            prefetch(u + 1, next_slot, next_tok0, next_ntok);
             continue;
         }
         {  // this pass's z rows (their buffer was last read before the barrier above)
             const int nv = NH * DV / 8;
-            for (int i = tid; i < T * nv; i += Geo::NT) {
+            for (int i = tid; i < ntok * nv; i += Geo::NT) {
                 const int t = i / nv, o = (i - t * nv) * 8;
-                cp_async_16(zb + t * NH * DV + o, p.z + (((size_t)seq * T + t) * Hv + h0) * DV + o);
+                cp_async_16(zb + t * NH * DV + o, p.z + (((size_t)tok0 + t) * Hv + h0) * DV + o);
             }
             cp_async_arrive(zbar);
         }
         // the gate inputs of this pass's heads, loaded now and used after the conv
         uint16_t g_a = 0, g_b = 0;
         float g_A = 0.f, g_dt = 0.f;
-        if (tid < T * NH) {
+        if (tid < ntok * NH) {
             const int t = tid / NH, k = tid - t * NH;
-            const size_t ai = ((size_t)seq * T + t) * Hv + h0 + k;
+            const size_t ai = ((size_t)tok0 + t) * Hv + h0 + k;
             g_a = p.a[ai];
             g_b = p.b[ai];
             g_A = p.A_log[h0 + k];
@@ -281,7 +315,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                 win[m] = j >= 1 ? bf16_bits_to_float(rows[(j - 1) * NCH + lc]) : 0.f;
             }
 #pragma unroll 4
-            for (int t = 0; t < T; ++t) {
+            for (int t = 0; t < ntok; ++t) {
 #pragma unroll
                 for (int m = 0; m < kMaxConvWidth - 1; ++m) win[m] = win[m + 1];
                 win[kMaxConvWidth - 1] = bf16_bits_to_float(rows[(t + W - 1) * NCH + lc]);
@@ -307,18 +341,18 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                 const int r = i / nvec, lc = lc0 + (i - r * nvec) * 8;
                 const int ch = lc < DK ? ch_q + lc : (lc < 2 * DK ? ch_k + lc - DK : ch_v + lc - 2 * DK);
                 *reinterpret_cast<uint4*>(hw + (size_t)r * C + ch) =
-                    *reinterpret_cast<const uint4*>(rows + (T + r) * NCH + lc);
+                    *reinterpret_cast<const uint4*>(rows + (ntok + r) * NCH + lc);
             }
         }
         // ---- steps 4, 5: decay and write strength per v-head and token
-        if (tid < T * NH) {
+        if (tid < ntok * NH) {
             const int t = tid / NH, k = tid - t * NH;
             gate_and_beta(g_a, g_b, g_A, g_dt, sc[t * Geo::NHC + k].alpha, sc[t * Geo::NHC + k].beta);
         }
         __syncthreads();  // the stage is empty; k, q, v are in
-        prefetch(u + 1, next_slot);
+        prefetch(u + 1, next_slot, next_tok0, next_ntok);
         // ---- L2 norms of q and k (step 3) as factors on the raw values, and k.q: a warp per token
-        for (int t = warp; t < T; t += Geo::NW) {
+        for (int t = warp; t < ntok; t += Geo::NW) {
             float sq = 0.f, sk = 0.f, dot = 0.f;
             for (int r = lane; r < DK; r += 32) {
                 const float a = qk[t * 2 * DK + r], b = qk[t * 2 * DK + DK + r];
@@ -345,7 +379,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         // ---- steps 6, 7: the recurrence, token by token, on this warp's columns
         if (active) {
             float c = 1.f;  // S = c * S~ (the registers hold S~)
-            for (int t = 0; t < T; ++t) {
+            for (int t = 0; t < ntok; ++t) {
                 const float* qr = qk + t * 2 * DK;
                 const float* kr = qr + DK;
                 f2 ak[4], aq[4];  // per column: S~^T k and S~^T q over the even and the odd rows
@@ -463,7 +497,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
             }
         }
         ++zphase;
-        for (int task = warp; task < T * NH; task += Geo::NW) {
+        for (int task = warp; task < ntok * NH; task += Geo::NW) {
             const int t = task / NH, k = task - t * NH;
             const float4 o = has_cols ? reinterpret_cast<const float4*>(os + (k * T + t) * DV)[lane]
                                       : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -472,7 +506,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
             for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
             if (!has_cols) continue;
             const float inv = rsqrtf(ss / (float)DV + p.sh.rms_eps);
-            const size_t base = (((size_t)seq * T + t) * Hv + h0 + k) * DV + 4 * lane;
+            const size_t base = (((size_t)tok0 + t) * Hv + h0 + k) * DV + 4 * lane;
             const uint2 zz = *reinterpret_cast<const uint2*>(zb + (t * NH + k) * DV + 4 * lane);
             const float y0 = o.x * inv * bf16_bits_to_float(nw.x & 0xffffu) * silu_fast(bf16_bits_to_float(zz.x & 0xffffu));
             const float y1 = o.y * inv * bf16_bits_to_float(nw.x >> 16) * silu_fast(bf16_bits_to_float(zz.x >> 16));

@@ -15,6 +15,7 @@ namespace gdn {
 // Bits a kernel ORs into the caller's error flag (values of the public header).
 constexpr int GDN_DEVICE_ERR_SLOT_RANGE_BIT = 1;
 constexpr int GDN_DEVICE_ERR_TIMEOUT_BIT = 2;
+constexpr int GDN_DEVICE_ERR_SEQLEN_BIT = 4;
 
 // Longest conv supported (taps) and most tokens per launch.
 constexpr int kMaxConvWidth = 8;

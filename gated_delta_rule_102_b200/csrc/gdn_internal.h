@@ -32,6 +32,11 @@ struct DecodeArgs {
     float* out_f32;
     int32_t* err_flag;
     unsigned int* sched;  // nullable: two zeroed counters for the dynamic schedule of the persistent kernel
+    // nullable: [B+1] device offsets of each sequence's tokens in the packed inputs and
+    // outputs (sequence i has the rows cu_seqlens[i] .. cu_seqlens[i+1]-1, at most T of
+    // them); null: every sequence has T tokens, sequence i at rows i*T ..
+    const int32_t* cu_seqlens;
+    int32_t total_rows;  // with cu_seqlens: rows of the packed tensors (a sequence's rows must lie inside)
 };
 
 struct ConvArgs {

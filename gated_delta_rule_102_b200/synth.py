@@ -215,6 +215,37 @@ def step_inputs(wl: Workload, step: int, rows: Optional[Sequence[int]] = None) -
     }
 
 
+def varlen_counts(wl: Workload, step: int, t_max: int) -> np.ndarray:
+    """int32 [B]: token counts of a ragged launch, each in 0..t_max: sequence 0 gets
+    t_max, sequence 1 one token, sequence 2 none (when the batch has them), the rest
+    uniform draws."""
+    u = uniform(stream_key(wl.seed, "varlen", step), wl.batch)
+    n = np.minimum((u * (t_max + 1)).astype(np.int64), t_max)
+    for i, v in enumerate((t_max, 1, 0)[: wl.batch]):
+        n[i] = v
+    return n.astype(np.int32)
+
+
+def varlen_inputs(wl: Workload, step: int, counts: Sequence[int],
+                  rows: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
+    """Inputs of a ragged launch packed row after row (the sequences `rows`, default
+    all, in order; sequence i brings counts[i] tokens): qkv [total][C], a, b
+    [total][Hv], z [total][Hv][dv]. Sequence i's tokens are the first counts[i]
+    tokens of its own (step, sequence) streams, so a subset regenerates alone."""
+    C, Hv, dv = wl.channels, wl.num_v_heads, wl.head_v_dim
+    rows = list(_seq_rows(wl, rows))
+    parts = {k: [] for k in ("qkv", "a", "b", "z")}
+    for r in rows:
+        n = int(counts[r])
+        if n <= 0:
+            continue
+        x = step_inputs(wl.replace(tokens=n), step, rows=[r])
+        for k in parts:
+            parts[k].append(x[k][0])
+    shapes = {"qkv": (C,), "a": (Hv,), "b": (Hv,), "z": (Hv, dv)}
+    return {k: (np.concatenate(v) if v else np.zeros((0,) + shapes[k], dtype=np.uint16)) for k, v in parts.items()}
+
+
 def initial_state(wl: Workload, slot_ids: Optional[Sequence[int]] = None) -> np.ndarray:
     """fp32 [n][Hv][dk][dv]: initial delta-rule state of the given pool slots
     (default: every slot), N(0, state_std) per slot stream, or zeros."""

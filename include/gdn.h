@@ -66,6 +66,7 @@ typedef enum {
 /* Bits a kernel ORs into *err_flag. */
 #define GDN_DEVICE_ERR_SLOT_RANGE 1 /* a sequence's slot is outside [0, pool_slots) */
 #define GDN_DEVICE_ERR_TIMEOUT 2    /* a bounded wait inside the kernel ran out */
+#define GDN_DEVICE_ERR_SEQLEN 4     /* gdn_decode_step_varlen: a token count < 0 or > T_max */
 
 typedef struct {
     int32_t num_k_heads; /* Hk */
@@ -160,6 +161,37 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
 size_t gdn_decode_workspace_bytes(void);
 
 /*
+ * The fused decode step for a batch whose sequences bring different numbers of tokens
+ * (a chunk of a prompt for some, one token for others) in ONE kernel launch. The
+ * pages launch per sequence and have no such layout; each sequence's tokens are
+ * processed exactly as gdn_decode_step processes T tokens (steps 3 to 8 and the
+ * SiLU(z) gate of steps 9+10+11, the tokens in order, the state on chip in between).
+ * The tokens of all sequences are packed row after row:
+ *   cu_seqlens [B+1] int32 device, 4-byte aligned: sequence i owns the n_i =
+ *            cu_seqlens[i+1] - cu_seqlens[i] rows cu_seqlens[i] .. cu_seqlens[i+1]-1;
+ *            cu_seqlens[0] = 0 and cu_seqlens[B] = total_tokens are expected
+ *   T_max    the largest n_i, 1..16 (sizes the kernel's on-chip buffers)
+ *   total_tokens  rows of the packed tensors (>= 0; only checked on the host)
+ *   qkv [total][C], a [total][Hv], b [total][Hv], z [total][Hv][dv]   bf16 inputs
+ *   out_bf16 [total][Hv][dv] bf16, out_f32 [total][Hv][dv] fp32 nullable
+ *   the weights, pools, slots and err_flag as for gdn_decode_step.
+ * A sequence with n_i = 0 is left untouched. A sequence with n_i < 0, n_i > T_max or
+ * rows outside [0, total_tokens) is skipped (pools and outputs untouched) and
+ * GDN_DEVICE_ERR_SEQLEN is OR-ed into *err_flag; a slot outside [0, pool_slots) is
+ * handled as in gdn_decode_step. Rows that no sequence owns are neither read nor
+ * written. total_tokens = 0 returns GDN_OK without launching. Launched like
+ * gdn_decode_step (programmatic stream serialization, no allocation, no
+ * synchronization).
+ */
+gdn_status gdn_decode_step_varlen(const gdn_config* cfg, int32_t B, const int32_t* cu_seqlens,
+                                  int32_t T_max, int32_t total_tokens, const uint16_t* qkv,
+                                  const uint16_t* a, const uint16_t* b, const uint16_t* z,
+                                  const uint16_t* conv_w, const float* A_log, const float* dt_bias,
+                                  const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                                  int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
+                                  float* out_f32, int32_t* err_flag, void* stream);
+
+/*
  * gdn_decode_step for callers that cannot allocate device memory. The pages have
  * no counterpart of this entry point; it exists for the library's users.
  *
@@ -205,7 +237,7 @@ gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t po
 const char* gdn_status_string(gdn_status status);
 
 /* ABI version of this header: (major << 16) | minor. */
-#define GDN_ABI_VERSION ((1 << 16) | 0)
+#define GDN_ABI_VERSION ((1 << 16) | 1)
 int32_t gdn_abi_version(void);
 
 #ifdef __cplusplus

@@ -53,7 +53,7 @@ def test_status_codes_match_header(L):
         m = re.search(rf"\b{name} = (\d+)", HEADER)
         assert m and int(m.group(1)) == getattr(gdn, name)
         assert gdn.status_string(getattr(gdn, name))
-    for name in ("GDN_DEVICE_ERR_SLOT_RANGE", "GDN_DEVICE_ERR_TIMEOUT"):
+    for name in ("GDN_DEVICE_ERR_SLOT_RANGE", "GDN_DEVICE_ERR_TIMEOUT", "GDN_DEVICE_ERR_SEQLEN"):
         m = re.search(rf"#define {name} (\d+)", HEADER)
         assert int(m.group(1)) == getattr(gdn, name)
 
@@ -149,3 +149,36 @@ def test_binding_fails_loudly_without_cuda_tensors():
     x = torch.zeros(1, 1, cfg.channels, dtype=torch.bfloat16)
     with pytest.raises((ValueError, TypeError)):
         gdn.gdn_decode_step(cfg, x, x, x, x, x, x, x, x, x, x, x, x)
+
+
+def varlen(L, cfg, B=4, cu=FAKE, T_max=16, total=40, ptrs=None, pool=8, out_f32=None, err=None):
+    # qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool; then slots, out
+    p = [FAKE] * 10 if ptrs is None else ptrs
+    return L.gdn_decode_step_varlen(ctypes.byref(cfg), B, cu, T_max, total, *p, pool, FAKE, FAKE, out_f32, err,
+                                    None)
+
+
+def test_varlen_checks_its_arguments_on_the_host(L):
+    cfg = good_cfg()
+    assert varlen(L, good_cfg(head_k_dim=96)) == gdn.GDN_ERR_UNSUPPORTED
+    assert varlen(L, cfg, B=-1) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert varlen(L, cfg, T_max=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert varlen(L, cfg, T_max=17) == gdn.GDN_ERR_UNSUPPORTED
+    assert varlen(L, cfg, total=-1) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert varlen(L, cfg, cu=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert varlen(L, cfg, cu=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED        # int32 offsets: 4-byte aligned
+    assert varlen(L, cfg, pool=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    for i in range(10):
+        ptrs = [FAKE] * 10
+        ptrs[i] = None
+        assert varlen(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
+        ptrs[i] = FAKE_ODD
+        assert varlen(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
+    assert varlen(L, cfg, out_f32=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    assert varlen(L, cfg, err=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+
+
+def test_varlen_without_tokens_is_a_no_op(L):
+    # no sequence, or no token at all: returns before any pointer is looked at or any launch
+    assert varlen(L, good_cfg(), B=0, cu=None, ptrs=[None] * 10) == gdn.GDN_OK
+    assert varlen(L, good_cfg(), total=0, cu=None, ptrs=[None] * 10) == gdn.GDN_OK

@@ -61,11 +61,28 @@ def algorithmic_bytes(wl) -> int:
     return wl.batch * per_seq + per_launch
 
 
+def ragged_bytes_flops(wl, counts):
+    """Algorithmic bytes and FP32 flops of one ragged launch (token counts `counts`):
+    per sequence with tokens its state read+write, conv history read+write, the slot,
+    and per token qkv, a, b, z in and out; per launch the weights and the offsets."""
+    Hk, Hv, dk, dv, W, C = (wl.num_k_heads, wl.num_v_heads, wl.head_k_dim, wl.head_v_dim, wl.conv_width,
+                            wl.channels)
+    nbytes, ntok = 0, 0
+    for n in (int(v) for v in counts):
+        if n > 0:
+            nbytes += 2 * Hv * dk * dv * 4 + 2 * (W - 1) * C * 2 + 4 + n * (C * 2 + 2 * Hv * 2 + 2 * Hv * dv * 2)
+            ntok += n
+    nbytes += C * W * 2 + 2 * Hv * 4 + dv * 2 + (len(counts) + 1) * 4
+    return nbytes, 7 * ntok * Hv * dk * dv
+
+
 def kernel_for(wl, num_sms: int) -> str:
     """The kernel the launcher picks for the workload (the rule of launch_decode_fused):
     the persistent kernel for one token over at least two waves of co-resident clusters
     (one CTA per SM, G CTAs per cluster), else the cluster-per-group kernels."""
     G = wl.num_v_heads // wl.num_k_heads
+    if wl.ragged:
+        return "decode_mt_kernel"
     if wl.tokens == 1 and wl.batch * wl.num_k_heads >= 2 * (num_sms // G):
         return "decode_ws_kernel"
     return "decode_fused_tma_kernel" if wl.tokens == 1 else "decode_mt_kernel"
@@ -278,7 +295,9 @@ def l2_note(wl, pools: int) -> str:
 
 
 def workload_config(wl, args, world):
-    return {"workload": f"{wl.name}: B={wl.batch} sequences x T={wl.tokens} token, Hk={wl.num_k_heads}, "
+    tok = (f"0..{wl.tokens} tokens each (seeded uniform counts, packed rows)" if wl.ragged
+           else f"T={wl.tokens} token")
+    return {"workload": f"{wl.name}: B={wl.batch} sequences x {tok}, Hk={wl.num_k_heads}, "
                         f"Hv={wl.num_v_heads}, dk={wl.head_k_dim}, dv={wl.head_v_dim}, conv width {wl.conv_width}, "
                         f"{wl.pool_slots}-slot fp32 state pool per layer",
             "batch_per_gpu": wl.batch, "tokens_per_sequence": wl.tokens, "state_pools_cycled": args.pools,
@@ -329,14 +348,41 @@ def main():
               for p in range(args.pools)]
     convs = [bf16(synth.initial_conv_state(wlr)) for _ in range(args.pools)]
     n_inputs = args.pools * 4
-    xs = [{k: bf16(v) for k, v in synth.step_inputs(wlr, s).items()} for s in range(n_inputs)]
-    out = torch.empty(wl.batch, wl.tokens, wl.num_v_heads, wl.head_v_dim, dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     ws = gdn.decode_workspace(dev)  # dynamic spread of the sequences over the SMs
     stream = torch.cuda.current_stream(dev)
-    plans = [gdn.DecodePlan(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
-                            convs[i % args.pools], states[i % args.pools], slots, out, None, err, ws, stream)
-             for i, x in enumerate(xs)]
+    if wl.ragged:
+        # every input set gives each sequence its own token count, packed row after row
+        counts = [synth.varlen_counts(wlr, s, wl.tokens) for s in range(n_inputs)]
+        xs = [{k: bf16(v) for k, v in synth.varlen_inputs(wlr, s, counts[s]).items()} for s in range(n_inputs)]
+        cus = [torch.from_numpy(np.concatenate([[0], np.cumsum(c)]).astype(np.int32)).to(dev) for c in counts]
+        outs = [torch.empty(int(c.sum()), wl.num_v_heads, wl.head_v_dim, dtype=torch.bfloat16, device=dev)
+                for c in counts]
+        set_tokens = [int(c.sum()) for c in counts]
+        set_cost = [ragged_bytes_flops(wl, c) for c in counts]
+
+        def launch(i):
+            x = xs[i]
+            gdn.gdn_decode_step_varlen(cfg, cus[i], wl.tokens, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log,
+                                       dt_bias, norm_w, convs[i % args.pools], states[i % args.pools], slots,
+                                       outs[i], None, err)
+        eager_launch = launch
+    else:
+        xs = [{k: bf16(v) for k, v in synth.step_inputs(wlr, s).items()} for s in range(n_inputs)]
+        out = torch.empty(wl.batch, wl.tokens, wl.num_v_heads, wl.head_v_dim, dtype=torch.bfloat16, device=dev)
+        plans = [gdn.DecodePlan(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
+                                convs[i % args.pools], states[i % args.pools], slots, out, None, err, ws, stream)
+                 for i, x in enumerate(xs)]
+        set_tokens = [wl.batch * wl.tokens] * n_inputs
+        set_cost = [(algorithmic_bytes(wl), algorithmic_flops(wl))] * n_inputs
+
+        def launch(i):
+            x = xs[i]
+            gdn.gdn_decode_step(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
+                                convs[i % args.pools], states[i % args.pools], slots, out, None, err, ws)
+
+        def eager_launch(i):
+            plans[i].launch()
 
     def barrier():
         if world > 1:
@@ -344,7 +390,7 @@ def main():
 
     sampler = ClockSampler(local) if rank == 0 else None
     for i in range(args.warmup):
-        plans[i % n_inputs].launch()
+        eager_launch(i % n_inputs)
     torch.cuda.synchronize()
 
     # ---- timed region: exactly K steps, replayed from CUDA graphs (how a decode engine
@@ -360,9 +406,7 @@ def main():
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
             for i in range(count):
-                x = xs[i]
-                gdn.gdn_decode_step(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w,
-                                    convs[i % args.pools], states[i % args.pools], slots, out, None, err, ws)
+                launch(i)
         graphs.append(g)
     for _ in range(max(1, args.warmup // n_inputs)):
         graphs[0].replay()
@@ -387,7 +431,7 @@ def main():
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
     for i in range(Ke):
         ev_s[i].record(stream)
-        plans[i % n_inputs].launch()
+        eager_launch(i % n_inputs)
         ev_e[i].record(stream)
     torch.cuda.synchronize()
     kernel_ms_eager = max_over_ranks(statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(Ke)), dev, world)
@@ -404,7 +448,7 @@ def main():
     # and public-API calls) are captured once in a CUDA graph and replayed, as a decode
     # engine issues its steps. Every step's copies and launch lie inside the timed region.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not wl.ragged:
         names = ("qkv", "a", "b", "z")
         sizes = [xs[0][k].numel() for k in names]  # bf16 elements
         offs = [sum(sizes[:j]) for j in range(len(names))]
@@ -488,7 +532,9 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
-    nbytes = algorithmic_bytes(wl)
+    # the timed steps cycle the input sets: step j uses set j % n_inputs
+    step_sets = [j % n_inputs for j in range(K)]
+    nbytes = statistics.fmean(set_cost[i][0] for i in step_sets)  # per launch
     peak, peak_kind = hbm_peak()
     kernel_ms = elapsed_ms / K  # graph-replayed launches back to back: includes the gaps between them
     achieved = nbytes / (kernel_ms / 1e3) / 1e9
@@ -496,7 +542,7 @@ def main():
     kernel = kernel_for(wl, num_sms)
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "traffic": profiled_traffic(kernel, wl.name), "peak_source": f"{peak_kind} copy bandwidth"}
-    flops = algorithmic_flops(wl)
+    flops = statistics.fmean(set_cost[i][1] for i in step_sets)
     sm_mhz = (clocks or {}).get("sm_mhz")
     if sm_mhz and flops / (kernel_ms / 1e3) / 1e12 / (num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6) > roof["frac"]:
         # closer to the FP32 FMA peak (SMs x 128 lanes x 2 flops x the median SM clock
@@ -506,7 +552,7 @@ def main():
         roof = {"bound": "alu", "achieved": alu, "peak": alu_peak, "unit": "TFLOP/s", "frac": alu / alu_peak,
                 "traffic": roof["traffic"], "peak_source": "FP32 FMA lanes x measured SM clock",
                 "hbm_gbs_achieved": achieved, "hbm_frac": achieved / peak}
-    tokens = world * wl.batch * wl.tokens * K
+    tokens = world * sum(set_tokens[i] for i in step_sets)
     value = tokens / (elapsed_ms / 1e3)
     job_gbs = world * nbytes * K / (elapsed_ms / 1e3) / 1e9
     line = {
@@ -521,7 +567,7 @@ def main():
                          eager_kernel_us=kernel_ms_eager * 1e3),
         "e2e": e2e, "clocks": clocks, "gpu_launches": K,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not wl.ragged:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -106,6 +106,8 @@ class Workload:
     ``decay_half_to_one`` (a chosen so that exp(g) is spread over [0.5, 1)) or
     ``decay_wide`` (exp(g) = 2^-u with u ~ U(0, 48), and 2^-200 for about one entry
     in eight: decays far below 1, down to values that underflow in fp32).
+    ``ragged``: each launch gives every sequence its own token count, 0..``tokens``
+    (``varlen_counts``), packed row after row (``varlen_inputs``).
     """
 
     name: str
@@ -122,6 +124,7 @@ class Workload:
     slot_mode: str
     gate_mode: str
     seed: int
+    ragged: bool = False
 
     @property
     def channels(self) -> int:
@@ -147,6 +150,8 @@ WORKLOADS: Dict[str, Workload] = {
                  state_std=0.02, slot_mode="sample", gate_mode="decay_half_to_one", seed=1003),
         Workload("multitoken_b32_t16", **_QWEN3_NEXT_LIKE, batch=32, tokens=16, pool_slots=32, steps=16,
                  state_std=0.02, slot_mode="permutation", gate_mode="normal", seed=1004),
+        Workload("ragged_b64_t16", **_QWEN3_NEXT_LIKE, batch=64, tokens=16, pool_slots=64, steps=8,
+                 state_std=0.02, slot_mode="permutation", gate_mode="normal", seed=1005, ragged=True),
     )
 }
 

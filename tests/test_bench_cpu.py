@@ -27,6 +27,7 @@ def test_kernel_choice_per_workload():
     assert b.kernel_for(w["single_seq"], 148) == "decode_fused_tma_kernel"
     assert b.kernel_for(w["tiny_d16"], 148) == "decode_fused_tma_kernel"
     assert b.kernel_for(w["multitoken_b32_t16"], 148) == "decode_mt_kernel"
+    assert b.kernel_for(w["ragged_b64_t16"], 148) == "decode_mt_kernel"
 
 
 def test_algorithmic_bytes_and_flops_match_the_stated_counts():
@@ -37,6 +38,14 @@ def test_algorithmic_bytes_and_flops_match_the_stated_counts():
     assert b.algorithmic_bytes(w["pool384_batch256"]) == 256 * 4325508 + 66048
     # 7 flops per state element per token: 1.879 GFLOP per multi-token launch
     assert b.algorithmic_flops(w["multitoken_b32_t16"]) == 7 * 32 * 16 * 32 * 128 * 128 == 1879048192
+    # a ragged launch whose sequences all bring T tokens moves what the uniform one moves,
+    # plus its B+1 offsets; sequences without tokens move nothing
+    import numpy as np
+    wu = w["multitoken_b32_t16"]
+    nb, nf = b.ragged_bytes_flops(wu, np.full(32, 16))
+    assert nb == b.algorithmic_bytes(wu) + 33 * 4 and nf == b.algorithmic_flops(wu)
+    nb0, nf0 = b.ragged_bytes_flops(wu, np.r_[np.full(16, 16), np.zeros(16, int)])
+    assert nf0 == nf // 2 and nb0 == nb - 16 * (nb - b.ragged_bytes_flops(wu, np.zeros(32, int))[0]) // 32
 
 
 def test_profile_counts_only_for_the_code_it_was_taken_on(tmp_path, monkeypatch):

@@ -441,12 +441,13 @@ def main():
 
     # ---- end to end through the C ABI: pinned host inputs in, host output back, every step.
     # A step's four inputs sit in one pinned host buffer and travel in one copy. The steps
-    # are pipelined over three streams: step i's inputs travel host -> device on the
-    # copy-in stream while step i-1 computes, and each step's output travels back on the
-    # copy-out stream once its launch is done; device inputs and outputs are double
-    # buffered, events order each buffer's reuse. Blocks of n_inputs such steps (copies
-    # and public-API calls) are captured once in a CUDA graph and replayed, as a decode
-    # engine issues its steps. Every step's copies and launch lie inside the timed region.
+    # are pipelined: step i's inputs travel host -> device on copy-in stream i % 2 (two
+    # input copies can be in flight) while earlier steps compute, and each step's output
+    # travels back on the copy-out stream once its launch is done; device inputs and
+    # outputs are double buffered, events order each buffer's reuse. Blocks of n_inputs
+    # such steps (copies and public-API calls) are captured once in a CUDA graph and
+    # replayed on the timing stream, as a decode engine issues its steps. Every step's
+    # copies and launch lie inside the timed region.
     e2e = None
     if not args.no_e2e and not wl.ragged:
         names = ("qkv", "a", "b", "z")
@@ -466,16 +467,18 @@ def main():
         h2d = total * 2
         d2h = houts[0].numel() * houts[0].element_size()
         cstream = torch.cuda.Stream(dev)  # compute stream of the captured steps
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        s_ins, s_out = [torch.cuda.Stream(dev) for _ in range(2)], torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b are on the device
         ev_done = [torch.cuda.Event() for _ in range(2)]  # the launch reading buffer b has finished
         ev_out = [torch.cuda.Event() for _ in range(2)]   # output buffer b has reached the host
 
         def e2e_block():  # n_inputs pipelined steps, issued on cstream
-            s_in.wait_stream(cstream)
+            for s_in in s_ins:
+                s_in.wait_stream(cstream)
             s_out.wait_stream(cstream)
             for i in range(n_inputs):
                 b = i % 2
+                s_in = s_ins[b]
                 if i >= 2:
                     s_in.wait_event(ev_done[b])
                 with torch.cuda.stream(s_in):
@@ -493,7 +496,8 @@ def main():
                 with torch.cuda.stream(s_out):
                     houts[b].copy_(outs[b], non_blocking=True)
                 ev_out[b].record(s_out)
-            cstream.wait_stream(s_in)
+            for s_in in s_ins:
+                cstream.wait_stream(s_in)
             cstream.wait_stream(s_out)
 
         cstream.wait_stream(stream)
@@ -508,11 +512,13 @@ def main():
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
+        # replay() launches the graph on the current stream: the events go on that stream
+        replay_stream = torch.cuda.current_stream(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(cstream)
+        e0.record(replay_stream)
         for _ in range(reps):
             eg.replay()
-        e1.record(cstream)
+        e1.record(replay_stream)
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
@@ -520,8 +526,9 @@ def main():
         e2e = {"value": world * wl.batch * wl.tokens * reps * n_inputs / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "method": "gdn_decode_step (public C ABI) per step; each step's inputs copied in from pinned host memory "
-                         "and its output copied out, pipelined over copy-in, compute and copy-out streams "
-                         f"(double-buffered), {n_inputs}-step blocks captured in a CUDA graph and replayed"}
+                         "and its output copied out, pipelined over two copy-in streams, the compute stream and a "
+                         f"copy-out stream (double-buffered), {n_inputs}-step blocks captured in a CUDA graph and "
+                         "replayed; timed with events on the replay stream"}
 
     clocks = None
     if sampler is not None:
@@ -567,6 +574,9 @@ def main():
                          eager_kernel_us=kernel_ms_eager * 1e3),
         "e2e": e2e, "clocks": clocks, "gpu_launches": K,
     }
+    if e2e is not None and e2e["value"] > value * 1.02:
+        # the end-to-end steps launch the same kernels plus copies: they cannot be faster
+        raise RuntimeError(f"e2e {e2e['value']:.0f} tokens/s above the kernel-only {value:.0f}: timing error")
     if world == 1 and not args.no_cpu_baseline and not wl.ragged:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     print(json.dumps(line), flush=True)

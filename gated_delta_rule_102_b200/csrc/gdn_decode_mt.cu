@@ -101,6 +101,11 @@ struct MtGeo {
     // the stage's first packed row and token count
 };
 
+template <int K>
+struct Taps {  // a conv window of K taps, as a type
+    static constexpr int value = K;
+};
+
 // Row held by lane row group rg in register block j, element e.
 template <int RPL>
 __device__ __forceinline__ int mt_row(int j, int rg, int e) {
@@ -157,19 +162,20 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         const int nrow = W - 1 + ntok;
         const int ch_q = hk * DK, ch_k = Hk * DK + hk * DK, ch_v = 2 * Hk * DK + h0 * DV;
         auto run_channel = [&](int lc) { return lc < DK ? ch_q + lc : (lc < 2 * DK ? ch_k + lc - DK : ch_v + lc - 2 * DK); };
-        if (warp == 0) {  // the NH state tiles, contiguous in the pool
-            if (lane == 0) {
-                *stage_slot = slot;
-                *stage_tok0 = tok0;
-                *stage_ntok = ntok;
-                mbar_arrive_expect_tx(full, (uint32_t)(NH * Geo::TILE));
-            }
-            __syncwarp();
-            fence_proxy_async_smem();  // the stage's last reads (generic proxy) before the copies overwrite it
+        if (tid == 0) {
+            *stage_slot = slot;
+            *stage_tok0 = tok0;
+            *stage_ntok = ntok;
+            mbar_arrive_expect_tx(full, (uint32_t)(NH * Geo::TILE));
+        }
+        if (lane == 0) {  // the NH state tiles, contiguous in the pool: one bulk copy per warp (a
+                          // warp issuing many serialises them)
             const char* tiles = reinterpret_cast<const char*>(p.state_pool + ((size_t)slot * Hv + h0) * (size_t)(DK * DV));
             const int tile_bytes = NH * Geo::TILE;
-            for (int c = lane * kMtChunk; c < tile_bytes; c += 32 * kMtChunk)
+            for (int c = warp * kMtChunk; c < tile_bytes; c += Geo::NW * kMtChunk) {
+                fence_proxy_async_smem();  // the stage's last reads (generic proxy) before the copies overwrite it
                 tma_load_1d(smem + c, tiles + c, (uint32_t)min(kMtChunk, tile_bytes - c), full);
+            }
         }
         // the W-1 history rows, then the T token rows, of the pass's channels; then the
         // channels' weights ([channel][W], three runs of consecutive channels; a 16-byte
@@ -301,36 +307,43 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                     pr[2] = f2_pack(a.z, b.z); pr[3] = f2_pack(a.w, b.w);
                 }
         }
-        // ---- step 3: conv + SiLU of every channel for every token. The window of the
-        // last kMaxConvWidth staged rows slides through registers with the newest row
-        // at the top, the weights aligned to it (taps beyond W are zero), so every
-        // register index is a compile-time constant whatever W is.
-        for (int lc = tid; lc < NCH; lc += Geo::NT) {
-            float wr[kMaxConvWidth], win[kMaxConvWidth];
+        // ---- step 3: conv + SiLU of every channel for every token. A window of the last
+        // K staged rows slides through registers with the newest row at the top, the
+        // weights aligned to it (taps beyond W are zero), so every register index is a
+        // compile-time constant: K = 4 when W = 4, else the widest conv supported.
+        auto conv_channels = [&](auto taps) {
+            constexpr int K = decltype(taps)::value;
+            for (int lc = tid; lc < NCH; lc += Geo::NT) {
+                float wr[K], win[K];
 #pragma unroll
-            for (int m = 0; m < kMaxConvWidth; ++m) {
-                const int j = W - kMaxConvWidth + m;  // tap of window position m: it multiplies staged row t + j
-                wr[m] = j >= 0 ? bf16_bits_to_float(wts[lc * W + j]) : 0.f;
-                // before token 0's shift position m holds staged row j - 1 (history rows only)
-                win[m] = j >= 1 ? bf16_bits_to_float(rows[(j - 1) * NCH + lc]) : 0.f;
-            }
+                for (int m = 0; m < K; ++m) {
+                    const int j = W - K + m;  // tap of window position m: it multiplies staged row t + j
+                    wr[m] = j >= 0 ? bf16_bits_to_float(wts[lc * W + j]) : 0.f;
+                    // before token 0's shift position m holds staged row j - 1 (history rows only)
+                    win[m] = j >= 1 ? bf16_bits_to_float(rows[(j - 1) * NCH + lc]) : 0.f;
+                }
 #pragma unroll 4
-            for (int t = 0; t < ntok; ++t) {
+                for (int t = 0; t < ntok; ++t) {
 #pragma unroll
-                for (int m = 0; m < kMaxConvWidth - 1; ++m) win[m] = win[m + 1];
-                win[kMaxConvWidth - 1] = bf16_bits_to_float(rows[(t + W - 1) * NCH + lc]);
-                float u2 = 0.f;
+                    for (int m = 0; m < K - 1; ++m) win[m] = win[m + 1];
+                    win[K - 1] = bf16_bits_to_float(rows[(t + W - 1) * NCH + lc]);
+                    float u2 = 0.f;
 #pragma unroll
-                for (int m = 0; m < kMaxConvWidth; ++m) u2 = fmaf(wr[m], win[m], u2);
-                const float sv = silu_fast(u2);
-                if (lc < 2 * DK) {
-                    qk[t * 2 * DK + lc] = sv;
-                } else {
-                    const int v_h = (lc - 2 * DK) / DV, v_j = lc - 2 * DK - v_h * DV;
-                    vs[(v_h * T + t) * DV + v_j] = sv;
+                    for (int m = 0; m < K; ++m) u2 = fmaf(wr[m], win[m], u2);
+                    const float sv = silu_fast(u2);
+                    if (lc < 2 * DK) {
+                        qk[t * 2 * DK + lc] = sv;
+                    } else {
+                        const int v_h = (lc - 2 * DK) / DV, v_j = lc - 2 * DK - v_h * DV;
+                        vs[(v_h * T + t) * DV + v_j] = sv;
+                    }
                 }
             }
-        }
+        };
+        if (W == 4)
+            conv_channels(Taps<4>{});
+        else
+            conv_channels(Taps<kMaxConvWidth>{});
         // ---- the new conv history: the last W-1 raw inputs. The v channels of this
         // pass's heads always; the k-head's q/k channels by the group's last pass.
         {

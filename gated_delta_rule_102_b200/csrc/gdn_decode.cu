@@ -71,10 +71,11 @@ struct TmaSmem {
     static __host__ __device__ size_t total_bytes(int T, int NS) { return bar_bytes_offset(T, NS) + 8; }
 };
 
-// Same work decomposition as decode_fused_kernel, with the state tile staged into
-// shared memory by TMA bulk copies issued before the conv work. The copies are in
-// the async proxy, so the cluster barriers' release fences do not wait for them and
-// the tile occupies no registers; the update streams back to HBM from registers.
+// The cluster kernel (work decomposition at the top of this file). The state tile is
+// staged into shared memory before the conv work: by TMA bulk copies when the slice is
+// whole rows, else by 16-byte cp.async from every thread, completing on one mbarrier.
+// The copies run beside the conv and the cluster barriers, and the tile occupies no
+// registers; the update streams back to HBM from registers.
 template <int DK, int DVS>
 __global__ void __launch_bounds__(Tile<DK, DVS>::NT)
 decode_fused_tma_kernel(const DecodeArgs p) {

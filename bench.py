@@ -272,6 +272,17 @@ def rank_workload(wl, rank: int):
     return wl.replace(seed=wl.seed + 7919 * rank)
 
 
+def sum_over_ranks(v: float, device, world: int) -> float:
+    """The sum of a per-rank count over all ranks (every rank calls it, in the same order)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def max_over_ranks(v: float, device, world: int) -> float:
     """The largest value over all ranks (timings are reported as the slowest rank)."""
     if world == 1:
@@ -534,14 +545,17 @@ def main():
     if sampler is not None:
         sampler.stop()
         clocks = sampler.summary(t_wall0, t_wall1)
+    # tokens processed in the timed steps, over all ranks (each rank has its own sequences,
+    # and in a ragged workload its own token counts): step j used input set j % n_inputs
+    step_sets = [j % n_inputs for j in range(K)]
+    tokens = sum_over_ranks(float(sum(set_tokens[i] for i in step_sets)), dev, world)
+    job_bytes = sum_over_ranks(float(sum(set_cost[i][0] for i in step_sets)), dev, world)
 
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
-    # the timed steps cycle the input sets: step j uses set j % n_inputs
-    step_sets = [j % n_inputs for j in range(K)]
-    nbytes = statistics.fmean(set_cost[i][0] for i in step_sets)  # per launch
+    nbytes = statistics.fmean(set_cost[i][0] for i in step_sets)  # per launch (this rank's sets)
     peak, peak_kind = hbm_peak()
     kernel_ms = elapsed_ms / K  # graph-replayed launches back to back: includes the gaps between them
     achieved = nbytes / (kernel_ms / 1e3) / 1e9
@@ -559,9 +573,8 @@ def main():
         roof = {"bound": "alu", "achieved": alu, "peak": alu_peak, "unit": "TFLOP/s", "frac": alu / alu_peak,
                 "traffic": roof["traffic"], "peak_source": "FP32 FMA lanes x measured SM clock",
                 "hbm_gbs_achieved": achieved, "hbm_frac": achieved / peak}
-    tokens = world * sum(set_tokens[i] for i in step_sets)
     value = tokens / (elapsed_ms / 1e3)
-    job_gbs = world * nbytes * K / (elapsed_ms / 1e3) / 1e9
+    job_gbs = job_bytes / (elapsed_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

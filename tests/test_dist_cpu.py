@@ -34,7 +34,13 @@ def _worker(rank, world, port, q):
         seen = [None] * world
         dist.all_gather_object(seen, mine)
         slowest = bench.max_over_ranks(1.5 + rank, torch.device("cpu"), world)
-        q.put((rank, slowest, len(set(seen)) == world))
+        # ragged launches: each rank draws its own token counts; the job total is their sum
+        rag = bench.rank_workload(synth.WORKLOADS["ragged_b64_t16"], rank)
+        mine_tokens = float(synth.varlen_counts(rag, 0, rag.tokens).sum())
+        everyone = [None] * world
+        dist.all_gather_object(everyone, mine_tokens)
+        total = bench.sum_over_ranks(mine_tokens, torch.device("cpu"), world)
+        q.put((rank, slowest, len(set(seen)) == world, total == sum(everyone) and len(set(everyone)) == world))
     finally:
         dist.destroy_process_group()
 
@@ -52,6 +58,7 @@ def test_two_gloo_ranks_shard_sequences_and_report_the_slowest():
     res = sorted(q.get(timeout=10) for _ in range(2))
     assert [r[1] for r in res] == [2.5, 2.5]      # max over ranks on every rank
     assert all(r[2] for r in res)                 # each rank draws different sequences
+    assert all(r[3] for r in res)                 # token totals are summed over ranks
 
 
 def test_reference_arm_under_torchrun_prints_once():

@@ -555,7 +555,10 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
-    nbytes = statistics.fmean(set_cost[i][0] for i in step_sets)  # per launch (this rank's sets)
+    def whole(x):  # integral counts print as integers
+        return int(x) if float(x).is_integer() else x
+
+    nbytes = whole(statistics.fmean(set_cost[i][0] for i in step_sets))  # per launch (this rank's sets)
     peak, peak_kind = hbm_peak()
     kernel_ms = elapsed_ms / K  # graph-replayed launches back to back: includes the gaps between them
     achieved = nbytes / (kernel_ms / 1e3) / 1e9
@@ -563,7 +566,7 @@ def main():
     kernel = kernel_for(wl, num_sms)
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "traffic": profiled_traffic(kernel, wl.name), "peak_source": f"{peak_kind} copy bandwidth"}
-    flops = statistics.fmean(set_cost[i][1] for i in step_sets)
+    flops = whole(statistics.fmean(set_cost[i][1] for i in step_sets))
     sm_mhz = (clocks or {}).get("sm_mhz")
     if sm_mhz and flops / (kernel_ms / 1e3) / 1e12 / (num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6) > roof["frac"]:
         # closer to the FP32 FMA peak (SMs x 128 lanes x 2 flops x the median SM clock

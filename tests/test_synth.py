@@ -84,3 +84,24 @@ def test_wide_decay_gate_range():
     assert 0.3 < np.mean(log2a < -24.0) < 0.7                # many far below fp32 epsilon
     tiny = np.mean(log2a < -150.0)
     assert 0.05 < tiny < 0.25                                # the 2^-200 entries (fp32 underflow)
+
+
+def test_ragged_counts_and_packed_inputs():
+    wl = synth.WORKLOADS["ragged_b64_t16"].replace(num_k_heads=2, num_v_heads=4, head_k_dim=16, head_v_dim=16)
+    c = synth.varlen_counts(wl, 3, wl.tokens)
+    assert c.dtype == np.int32 and c.shape == (wl.batch,)
+    assert c.min() >= 0 and c.max() <= wl.tokens
+    assert c[0] == wl.tokens and c[1] == 1 and c[2] == 0          # the edge counts are always present
+    assert len(set(c[3:].tolist())) > 5                              # the rest spread over the range
+    x = synth.varlen_inputs(wl, 3, c)
+    total = int(c.sum())
+    assert x["qkv"].shape == (total, wl.channels) and x["z"].shape == (total, wl.num_v_heads, wl.head_v_dim)
+    assert x["a"].shape == x["b"].shape == (total, wl.num_v_heads)
+    cu = np.concatenate([[0], np.cumsum(c)])
+    for r in (0, 1, 2, 17, wl.batch - 1):                            # each sequence's rows regenerate alone
+        xr = synth.varlen_inputs(wl, 3, c, rows=[r])
+        for k in x:
+            assert np.array_equal(xr[k], x[k][cu[r]:cu[r + 1]])
+    # a sequence's tokens are the first counts[r] tokens of its own uniform-T stream
+    full = synth.step_inputs(wl.replace(tokens=int(c[0])), 3, rows=[0])
+    assert np.array_equal(full["qkv"][0], x["qkv"][:c[0]])

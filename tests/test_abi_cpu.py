@@ -182,3 +182,36 @@ def test_varlen_without_tokens_is_a_no_op(L):
     # no sequence, or no token at all: returns before any pointer is looked at or any launch
     assert varlen(L, good_cfg(), B=0, cu=None, ptrs=[None] * 10) == gdn.GDN_OK
     assert varlen(L, good_cfg(), total=0, cu=None, ptrs=[None] * 10) == gdn.GDN_OK
+
+
+def test_a_plain_c_program_builds_against_the_header_and_library(tmp_path, L):
+    """The boundary is plain C: a C99 program includes gdn.h, links libgdn.so and calls
+    the entry points that need no GPU (status strings, ABI version, host slot check, an
+    argument check that fails before any launch)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_gdn.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "gdn.h"
+int main(void) {
+    const int32_t slots[3] = {0, 2, 1};
+    gdn_config cfg = {16, 32, 128, 128, 4, 1e-6f, 1e-6f, 0.0f};
+    if (gdn_abi_version() != GDN_ABI_VERSION) return 1;
+    if (gdn_check_slots_host(slots, 3, 3) != GDN_OK) return 2;
+    if (gdn_decode_step(&cfg, 2, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 4, 0, 0, 0, 0, 0, 0) !=
+        GDN_ERR_INVALID_ARGUMENT) return 3;                    /* T = 0: rejected on the host */
+    printf("%s\n", gdn_status_string(GDN_ERR_MISALIGNED));
+    return 0;
+}
+''')
+    libdir = os.path.dirname(gdn.LIB_PATH)
+    exe = tmp_path / "use_gdn"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                    "-L", libdir, "-lgdn", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.strip() == gdn.status_string(gdn.GDN_ERR_MISALIGNED)

@@ -39,7 +39,7 @@ FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (4 partitions x 32)
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=("b200", "reference"), default="b200")
     ap.add_argument("--workload", default="batch64")
@@ -47,6 +47,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--timed-seconds", type=float, default=1.0,
+                    help="the K-step timed region is repeated back to back for about this long; "
+                         "the median region is reported")
+    ap.add_argument("--max-repeats", type=int, default=2000)
     return ap.parse_args()
 
 
@@ -112,15 +116,14 @@ def _code_only(text: str) -> bytes:
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the code `kernel` is built from (its own file, the shared headers and the
-    C-ABI header, comments left out): a profile taken on other code of this kernel no
-    longer describes it."""
+    """Hash of the code `kernel` is compiled from (its own file and the shared internal
+    headers, comments left out): a profile taken on other code of this kernel no longer
+    describes it. The public header is not part of any kernel's compilation."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_102_b200", "csrc")
     for f in sorted(KERNEL_SOURCES.get(kernel, ()) + SHARED_SOURCES):
         h.update(f.encode())
         h.update(_code_only(open(os.path.join(csrc, f)).read()))
-    h.update(_code_only(open(os.path.join(ROOT, "include", "gdn.h")).read()))
     return h.hexdigest()[:16]
 
 
@@ -190,6 +193,7 @@ class ClockSampler:
     def summary(self, t0: float, t1: float):
         win = [p for (t, p) in self.samples if t0 <= t <= t1]
         used = win if win else [p for (_, p) in self.samples]
+        source = "timed region" if win else "outside the timed region (no sample fell inside it)"
 
         def num(x):
             try:
@@ -200,31 +204,75 @@ class ClockSampler:
         mx = [num(p[1]) for p in used if num(p[1]) is not None]
         reasons = sorted({r for p in used for r, v in zip(self.REASONS, p[3:]) if v.strip().lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(win)}
+                "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(win),
+                "source": source}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def cpu_baseline(wl, budget_s: float):
-    """The FP64 oracle, single-threaded, on whole steps of the same batch until the
-    time budget is spent."""
+    """The FP64 oracle as it stands, on whole steps of the same batch until the time
+    budget is spent: once on one thread, once on all host cores. The all-cores run
+    splits the batch's sequences (independent of one another) over threads, each
+    calling the oracle on its own sequences and its own copy of their pools; the
+    oracle's C calls release the interpreter lock, so the threads run in parallel.
+    Input generation is not timed."""
     import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
     import oracle
     from gated_delta_rule_102_b200 import synth
     sh = oracle.Shape.of(wl)
     w = synth.weights(wl)
-    st = synth.initial_state(wl).astype(np.float64)
-    cv = synth.initial_conv_state(wl)
     slots = synth.slots(wl)
-    steps, elapsed = 0, 0.0
-    while elapsed < budget_s:
-        x = synth.step_inputs(wl, steps)  # input generation is not timed
-        t = time.perf_counter()
-        oracle.decode_step(sh, x["qkv"], x["a"], x["b"], x["z"], w["conv_w"], w["A_log"], w["dt_bias"], w["norm_w"],
-                           cv, st, slots)
-        elapsed += time.perf_counter() - t
-        steps += 1
-    return {"value": wl.batch * wl.tokens * steps / elapsed, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{steps} full steps of {wl.name} ({wl.batch} sequences x {wl.tokens} token), "
-                      f"single-threaded FP64 C oracle, {elapsed:.1f} s"}
+
+    def run(nthreads: int):
+        shards = [list(range(i, wl.batch, nthreads)) for i in range(nthreads)]
+        shards = [s for s in shards if s]
+        state = [synth.initial_state(wl, [int(slots[r]) for r in s]).astype(np.float64) for s in shards]
+        conv = [synth.initial_conv_state(wl, [int(slots[r]) for r in s]) for s in shards]
+        local = [np.arange(len(s), dtype=np.int32) for s in shards]
+
+        def one(j, x):
+            rows = shards[j]
+            oracle.decode_step(sh, x["qkv"][rows], x["a"][rows], x["b"][rows], x["z"][rows], w["conv_w"],
+                               w["A_log"], w["dt_bias"], w["norm_w"], conv[j], state[j], local[j])
+
+        steps, elapsed = 0, 0.0
+        with ThreadPoolExecutor(max_workers=len(shards)) as ex:
+            while elapsed < budget_s:
+                x = synth.step_inputs(wl, steps)
+                xs = {k: np.ascontiguousarray(v) for k, v in x.items()}
+                t = time.perf_counter()
+                list(ex.map(lambda j: one(j, xs), range(len(shards))))
+                elapsed += time.perf_counter() - t
+                steps += 1
+        return wl.batch * wl.tokens * steps / elapsed, steps, elapsed, len(shards)
+
+    single, s1, e1, _ = run(1)
+    cores = host_cores()
+    multi, sm, em, used = run(min(cores, wl.batch))
+    return {"value": multi, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{sm} full steps of {wl.name} ({wl.batch} sequences x {wl.tokens} token) in {em:.1f} s, "
+                      f"the FP64 C oracle on {used} threads (sequences split over the threads); "
+                      f"single-threaded: {s1} steps in {e1:.1f} s",
+            "single_thread_value": single, "host_cores": cores, "cpu_model": cpu_model()}
 
 
 def run_reference(args, wl, rank: int, world: int):
@@ -422,20 +470,40 @@ def main():
     for _ in range(max(1, args.warmup // n_inputs)):
         graphs[0].replay()
     torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    def k_steps():  # exactly K steps
+        for _ in range(K // n_inputs):
+            graphs[0].replay()
+        if graphs[1] is not None:
+            graphs[1].replay()
+
+    # one K-step region to size the repeats: the K-step region is timed R times back to
+    # back (about a second in all, so the clock samples fall inside it and one slow
+    # region does not decide the number); the median region is reported
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    k_steps()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
+    R = int(min(args.max_repeats, max(3, round(args.timed_seconds * 1e3 / max(one_ms, 1e-3)))))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(R)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(R)]
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    start.record(stream)
-    for _ in range(K // n_inputs):
-        graphs[0].replay()
-    if graphs[1] is not None:
-        graphs[1].replay()
-    end.record(stream)
+    for r in range(R):
+        starts[r].record(stream)
+        k_steps()
+        ends[r].record(stream)
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
-    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev, world)
+    rep_ms = [starts[r].elapsed_time(ends[r]) for r in range(R)]
+    if world > 1:  # each repeat's time is the slowest rank's
+        t = torch.tensor(rep_ms, device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        rep_ms = t.tolist()
+    elapsed_ms = statistics.median(rep_ms)
     # per-launch kernel time from events around eager launches of the same plans
     Ke = min(K, 2000)
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
@@ -581,6 +649,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "timing": {"repeats": R, "reported": "median of the repeated K-step regions",
+                   "ms_per_step_min": min(rep_ms) / K, "ms_per_step_max": max(rep_ms) / K},
         "dtype": "f32", "data": "synthetic (seeded SplitMix64 draws; bf16 inputs, fp32 state)",
         "config": workload_config(wl, args, world),
         "hbm_gbs": job_gbs / world, "frac_of_8tbs": job_gbs / world / NOMINAL_HBM_GBS,

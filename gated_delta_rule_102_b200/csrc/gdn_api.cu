@@ -66,6 +66,28 @@ gdn_status check_pointers(std::initializer_list<const void*> required, std::init
     return GDN_OK;
 }
 
+// Every check of gdn_decode_step, and its kernel arguments: nothing is enqueued here.
+// B == 0 returns GDN_OK with `d` unset (the call is a no-op).
+gdn_status check_decode(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv, const uint16_t* a,
+                        const uint16_t* b, const uint16_t* z, const uint16_t* conv_w, const float* A_log,
+                        const float* dt_bias, const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                        int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16, float* out_f32,
+                        int32_t* err_flag, void* workspace, gdn::DecodeArgs* d) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((st = check_pointers({qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots, out_bf16},
+                             {out_f32, err_flag, workspace})) != GDN_OK)
+        return st;
+    const int G = sh.Hv / sh.Hk;
+    *d = gdn::DecodeArgs{sh, B, T, pool_slots, gdn::decode_column_splits(B, sh.Hv, G, sh.dv),
+                         qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots,
+                         out_bf16, out_f32, err_flag, static_cast<unsigned int*>(workspace)};
+    return GDN_OK;
+}
+
 gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
 }  // namespace
@@ -118,18 +140,10 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
                            const float* dt_bias, const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
                            int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16, float* out_f32,
                            int32_t* err_flag, void* workspace, void* stream) {
-    gdn::Shape sh;
-    gdn_status st = check_config(cfg, &sh);
-    if (st != GDN_OK) return st;
-    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
-    if (B == 0) return GDN_OK;
-    if ((st = check_pointers({qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots, out_bf16},
-                             {out_f32, err_flag, workspace})) != GDN_OK)
-        return st;
-    const int G = sh.Hv / sh.Hk;
-    gdn::DecodeArgs d{sh, B, T, pool_slots, gdn::decode_column_splits(B, sh.Hv, G, sh.dv),
-                      qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots,
-                      out_bf16, out_f32, err_flag, static_cast<unsigned int*>(workspace)};
+    gdn::DecodeArgs d;
+    gdn_status st = check_decode(cfg, B, T, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
+                                 pool_slots, slots, out_bf16, out_f32, err_flag, workspace, &d);
+    if (st != GDN_OK || B == 0) return st;
     return from_cuda(gdn::launch_decode_fused(d, (cudaStream_t)stream));
 }
 
@@ -170,7 +184,7 @@ namespace {
 constexpr size_t kStaticScratchBytes = 256;  // fixed maximum
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-constexpr int kMaxScratchDevices = 64;
+constexpr int kMaxScratchDevices = gdn::kMaxDevices;
 std::mutex g_scratch_mutex;
 void* g_scratch_addr[kMaxScratchDevices];  // device address of g_decode_scratch, per device
 
@@ -201,17 +215,17 @@ gdn_status gdn_decode_step_static_scratch(const gdn_config* cfg, int32_t B, int3
                                           float* out_f32, int32_t* err_flag, void* stream) {
     const size_t need = gdn_decode_workspace_bytes();
     if (need > kStaticScratchBytes) return GDN_ERR_UNSUPPORTED;  // the fixed array is too small for this build
-    gdn::Shape sh;
-    gdn_status st = check_config(cfg, &sh);
-    if (st != GDN_OK) return st;
-    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
-    if (B == 0) return GDN_OK;
+    // every argument check first: an error return must leave the stream untouched
+    gdn::DecodeArgs d;
+    gdn_status st = check_decode(cfg, B, T, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
+                                 pool_slots, slots, out_bf16, out_f32, err_flag, nullptr, &d);
+    if (st != GDN_OK || B == 0) return st;
     void* scratch = nullptr;
     if ((st = static_scratch_address(&scratch)) != GDN_OK) return st;
+    d.sched = static_cast<unsigned int*>(scratch);
     // the counters must start at zero; clear them in stream order before the launch
     if (cudaMemsetAsync(scratch, 0, need, (cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
-    return gdn_decode_step(cfg, B, T, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
-                           pool_slots, slots, out_bf16, out_f32, err_flag, scratch, stream);
+    return from_cuda(gdn::launch_decode_fused(d, (cudaStream_t)stream));
 }
 
 size_t gdn_decode_static_scratch_bytes(void) { return kStaticScratchBytes; }

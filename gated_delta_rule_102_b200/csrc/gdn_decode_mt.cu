@@ -35,6 +35,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
 
@@ -546,20 +549,52 @@ int heads_per_pass(int G) {
     return nh;
 }
 
+// Per device and dynamic shared-memory size: the kernel attribute set, the SM count and
+// the co-resident CTAs per SM, found once (eager callers pay no device queries per call).
+struct MtLaunchInfo {
+    int dev, smem, sms, per_sm;
+};
+
+template <int DK, int DV>
+cudaError_t mt_launch_info(int smem, int* grid_cap) {
+    static std::mutex mu;
+    static std::vector<MtLaunchInfo> known;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const MtLaunchInfo& k : known)
+        if (k.dev == dev && k.smem == smem) {
+            *grid_cap = k.sms * k.per_sm;
+            return cudaSuccess;
+        }
+    auto kern = decode_mt_kernel<DK, DV>;
+    // the attribute is the largest size any launch on this device asks for
+    int largest = smem;
+    for (const MtLaunchInfo& k : known)
+        if (k.dev == dev && k.smem > largest) largest = k.smem;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, largest)) != cudaSuccess)
+        return e;
+    int sms = 0, per_sm = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, MtGeo<DK, DV>::NT, smem)) != cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    known.push_back({dev, smem, sms, per_sm});
+    *grid_cap = sms * per_sm;
+    return cudaSuccess;
+}
+
 template <int DK, int DV>
 cudaError_t launch_mt(const DecodeArgs& a, cudaStream_t stream) {
     using Geo = MtGeo<DK, DV>;
     auto kern = decode_mt_kernel<DK, DV>;
     const int smem = Geo::total(a.sh.W, a.T);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int cap = 0;
+    cudaError_t e = mt_launch_info<DK, DV>(smem, &cap);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Geo::NT, smem)) != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int ngroups = a.B * a.sh.Hk;
-    const int grid = ngroups < sms * per_sm ? ngroups : sms * per_sm;
+    const int grid = ngroups < cap ? ngroups : cap;
     if (grid <= 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);

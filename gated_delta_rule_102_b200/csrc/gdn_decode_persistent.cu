@@ -37,6 +37,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
 
@@ -591,10 +593,13 @@ template <int DK, int DV>
 cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool query_only, int* cap_out) {
     using L = WS<DK, DV>;
     auto kern = decode_ws_kernel<DK, DV>;
-    static int cap_cache[16][9];  // co-resident clusters per (device, cluster size), queried once
+    // co-resident clusters per (device, cluster size), queried once; threads may race to
+    // fill an entry, and all of them store the same value
+    static std::atomic<int> cap_cache[kMaxDevices][9];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(L::NT);
     cfg.dynamicSmemBytes = L::TOTAL;
@@ -608,7 +613,7 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;  // the occupancy query takes the cluster shape only
-    int& cap = cap_cache[dev & 15][G];
+    int cap = cap_cache[dev][G].load(std::memory_order_relaxed);
     if (cap <= 0) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
         if (e != cudaSuccess) return e;
@@ -617,6 +622,7 @@ cudaError_t launch_ws_tile(const DecodeArgs& a, int G, cudaStream_t stream, bool
         e = cudaOccupancyMaxActiveClusters(&maxc, kern, &cfg);
         if (e != cudaSuccess) return e;
         cap = maxc;
+        cap_cache[dev][G].store(maxc, std::memory_order_relaxed);
     }
     if (cap_out) *cap_out = cap;
     if (query_only) return cudaSuccess;

@@ -7,6 +7,9 @@
 
 namespace gdn {
 
+// Devices a process may use with this library (per-device host caches are this large).
+constexpr int kMaxDevices = 64;
+
 struct Shape {
     int Hk, Hv, dk, dv, W;  // heads, head dims, conv width
     int C;                  // 2*Hk*dk + Hv*dv

@@ -121,6 +121,32 @@ def test_decode_rejects_bad_sizes_and_pointers(L):
     assert gdn.decode_workspace_bytes() % 16 == 0 and gdn.decode_workspace_bytes() >= 8
 
 
+def static_scratch(L, cfg, B=4, T=1, ptrs=None, pool=8, out_f32=None, err=None):
+    p = [FAKE] * 10 if ptrs is None else ptrs
+    return L.gdn_decode_step_static_scratch(ctypes.byref(cfg) if cfg is not None else None, B, T, *p, pool, FAKE,
+                                            FAKE, out_f32, err, None)
+
+
+def test_static_scratch_checks_every_argument_before_touching_the_device(L):
+    # Without a GPU any CUDA call fails, so a status other than GDN_ERR_CUDA shows that
+    # the check ran before the scratch lookup and the memset were enqueued.
+    cfg = good_cfg()
+    assert static_scratch(L, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert static_scratch(L, good_cfg(head_k_dim=96)) == gdn.GDN_ERR_UNSUPPORTED
+    assert static_scratch(L, cfg, T=17) == gdn.GDN_ERR_UNSUPPORTED
+    assert static_scratch(L, cfg, B=-1) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert static_scratch(L, cfg, B=0, ptrs=[None] * 10) == gdn.GDN_OK
+    for i in range(10):
+        ptrs = [FAKE] * 10
+        ptrs[i] = None
+        assert static_scratch(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
+        ptrs[i] = FAKE_ODD
+        assert static_scratch(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
+    assert static_scratch(L, cfg, out_f32=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    assert static_scratch(L, cfg, err=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    assert gdn.decode_static_scratch_bytes() >= gdn.decode_workspace_bytes()
+
+
 def test_empty_batch_is_a_no_op(L):
     # B = 0 returns before any pointer is looked at or any launch is made
     assert decode(L, good_cfg(), B=0, ptrs=[None] * 10) == gdn.GDN_OK

@@ -6,13 +6,12 @@ place of the caller's workspace, and must give what gdn_decode_step gives.
 
 This file is collected last, so a run that stops at the first failure has already
 run every other test; it also passes on its own in a fresh process."""
-import numpy as np
 import pytest
 import torch
 
 import gated_delta_rule_102_b200 as gdn
 from gated_delta_rule_102_b200 import synth
-from gdn_harness import OUT_ABS_TOL, STATE_REL_TOL, DeviceRun, bf16_host
+from gdn_harness import DeviceRun
 
 pytestmark = pytest.mark.gpu
 
@@ -34,12 +33,9 @@ def test_static_scratch_matches_the_workspace_entry_point_on_two_calls_in_a_row(
                                            nal.err)
         torch.cuda.synchronize()
         assert int(nal.err.item()) == 0 and int(ref.err.item()) == 0
-        assert (out_n32 - out_r32).abs().max().item() <= OUT_ABS_TOL
-        gb_n = synth.bf16_bits_to_f32(bf16_host(out_n)).astype(np.float64)
-        gb_r = synth.bf16_bits_to_f32(bf16_host(out_r)).astype(np.float64)
-        assert np.abs(gb_n - gb_r).max() <= OUT_ABS_TOL + 2.0 ** -7 * max(1.0, np.abs(gb_r).max())
-        # the states agree per (slot, head) within the state tolerance; the conv history bit for bit
-        d = (nal.state - ref.state).abs().amax(dim=(2, 3))
-        scale = ref.state.abs().amax(dim=(2, 3)).clamp_min(1e-30)
-        assert (d / scale).max().item() <= STATE_REL_TOL
+        # Both calls run the same dynamically scheduled kernel, and every (sequence, head)
+        # is computed by one cluster in a fixed order, so the results are the same bits.
+        assert torch.equal(out_n32, out_r32)
+        assert torch.equal(out_n, out_r)
+        assert torch.equal(nal.state, ref.state)
         assert torch.equal(nal.conv, ref.conv)

@@ -28,7 +28,8 @@ GDN_DEVICE_ERR_TIMEOUT = 2
 GDN_DEVICE_ERR_SEQLEN = 4
 
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
-           "gdn_decode_workspace_bytes", "gdn_decode_step_varlen", "gdn_decode_step_static_scratch", "gdn_decode_static_scratch_bytes",
+           "gdn_decode_workspace_bytes", "gdn_decode_step_varlen", "gdn_decode_step_static_scratch",
+           "gdn_decode_static_scratch_bytes", "gdn_spec_verify", "gdn_spec_commit", "gdn_in_proj", "gdn_out_proj",
            "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
 
 
@@ -78,12 +79,18 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_step_static_scratch.restype = ctypes.c_int32
         L.gdn_decode_static_scratch_bytes.argtypes = []
         L.gdn_decode_static_scratch_bytes.restype = ctypes.c_size_t
+        L.gdn_spec_verify.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32] + [vp] * 8
+        L.gdn_spec_commit.argtypes = [cfgp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_in_proj.argtypes = [cfgp, i32, i32] + [vp] * 9
+        L.gdn_out_proj.argtypes = [cfgp, i32, i32] + [vp] * 6
         L.gdn_check_slots_host.argtypes = [vp, i32, i32]
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_abi_version.argtypes = []
         for f in ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
-                  "gdn_decode_step_varlen", "gdn_check_slots_host", "gdn_abi_version"):
+                  "gdn_decode_step_varlen", "gdn_spec_verify", "gdn_spec_commit", "gdn_in_proj", "gdn_out_proj",
+                  "gdn_check_slots_host",
+                  "gdn_abi_version"):
             getattr(L, f).restype = ctypes.c_int32
         _lib = L
     return _lib
@@ -195,6 +202,51 @@ def gdn_decode_step_static_scratch(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, 
         _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0], _ptr(slots, _I32, "slots"),
         _ptr(out, _BF16, "out"), _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
         _stream(stream, qkv)), "gdn_decode_step_static_scratch")
+
+
+def gdn_spec_verify(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool, slots,
+                    out, spec_k, spec_delta, spec_alpha, out_f32=None, err_flag=None, stream=None) -> None:
+    """Verify T drafted tokens (qkv [B][T][C], ...): the outputs of a T-token decode step,
+    the pools untouched, and per token the normalised key spec_k [B][T][Hk][dk], the
+    write spec_delta [B][T][Hv][dv] and the decay spec_alpha [B][T][Hv] (fp32)."""
+    B, T = qkv.shape[0], qkv.shape[1]
+    _check(lib().gdn_spec_verify(
+        ctypes.byref(cfg), B, T, _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"), _ptr(b, _BF16, "b"),
+        _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"), _ptr(A_log, _F32, "A_log"),
+        _ptr(dt_bias, _F32, "dt_bias"), _ptr(norm_w, _BF16, "norm_w"), _ptr(conv_pool, _BF16, "conv_pool"),
+        _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0], _ptr(slots, _I32, "slots"),
+        _ptr(out, _BF16, "out"), _ptr(out_f32, _F32, "out_f32"), _ptr(spec_k, _F32, "spec_k"),
+        _ptr(spec_delta, _F32, "spec_delta"), _ptr(spec_alpha, _F32, "spec_alpha"),
+        _ptr(err_flag, _I32, "err_flag"), _stream(stream, qkv)), "gdn_spec_verify")
+
+
+def gdn_spec_commit(cfg: GdnConfig, n_accept, qkv, conv_pool, state_pool, slots, spec_k, spec_delta, spec_alpha,
+                    err_flag=None, stream=None) -> None:
+    """Keep the first n_accept[b] verified tokens of every sequence b (device int32 [B])."""
+    B, T = qkv.shape[0], qkv.shape[1]
+    _check(lib().gdn_spec_commit(
+        ctypes.byref(cfg), B, T, _ptr(n_accept, _I32, "n_accept"), _ptr(qkv, _BF16, "qkv"),
+        _ptr(conv_pool, _BF16, "conv_pool"), _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0],
+        _ptr(slots, _I32, "slots"), _ptr(spec_k, _F32, "spec_k"), _ptr(spec_delta, _F32, "spec_delta"),
+        _ptr(spec_alpha, _F32, "spec_alpha"), _ptr(err_flag, _I32, "err_flag"), _stream(stream, qkv)),
+        "gdn_spec_commit")
+
+
+def gdn_in_proj(cfg: GdnConfig, x, w_in, qkv, z, a, b, out_f32=None, err_flag=None, stream=None) -> None:
+    """[qkv | z | a | b] = x @ w_in^T: x [rows][hidden], w_in [C + Hv*dv + 2*Hv][hidden] (bf16)."""
+    rows, hidden = x.shape[0], x.shape[-1]
+    _check(lib().gdn_in_proj(ctypes.byref(cfg), hidden, rows, _ptr(x, _BF16, "x"), _ptr(w_in, _BF16, "w_in"),
+                             _ptr(qkv, _BF16, "qkv"), _ptr(z, _BF16, "z"), _ptr(a, _BF16, "a"), _ptr(b, _BF16, "b"),
+                             _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"), _stream(stream, x)),
+           "gdn_in_proj")
+
+
+def gdn_out_proj(cfg: GdnConfig, y, w_out, out, out_f32=None, err_flag=None, stream=None) -> None:
+    """out = y @ w_out^T: y [rows][Hv*dv], w_out [hidden][Hv*dv] (bf16), out [rows][hidden]."""
+    rows, hidden = y.shape[0], w_out.shape[0]
+    _check(lib().gdn_out_proj(ctypes.byref(cfg), hidden, rows, _ptr(y, _BF16, "y"), _ptr(w_out, _BF16, "w_out"),
+                              _ptr(out, _BF16, "out"), _ptr(out_f32, _F32, "out_f32"),
+                              _ptr(err_flag, _I32, "err_flag"), _stream(stream, y)), "gdn_out_proj")
 
 
 def decode_static_scratch_bytes() -> int:

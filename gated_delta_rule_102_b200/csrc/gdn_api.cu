@@ -7,6 +7,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -90,6 +91,37 @@ gdn_status check_decode(const gdn_config* cfg, int32_t B, int32_t T, const uint1
 
 gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
+// hidden: a multiple of 8 (16-byte rows for the tile copies); rows: 0..256 token rows.
+gdn_status check_proj_sizes(int32_t hidden, int32_t rows) {
+    if (hidden <= 0 || rows < 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (hidden % 8 != 0 || hidden > (1 << 20) || rows > gdn::kProjMaxRows) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+// The SM count of the current device, queried once per device.
+gdn_status sm_count(int* out) {
+    static std::atomic<int> cache[gdn::kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    if (dev < 0 || dev >= gdn::kMaxDevices) return GDN_ERR_UNSUPPORTED;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return GDN_ERR_CUDA;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    *out = n;
+    return GDN_OK;
+}
+
+gdn_status launch_proj(gdn::ProjArgs& p, cudaStream_t stream) {
+    int sms = 0;
+    gdn_status st = sm_count(&sms);
+    if (st != GDN_OK) return st;
+    p.slices = gdn::proj_slices(p.N, p.K, sms);
+    return from_cuda(gdn::launch_proj_gemm(p, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -171,6 +203,96 @@ gdn_status gdn_decode_step_varlen(const gdn_config* cfg, int32_t B, const int32_
                       state_pool, slots, out_bf16, out_f32, err_flag, nullptr, cu_seqlens, total_tokens};
     if (!gdn::multitoken_supported(d)) return GDN_ERR_UNSUPPORTED;
     return from_cuda(gdn::launch_decode_multitoken(d, (cudaStream_t)stream));
+}
+
+gdn_status gdn_spec_verify(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv, const uint16_t* a,
+                           const uint16_t* b, const uint16_t* z, const uint16_t* conv_w, const float* A_log,
+                           const float* dt_bias, const uint16_t* norm_w, const uint16_t* conv_pool,
+                           const float* state_pool, int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
+                           float* out_f32, float* spec_k, float* spec_delta, float* spec_alpha, int32_t* err_flag,
+                           void* stream) {
+    gdn::DecodeArgs d;
+    // the pools are only read in verify mode
+    gdn_status st = check_decode(cfg, B, T, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w,
+                                 const_cast<uint16_t*>(conv_pool), const_cast<float*>(state_pool), pool_slots, slots,
+                                 out_bf16, out_f32, err_flag, nullptr, &d);
+    if (st != GDN_OK || B == 0) return st;
+    if ((st = check_pointers({spec_k, spec_delta, spec_alpha}, {})) != GDN_OK) return st;
+    d.T = T;
+    d.spec_k = spec_k;
+    d.spec_delta = spec_delta;
+    d.spec_alpha = spec_alpha;
+    if (!gdn::multitoken_supported(d)) return GDN_ERR_UNSUPPORTED;
+    return from_cuda(gdn::launch_decode_multitoken(d, (cudaStream_t)stream));
+}
+
+gdn_status gdn_spec_commit(const gdn_config* cfg, int32_t B, int32_t T, const int32_t* n_accept,
+                           const uint16_t* qkv, uint16_t* conv_pool, float* state_pool, int32_t pool_slots,
+                           const int32_t* slots, const float* spec_k, const float* spec_delta,
+                           const float* spec_alpha, int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_batch(B, T, pool_slots, sh)) != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((st = check_pointers({n_accept, qkv, conv_pool, state_pool, slots, spec_k, spec_delta, spec_alpha},
+                             {err_flag})) != GDN_OK)
+        return st;
+    gdn::SpecCommitArgs c{sh, B, T, pool_slots, n_accept, qkv, conv_pool, state_pool, slots,
+                          spec_k, spec_delta, spec_alpha, err_flag};
+    return from_cuda(gdn::launch_spec_commit(c, (cudaStream_t)stream));
+}
+
+gdn_status gdn_in_proj(const gdn_config* cfg, int32_t hidden, int32_t rows, const uint16_t* x,
+                       const uint16_t* w_in, uint16_t* qkv, uint16_t* z, uint16_t* a, uint16_t* b, float* out_f32,
+                       int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_proj_sizes(hidden, rows)) != GDN_OK) return st;
+    if (rows == 0) return GDN_OK;
+    if ((st = check_pointers({x, w_in, qkv, z, a, b}, {out_f32, err_flag})) != GDN_OK) return st;
+    const int Z = sh.Hv * sh.dv;
+    gdn::ProjArgs p{};
+    p.N = sh.C + Z + 2 * sh.Hv;
+    p.K = hidden;
+    p.R = rows;
+    p.x = x;
+    p.w = w_in;
+    p.nseg = 4;
+    const int starts[4] = {0, sh.C, sh.C + Z, sh.C + Z + sh.Hv}, widths[4] = {sh.C, Z, sh.Hv, sh.Hv};
+    uint16_t* outs[4] = {qkv, z, a, b};
+    for (int i = 0; i < 4; ++i) {
+        p.seg_start[i] = starts[i];
+        p.seg_width[i] = widths[i];
+        p.seg_out[i] = outs[i];
+    }
+    p.out_f32 = out_f32;
+    p.err_flag = err_flag;
+    return launch_proj(p, (cudaStream_t)stream);
+}
+
+gdn_status gdn_out_proj(const gdn_config* cfg, int32_t hidden, int32_t rows, const uint16_t* y,
+                        const uint16_t* w_out, uint16_t* out, float* out_f32, int32_t* err_flag, void* stream) {
+    gdn::Shape sh;
+    gdn_status st = check_config(cfg, &sh);
+    if (st != GDN_OK) return st;
+    if ((st = check_proj_sizes(hidden, rows)) != GDN_OK) return st;
+    if (rows == 0) return GDN_OK;
+    if ((st = check_pointers({y, w_out, out}, {out_f32, err_flag})) != GDN_OK) return st;
+    gdn::ProjArgs p{};
+    p.N = hidden;
+    p.K = sh.Hv * sh.dv;
+    p.R = rows;
+    p.x = y;
+    p.w = w_out;
+    p.nseg = 1;
+    p.seg_start[0] = 0;
+    p.seg_width[0] = hidden;
+    p.seg_out[0] = out;
+    p.out_f32 = out_f32;
+    p.err_flag = err_flag;
+    return launch_proj(p, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -40,6 +40,27 @@ struct DecodeArgs {
     // them); null: every sequence has T tokens, sequence i at rows i*T ..
     const int32_t* cu_seqlens;
     int32_t total_rows;  // with cu_seqlens: rows of the packed tensors (a sequence's rows must lie inside)
+    // speculative verify (all three set, multi-token kernel only): the pools are not
+    // written; per token the normalised key [rows][Hk][dk], the write delta
+    // [rows][Hv][dv] and the decay [rows][Hv] are
+    float* spec_k;
+    float* spec_delta;
+    float* spec_alpha;
+};
+
+// Commit of the accepted prefix of a speculative verify call.
+struct SpecCommitArgs {
+    Shape sh;
+    int B, T, P;
+    const int32_t* n_accept;
+    const uint16_t* qkv;
+    uint16_t* conv_pool;
+    float* state_pool;
+    const int32_t* slots;
+    const float* spec_k;
+    const float* spec_delta;
+    const float* spec_alpha;
+    int32_t* err_flag;
 };
 
 struct ConvArgs {
@@ -82,6 +103,27 @@ struct NormArgs {
     float* out_f32;
 };
 
+// The projection GEMM D = X W^T (bf16 in, fp32 accumulate, bf16 out): X [R][K] token
+// rows, W [N][K] weight rows; output features are routed to up to four row-major
+// outputs by consecutive ranges (segment i holds features seg_start[i] ..
+// seg_start[i] + seg_width[i] - 1 as [R][seg_width[i]]).
+constexpr int kProjMaxRows = 256;
+struct ProjArgs {
+    int N, K, R;
+    int slices;  // K-slices per weight tile (the cluster size)
+    const uint16_t* x;
+    const uint16_t* w;
+    int nseg;
+    int seg_start[4];
+    int seg_width[4];
+    uint16_t* seg_out[4];
+    float* out_f32;  // nullable: [R][N] fp32 before rounding
+    int32_t* err_flag;
+};
+int proj_slices(int N, int K, int num_sms);
+int proj_smem_bytes(int R);
+cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream);
+
 // Column slices per v-head for the fused kernel: the cluster of one (sequence,
 // k-head) holds G * NS CTAs, at most 8.
 int decode_column_splits(int B, int Hv, int G, int dv);
@@ -97,6 +139,7 @@ cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream);
 // Multi-token kernel (state in registers across the launch's tokens).
 bool multitoken_supported(const DecodeArgs& a);
 cudaError_t launch_decode_multitoken(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_spec_commit(const SpecCommitArgs& a, cudaStream_t stream);
 cudaError_t launch_conv_update(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_recurrent(const RecurrentArgs& a, cudaStream_t stream);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);

@@ -268,3 +268,30 @@ def initial_conv_state(wl: Workload, slot_ids: Optional[Sequence[int]] = None) -
     """bf16 bits [n][W-1][C]: the conv history starts at zeros."""
     n = wl.pool_slots if slot_ids is None else len(list(slot_ids))
     return np.zeros((n, wl.conv_width - 1, wl.channels), dtype=np.uint16)
+
+
+# Model width of the projections around the layer: a Qwen3-Next-like model with this
+# GDN head shape (16 k-heads, 32 v-heads of 128) has hidden size 2048.
+HIDDEN = 2048
+
+
+def proj_weights(wl: Workload, hidden: int = HIDDEN) -> Dict[str, np.ndarray]:
+    """Random-initialised projection weights (no trained checkpoint): the stacked
+    in_proj w_in [C + Hv*dv + 2*Hv][hidden] (rows: qkv | z | a | b) and out_proj w_out
+    [hidden][Hv*dv], bf16 bits ~ N(0, 0.02)."""
+    C, Z, Hv = wl.channels, wl.num_v_heads * wl.head_v_dim, wl.num_v_heads
+    n_in = C + Z + 2 * Hv
+    return {
+        "w_in": to_bf16_bits(normal(stream_key(wl.seed, "w_in"), n_in * hidden, 0.02)).reshape(n_in, hidden),
+        "w_out": to_bf16_bits(normal(stream_key(wl.seed, "w_out"), hidden * Z, 0.02)).reshape(hidden, Z),
+    }
+
+
+def proj_inputs(wl: Workload, step: int, rows: int, hidden: int = HIDDEN) -> Dict[str, np.ndarray]:
+    """Per-step inputs of the projections for `rows` token rows: the normalised layer
+    input x [rows][hidden] and the gated decode output y [rows][Hv*dv], bf16 bits ~ N(0, 1)."""
+    Z = wl.num_v_heads * wl.head_v_dim
+    return {
+        "x": to_bf16_bits(normal(stream_key(wl.seed, "x_norm", step), rows * hidden)).reshape(rows, hidden),
+        "y": to_bf16_bits(normal(stream_key(wl.seed, "y_gated", step), rows * Z)).reshape(rows, Z),
+    }

@@ -66,7 +66,7 @@ typedef enum {
 /* Bits a kernel ORs into *err_flag. */
 #define GDN_DEVICE_ERR_SLOT_RANGE 1 /* a sequence's slot is outside [0, pool_slots) */
 #define GDN_DEVICE_ERR_TIMEOUT 2    /* a bounded wait inside the kernel ran out */
-#define GDN_DEVICE_ERR_SEQLEN 4     /* gdn_decode_step_varlen: a token count < 0 or > T_max */
+#define GDN_DEVICE_ERR_SEQLEN 4     /* a token count (varlen) or accepted count (spec commit) out of range */
 
 typedef struct {
     int32_t num_k_heads; /* Hk */
@@ -192,6 +192,85 @@ gdn_status gdn_decode_step_varlen(const gdn_config* cfg, int32_t B, const int32_
                                   float* out_f32, int32_t* err_flag, void* stream);
 
 /*
+ * The projections on either side of the decode step, as GEMMs on the tensor cores
+ * (tcgen05, bf16 inputs, fp32 accumulation, bf16 outputs rounded to nearest even).
+ * Token rows: rows = B*T <= 256; hidden: the model width, a multiple of 8.
+ *
+ * gdn_in_proj — step 2 of the page (in_proj_qkv, in_proj_z and the dual-output
+ * in_proj_a / in_proj_b, all reading the same normalised input) as ONE GEMM over the
+ * four weights stacked row-wise:
+ *   x     [rows][hidden] bf16                      the normalised layer input
+ *   w_in  [C + Hv*dv + 2*Hv][hidden] bf16          rows: in_proj_qkv (C rows), in_proj_z
+ *                                                  (Hv*dv), in_proj_a (Hv), in_proj_b (Hv)
+ *   qkv [rows][C], z [rows][Hv*dv], a [rows][Hv], b [rows][Hv] bf16 outputs, laid out as
+ *                                                  gdn_decode_step takes them (T = 1 rows,
+ *                                                  or [B][T] flattened)
+ *   out_f32 [rows][C + Hv*dv + 2*Hv] fp32, nullable: the stacked outputs before rounding
+ * gdn_out_proj — the GEMV of the page's fused steps 9+10+11, out = out_proj @ y, on the
+ * decode step's output y (already normalised and gated by SiLU(z)):
+ *   y     [rows][Hv*dv] bf16, w_out [hidden][Hv*dv] bf16, out [rows][hidden] bf16
+ *   out_f32 [rows][hidden] fp32, nullable
+ * Errors: rows > 256 or hidden not a multiple of 8 give GDN_ERR_UNSUPPORTED; other
+ * checks as above, all before anything is enqueued. Every wait inside the kernel is
+ * bounded; on expiry GDN_DEVICE_ERR_TIMEOUT is OR-ed into *err_flag (nullable) and
+ * the outputs are unspecified. Launched with programmatic stream serialization.
+ */
+gdn_status gdn_in_proj(const gdn_config* cfg, int32_t hidden, int32_t rows, const uint16_t* x,
+                       const uint16_t* w_in, uint16_t* qkv, uint16_t* z, uint16_t* a, uint16_t* b, float* out_f32,
+                       int32_t* err_flag, void* stream);
+gdn_status gdn_out_proj(const gdn_config* cfg, int32_t hidden, int32_t rows, const uint16_t* y,
+                        const uint16_t* w_out, uint16_t* out, float* out_f32, int32_t* err_flag, void* stream);
+
+/*
+ * Speculative decoding: verify T drafted tokens, then keep the state after the
+ * accepted prefix only. The GDN analogue of the rewind of a rejected speculative
+ * draft on the page "metrale_model_arch/glm5next_dsa/layer.rs" (its lockstep check
+ * and rewind_to(seq_len) on a rejected draft): a linear-attention state cannot be
+ * rewound by truncation, so the verify call leaves both pools as they were and
+ * records, per token, the factors of that token's state update; the commit call
+ * applies the first n_accept[b] of them.
+ *
+ * gdn_spec_verify takes the arguments of gdn_decode_step (T = the drafted tokens,
+ * 1..16) and writes exactly the outputs a T-token gdn_decode_step would write
+ * (steps 3 to 8 and the SiLU(z) gate, the tokens in order), but neither conv_pool nor
+ * state_pool is written. Instead, for token t of sequence b:
+ *   spec_k     [B][T][Hk][dk] fp32  the normalised key k_t (L2 norm of step 3)
+ *   spec_delta [B][T][Hv][dv] fp32  the write delta_t = beta_t (v_t - alpha_t S_{t-1}^T k_t)
+ *   spec_alpha [B][T][Hv]     fp32  the decay alpha_t = exp(g_t)
+ * so that the state after token t is S_t = alpha_t S_{t-1} + k_t delta_t^T
+ * (v-head h uses k-head h / (Hv/Hk)). All three buffers are caller-owned device
+ * memory, 16-byte aligned, written in full for every sequence that is not skipped.
+ * Skipping (slot out of range) and err_flag are as in gdn_decode_step. Launched
+ * like gdn_decode_step (programmatic stream serialization, no allocation).
+ */
+gdn_status gdn_spec_verify(const gdn_config* cfg, int32_t B, int32_t T, const uint16_t* qkv, const uint16_t* a,
+                           const uint16_t* b, const uint16_t* z, const uint16_t* conv_w, const float* A_log,
+                           const float* dt_bias, const uint16_t* norm_w, const uint16_t* conv_pool,
+                           const float* state_pool, int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16,
+                           float* out_f32, float* spec_k, float* spec_delta, float* spec_alpha, int32_t* err_flag,
+                           void* stream);
+
+/*
+ * Commits the accepted prefix of a gdn_spec_verify call: sequence b keeps its first
+ * n = n_accept[b] drafted tokens. Its state becomes S_n (the updates of tokens
+ * 0..n-1 applied in order to the state the verify call read) and its conv history
+ * becomes the last W-1 raw inputs of [history, qkv tokens 0..n-1], bit for bit. The
+ * result equals that of a gdn_decode_step over the first n tokens only.
+ *   n_accept   [B] int32 device; 0 leaves the sequence's pools untouched
+ *   T          the T of the verify call (the layout of qkv and the spec buffers)
+ *   qkv        [B][T][C] bf16, the verify call's input (for the conv history)
+ *   spec_k, spec_delta, spec_alpha  as written by the verify call
+ *   conv_pool, state_pool, pool_slots, slots  the verify call's pools and slots
+ * A sequence whose n_accept is outside [0, T] is skipped and GDN_DEVICE_ERR_SEQLEN
+ * is OR-ed into *err_flag; a slot outside [0, pool_slots) is handled as in
+ * gdn_decode_step. Each named state is read once and written once (when n > 0).
+ */
+gdn_status gdn_spec_commit(const gdn_config* cfg, int32_t B, int32_t T, const int32_t* n_accept,
+                           const uint16_t* qkv, uint16_t* conv_pool, float* state_pool, int32_t pool_slots,
+                           const int32_t* slots, const float* spec_k, const float* spec_delta,
+                           const float* spec_alpha, int32_t* err_flag, void* stream);
+
+/*
  * gdn_decode_step for callers that cannot allocate device memory. The pages have
  * no counterpart of this entry point; it exists for the library's users.
  *
@@ -237,7 +316,7 @@ gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t po
 const char* gdn_status_string(gdn_status status);
 
 /* ABI version of this header: (major << 16) | minor. */
-#define GDN_ABI_VERSION ((1 << 16) | 1)
+#define GDN_ABI_VERSION ((1 << 16) | 2)
 int32_t gdn_abi_version(void);
 
 #ifdef __cplusplus

@@ -207,3 +207,64 @@ def round_bf16(x) -> np.ndarray:
     out = np.zeros(x.shape, dtype=np.uint16)
     lib.oracle_round_bf16(_p(x, np.float64), _p(out, np.uint16), ctypes.c_size_t(x.size))
     return out
+
+
+def speculative_step(shape: Shape, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w,
+                     conv_pool: np.ndarray, state_pool: np.ndarray, slots, n_accept) -> Dict[str, np.ndarray]:
+    """Speculative decoding of T drafted tokens with rollback to the accepted prefix,
+    written out from its definition: the returned outputs are those of a T-token
+    decode step (every drafted token is scored), and the pools end as after a decode
+    step over only the first n_accept[b] tokens of each sequence b. The GDN
+    counterpart of rewinding a rejected draft ("metrale_model_arch/glm5next_dsa/layer.rs",
+    the lockstep check and rewind_to): the recurrent state cannot be truncated, so
+    the accepted prefix is what the pools must hold.
+
+    Pools are updated in place (sequences are independent, so each is advanced on its
+    own); n_accept[b] = 0 leaves sequence b's pool entries untouched."""
+    qkv, a, b, z, slots = _u16(qkv), _u16(a), _u16(b), _u16(z), _i32(slots)
+    B, T = qkv.shape[:2]
+    n_accept = np.asarray(n_accept, dtype=np.int64)
+    assert n_accept.shape == (B,) and np.all((n_accept >= 0) & (n_accept <= T))
+    # every drafted token scored, on copies of the pools
+    r = decode_step(shape, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool.copy(), state_pool.copy(), slots)
+    for i in range(B):
+        n = int(n_accept[i])
+        if n == 0:
+            continue
+        decode_step(shape, qkv[i:i + 1, :n], a[i:i + 1, :n], b[i:i + 1, :n], z[i:i + 1, :n], conv_w, A_log,
+                    dt_bias, norm_w, conv_pool, state_pool, slots[i:i + 1])
+    return r
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """The exact values of bf16 bit patterns."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def linear(x_bits, w_bits) -> np.ndarray:
+    """out[r][n] = sum_k x[r][k] w[n][k] in FP64 on the exact bf16 values (a library
+    matmul as the one step: the products are exact, the sums FP64). The form of every
+    projection GEMV on the page "spark_model/forward/qwen3_5/linear_attention.rs"
+    (x @ W^T with W stored as [out_features][in_features])."""
+    x, w = bf16_to_f64(x_bits), bf16_to_f64(w_bits)
+    assert x.ndim == 2 and w.ndim == 2 and x.shape[1] == w.shape[1]
+    return x @ w.T
+
+
+def in_proj(shape: Shape, x_bits, w_in_bits) -> Dict[str, np.ndarray]:
+    """Step 2 of the page: the projections of the normalised input x_norm [R][hidden]
+    into qkv [R][C], z [R][Hv*dv] and the gate and beta inputs a, b [R][Hv], with the
+    four weights stacked row-wise in that order: w_in [C + Hv*dv + 2*Hv][hidden]
+    (in_proj_qkv | in_proj_z | in_proj_a | in_proj_b)."""
+    y = linear(x_bits, w_in_bits)
+    C, Z, Hv = shape.channels, shape.num_v_heads * shape.head_v_dim, shape.num_v_heads
+    assert y.shape[1] == C + Z + 2 * Hv
+    return {"qkv": y[:, :C], "z": y[:, C:C + Z], "a": y[:, C + Z:C + Z + Hv], "b": y[:, C + Z + Hv:], "all": y}
+
+
+def out_proj(shape: Shape, y_bits, w_out_bits) -> np.ndarray:
+    """The GEMV of the page's fused steps 9+10+11: out = out_proj @ y with y [R][Hv*dv]
+    the SiLU(z)-gated, normalised decode output and w_out [hidden][Hv*dv]."""
+    assert np.asarray(y_bits).shape[1] == shape.num_v_heads * shape.head_v_dim
+    return linear(y_bits, w_out_bits)

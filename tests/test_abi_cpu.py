@@ -147,6 +147,48 @@ def test_static_scratch_checks_every_argument_before_touching_the_device(L):
     assert gdn.decode_static_scratch_bytes() >= gdn.decode_workspace_bytes()
 
 
+def spec_verify(L, cfg, B=4, T=4, ptrs=None, pool=8, out_f32=None, spec=None, err=None):
+    p = [FAKE] * 10 if ptrs is None else ptrs
+    s = [FAKE] * 3 if spec is None else spec
+    return L.gdn_spec_verify(ctypes.byref(cfg) if cfg is not None else None, B, T, *p, pool, FAKE, FAKE, out_f32,
+                             *s, err, None)
+
+
+def spec_commit(L, cfg, B=4, T=4, ptrs=None, pool=8, err=None):
+    p = [FAKE] * 8 if ptrs is None else ptrs  # n_accept, qkv, conv_pool, state_pool, slots, k, delta, alpha
+    return L.gdn_spec_commit(ctypes.byref(cfg) if cfg is not None else None, B, T, p[0], p[1], p[2], p[3], pool,
+                             p[4], p[5], p[6], p[7], err, None)
+
+
+def test_spec_entry_points_check_every_argument_before_touching_the_device(L):
+    cfg = good_cfg()
+    for call in (spec_verify, spec_commit):
+        assert call(L, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+        assert call(L, good_cfg(head_v_dim=48)) == gdn.GDN_ERR_UNSUPPORTED
+        assert call(L, cfg, T=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+        assert call(L, cfg, T=17) == gdn.GDN_ERR_UNSUPPORTED
+        assert call(L, cfg, B=-2) == gdn.GDN_ERR_INVALID_ARGUMENT
+        assert call(L, cfg, pool=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+        assert call(L, cfg, B=0, ptrs=[None] * (10 if call is spec_verify else 8)) == gdn.GDN_OK
+        assert call(L, cfg, err=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    for i in range(3):
+        spec = [FAKE] * 3
+        spec[i] = None
+        assert spec_verify(L, cfg, spec=spec) == gdn.GDN_ERR_INVALID_ARGUMENT, i
+        spec[i] = FAKE_ODD
+        assert spec_verify(L, cfg, spec=spec) == gdn.GDN_ERR_MISALIGNED, i
+    for i in range(10):
+        ptrs = [FAKE] * 10
+        ptrs[i] = FAKE_ODD
+        assert spec_verify(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
+    for i in range(8):
+        ptrs = [FAKE] * 8
+        ptrs[i] = None
+        assert spec_commit(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
+        ptrs[i] = FAKE_ODD
+        assert spec_commit(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
+
+
 def test_empty_batch_is_a_no_op(L):
     # B = 0 returns before any pointer is looked at or any launch is made
     assert decode(L, good_cfg(), B=0, ptrs=[None] * 10) == gdn.GDN_OK

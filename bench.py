@@ -103,6 +103,8 @@ KERNEL_SOURCES = {
     "decode_ws_kernel": ("gdn_decode_persistent.cu",),
     "decode_mt_kernel": ("gdn_decode_mt.cu",),
     "decode_fused_tma_kernel": ("gdn_decode.cu",),
+    "proj_gemm_kernel": ("gdn_proj.cu",),
+    "spec_commit_kernel": ("gdn_spec.cu",),
 }
 SHARED_SOURCES = ("gdn_device.cuh", "gdn_internal.h")
 
@@ -364,6 +366,221 @@ def workload_config(wl, args, world):
             "parallelism": f"dp{world} (independent sequence shards, no collective)"}
 
 
+# ---------------------------------------------------------------------------------
+# The rows around the decode step: the projection GEMMs and speculative decoding.
+EXTRA_WORKLOADS = {
+    # name: (base decode workload, kind, token rows)
+    "in_proj_b64": ("batch64", "in_proj", 64),
+    "out_proj_b64": ("batch64", "out_proj", 64),
+    "spec_b32_t16": ("multitoken_b32_t16", "spec", None),
+}
+
+
+def time_graph_steps(launch, n_sets, K, args, dev, world, stream):
+    """W eager warm-up launches, then exactly K steps replayed from CUDA graphs (step j
+    uses input set j % n_sets), the K-step region repeated for about --timed-seconds;
+    returns (median ms per K steps, repeats, per-repeat ms, wall-clock window)."""
+    import torch
+    import torch.distributed as dist
+    for i in range(args.warmup):
+        launch(i % n_sets)
+    torch.cuda.synchronize()
+    graphs = []
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    for count in (n_sets, K % n_sets):
+        if count == 0:
+            graphs.append(None)
+            continue
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(count):
+                launch(i)
+        graphs.append(g)
+    for _ in range(max(1, args.warmup // n_sets)):
+        graphs[0].replay()
+    torch.cuda.synchronize()
+
+    def k_steps():
+        for _ in range(K // n_sets):
+            graphs[0].replay()
+        if graphs[1] is not None:
+            graphs[1].replay()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    k_steps()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
+    R = int(min(args.max_repeats, max(3, round(args.timed_seconds * 1e3 / max(one_ms, 1e-3)))))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(R)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(R)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for r in range(R):
+        starts[r].record(stream)
+        k_steps()
+        ends[r].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t1 = time.time()
+    rep = [starts[r].elapsed_time(ends[r]) for r in range(R)]
+    if world > 1:
+        t = torch.tensor(rep, device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        rep = t.tolist()
+    del graphs
+    return statistics.median(rep), R, rep, (t0, t1)
+
+
+def run_extra(args, name, rank, world):
+    """The projection GEMMs (gdn_in_proj / gdn_out_proj at B=64 token rows, hidden
+    2048) or speculative decoding (gdn_spec_verify of 16 drafted tokens for 32
+    sequences, then gdn_spec_commit of a seeded accepted count per sequence): one JSON
+    line with the roofline of the step's dominant kernel. Weights and pools are cycled
+    over independent sets larger than L2 so each step reads them from HBM."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_102_b200 as gdn
+    from gated_delta_rule_102_b200 import build as gdn_build
+    from gated_delta_rule_102_b200 import synth
+    base, kind, rows = EXTRA_WORKLOADS[name]
+    wl = rank_workload(synth.WORKLOADS[base], rank)
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        gdn_build.build()
+    if world > 1:
+        dist.barrier()
+    gdn.lib()
+    stream = torch.cuda.current_stream(dev)
+    cfg = gdn.GdnConfig.make(wl.num_k_heads, wl.num_v_heads, wl.head_k_dim, wl.head_v_dim, wl.conv_width)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    C, Z, Hv, H = wl.channels, wl.num_v_heads * wl.head_v_dim, wl.num_v_heads, synth.HIDDEN
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    sampler = ClockSampler(local) if rank == 0 else None
+    peak, peak_kind = hbm_peak()
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    if kind in ("in_proj", "out_proj"):
+        N, K = (C + Z + 2 * Hv, H) if kind == "in_proj" else (H, Z)
+        wbytes = N * K * 2
+        sets = max(2, -(-2 * L2_BYTES // wbytes))  # weight sets cycled: at least twice L2
+        ws = [(torch.randn(N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for _ in range(sets)]
+        xs = [torch.randn(rows, K, generator=gen, device=dev).to(torch.bfloat16) for _ in range(sets)]
+        if kind == "in_proj":
+            outs = [torch.empty(rows, n, dtype=torch.bfloat16, device=dev) for n in (C, Z, Hv, Hv)]
+
+            def launch(i):
+                gdn.gdn_in_proj(cfg, xs[i], ws[i], *outs, None, err)
+        else:
+            out = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+
+            def launch(i):
+                gdn.gdn_out_proj(cfg, xs[i], ws[i], out, None, err)
+        nbytes = wbytes + rows * K * 2 + rows * N * 2
+        flops = 2 * rows * N * K
+        tokens_per_step = rows
+        kernel = "proj_gemm_kernel"
+        note = f"{sets} weight sets x {wbytes / 2**20:.1f} MiB cycled (inputs larger than L2)"
+        desc = (f"{name}: {kind} GEMM, {rows} token rows x hidden {H}, weights [{N}][{K}] bf16 "
+                f"(Hk={wl.num_k_heads}, Hv={Hv}, dk={wl.head_k_dim}, dv={wl.head_v_dim})")
+        metric = f"GDN {kind} GEMM tokens/s and achieved HBM GB/s at B={rows}"
+    else:
+        B, T = wl.batch, wl.tokens
+        sets = args.pools
+        pool_bytes = wl.pool_slots * Hv * wl.head_k_dim * wl.head_v_dim * 4
+        states = [torch.from_numpy(synth.initial_state(wl.replace(seed=wl.seed + 101 * p))).to(dev)
+                  for p in range(sets)]
+        convs = [torch.zeros(wl.pool_slots, wl.conv_width - 1, C, dtype=torch.bfloat16, device=dev)
+                 for _ in range(sets)]
+        w = synth.weights(wl)
+
+        def bf16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+        conv_w, norm_w = bf16(w["conv_w"]), bf16(w["norm_w"])
+        A_log, dt_bias = torch.from_numpy(w["A_log"]).to(dev), torch.from_numpy(w["dt_bias"]).to(dev)
+        slots = torch.from_numpy(synth.slots(wl)).to(dev)
+        xin = [{k: bf16(v) for k, v in synth.step_inputs(wl, s).items()} for s in range(sets)]
+        rng = np.random.default_rng(wl.seed)
+        naccs = [rng.integers(0, T + 1, B).astype(np.int32) for _ in range(sets)]
+        nacc = [torch.from_numpy(a).to(dev) for a in naccs]
+        out = torch.empty(B, T, Hv, wl.head_v_dim, dtype=torch.bfloat16, device=dev)
+        sk = torch.empty(B, T, wl.num_k_heads, wl.head_k_dim, dtype=torch.float32, device=dev)
+        sd = torch.empty(B, T, Hv, wl.head_v_dim, dtype=torch.float32, device=dev)
+        sa = torch.empty(B, T, Hv, dtype=torch.float32, device=dev)
+
+        def launch(i):
+            x = xin[i]
+            gdn.gdn_spec_verify(cfg, x["qkv"], x["a"], x["b"], x["z"], conv_w, A_log, dt_bias, norm_w, convs[i],
+                                states[i], slots, out, sk, sd, sa, None, err)
+            gdn.gdn_spec_commit(cfg, nacc[i], x["qkv"], convs[i], states[i], slots, sk, sd, sa, err)
+        # verify: the state read once, the inputs, outputs and factors; commit: each accepted
+        # sequence's state read and written, its factors read, its history rolled
+        S = Hv * wl.head_k_dim * wl.head_v_dim * 4
+        per_tok = C * 2 + 2 * Hv * 2 + 2 * Z * 2 + (wl.num_k_heads * wl.head_k_dim + Z + Hv) * 4
+        acc = float(np.mean([int((a > 0).sum()) for a in naccs]))
+        ntok_acc = float(np.mean([int(a.sum()) for a in naccs]))
+        nbytes = (B * (S + 2 * (wl.conv_width - 1) * C * 2 + 4) + B * T * per_tok + C * wl.conv_width * 2 +
+                  acc * (2 * S + 4) + ntok_acc * (wl.num_k_heads * wl.head_k_dim + Z + Hv) * 4)
+        flops = 7 * B * T * Hv * wl.head_k_dim * wl.head_v_dim
+        tokens_per_step = B * T
+        kernel = "decode_mt_kernel"
+        note = f"{sets} state pools x {pool_bytes >> 20} MiB cycled (inputs larger than L2)"
+        desc = (f"{name}: verify {B} sequences x {T} drafted tokens, then commit a seeded accepted count "
+                f"(0..{T}, mean {ntok_acc / B:.1f}) per sequence; Hk={wl.num_k_heads}, Hv={Hv}, "
+                f"dk={wl.head_k_dim}, dv={wl.head_v_dim}, conv width {wl.conv_width}")
+        metric = "GDN speculative verify+commit drafted tokens/s at B=32, T=16"
+    K = args.steps
+    ms, R, rep, (tw0, tw1) = time_graph_steps(launch, sets, K, args, dev, world, stream)
+    if int(err.item()) != 0:
+        raise RuntimeError("device reported an error flag %d" % int(err.item()))
+    clocks = None
+    if sampler is not None:
+        sampler.stop()
+        clocks = sampler.summary(tw0, tw1)
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    step_s = ms / K / 1e3
+    gbs = nbytes / step_s / 1e9
+    roof = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+            "traffic": profiled_traffic(kernel, name),
+            "peak_source": f"{peak_kind} copy bandwidth", "kernel": kernel, "kernel_us": step_s * 1e6,
+            "algorithmic_bytes": int(nbytes), "algorithmic_flops": int(flops),
+            "tflops_achieved": flops / step_s / 1e12}
+    sm_mhz = (clocks or {}).get("sm_mhz")
+    if kind == "spec" and sm_mhz:
+        alu_peak = num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6
+        alu = flops / step_s / 1e12
+        if alu / alu_peak > roof["frac"]:
+            roof = dict(roof, bound="alu", achieved=alu, peak=alu_peak, unit="TFLOP/s", frac=alu / alu_peak,
+                        peak_source="FP32 FMA lanes x measured SM clock", hbm_gbs_achieved=gbs, hbm_frac=gbs / peak)
+    line = {"metric": metric, "value": world * tokens_per_step / step_s, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 in, f32 accumulate" if kind != "spec" else "f32",
+            "data": "synthetic (seeded normal weights and inputs)",
+            "timing": {"repeats": R, "reported": "median of the repeated K-step regions",
+                       "ms_per_step_min": min(rep) / K, "ms_per_step_max": max(rep) / K},
+            "config": {"workload": desc, "l2": note, "parallelism": f"dp{world} (independent shards, no collective)"},
+            "roofline": roof, "e2e": None, "clocks": clocks,
+            "gpu_launches": K * (2 if kind == "spec" else 1)}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -372,6 +589,12 @@ def main():
     if args.gpus != world:
         sys.exit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
     from gated_delta_rule_102_b200 import synth
+    if args.workload in EXTRA_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the oracle arm is timed on the decode workloads"}))
+            return
+        run_extra(args, args.workload, rank, world)
+        return
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl, rank, world)

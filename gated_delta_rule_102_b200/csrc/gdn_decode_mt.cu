@@ -74,14 +74,6 @@ __device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
 // few ulp; evaluated for every conv channel and every output element of every token).
 __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
-// Tokens of the recurrence taken together (a chunk); the on-chip buffers hold a whole
-// number of chunks, the tokens past a sequence's last one being zero.
-constexpr int kChunk = 4;
-// Per (v-head, chunk): the scalars of the chunked recurrence (see the token loop).
-constexpr int kCoefFloats = 36;
-// Per token: raw k.k and k.q against the tokens of its chunk, and q.q.
-constexpr int kGramFloats = 12;
-
 template <int DK, int DV>
 struct MtGeo {
     static constexpr int NWH = DV / 16;                       // warps per v-head: 16 columns each
@@ -93,28 +85,20 @@ struct MtGeo {
     static constexpr int NCHC = 2 * DK + NHC * DV;             // most conv channels of a pass
     static constexpr int TILE = DK * DV * 4;
     static_assert(DV % 16 == 0 && RPL >= 2 && (RPL == 2 || RPL % 4 == 0), "multi-token geometry");
-    static __host__ __device__ int padded(int T) { return (T + kChunk - 1) / kChunk * kChunk; }
     // Shared memory (bytes, every block 16-byte aligned): the stage (NHC state tiles,
     // the staged raw rows and the weights), then the raw q and k per token, v per v-head
     // and token (replaced by o: the warp that reads v_t of a column writes o_t of it),
-    // the z rows of the pass, the per-token scalars, the Gram entries, the chunk
-    // coefficients, the stage's slot and the abort flag, and the stage and z barriers.
-    // Token buffers hold padded(T) tokens.
+    // the z rows of the pass, the per-token scalars, the stage's slot and the abort
+    // flag, and the stage and z barriers.
     static __host__ __device__ int rows_off() { return NHC * TILE; }
     static __host__ __device__ int wts_off(int W, int T) { return rows_off() + ((W - 1 + T) * NCHC * 2 + 15) / 16 * 16; }
     static __host__ __device__ int qk_off(int W, int T) { return wts_off(W, T) + (NCHC * W * 2 + 15) / 16 * 16; }
-    static __host__ __device__ int vs_off(int W, int T) { return qk_off(W, T) + padded(T) * 2 * DK * 4; }
-    static __host__ __device__ int zb_off(int W, int T) { return vs_off(W, T) + padded(T) * NHC * DV * 4; }
+    static __host__ __device__ int vs_off(int W, int T) { return qk_off(W, T) + T * 2 * DK * 4; }
+    static __host__ __device__ int zb_off(int W, int T) { return vs_off(W, T) + T * NHC * DV * 4; }
     static __host__ __device__ int sc_off(int W, int T) { return zb_off(W, T) + T * NHC * DV * 2; }
-    static __host__ __device__ int gram_off(int W, int T) {
-        return (sc_off(W, T) + padded(T) * NHC * (int)sizeof(TokenScalars) + 15) / 16 * 16;
+    static __host__ __device__ int ctl_off(int W, int T) {
+        return (sc_off(W, T) + T * NHC * (int)sizeof(TokenScalars) + 15) / 16 * 16;
     }
-    static __host__ __device__ int coef_off(int W, int T) { return gram_off(W, T) + padded(T) * kGramFloats * 4; }
-    static __host__ __device__ int dsm_off(int W, int T) {
-        return coef_off(W, T) + NHC * (padded(T) / kChunk) * kCoefFloats * 4;
-    }
-    // per warp: the writes delta of the current chunk's tokens on its 16 columns
-    static __host__ __device__ int ctl_off(int W, int T) { return dsm_off(W, T) + NW * kChunk * 16 * 4; }
     static __host__ __device__ int total(int W, int T) { return ctl_off(W, T) + 32; }
     // the control block: the stage's slot, the abort flag, the stage and z barriers,
     // the stage's first packed row and token count
@@ -139,7 +123,6 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     extern __shared__ __align__(128) unsigned char smem[];
     // T: the most tokens a sequence has in this launch (it sizes the shared buffers)
     const int T = p.T, W = p.sh.W, C = p.sh.C, Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk;
-    const int TP = Geo::padded(T);  // token rows of the on-chip buffers
     const int npass = G / NH, NCH = 2 * DK + NH * DV;
     const int ngroups = p.B * Hk;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -151,9 +134,6 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     float* os = vs;  // o_t of a column replaces v_t once the warp owning the column has read it
     uint16_t* zb = reinterpret_cast<uint16_t*>(smem + Geo::zb_off(W, T));
     TokenScalars* sc = reinterpret_cast<TokenScalars*>(smem + Geo::sc_off(W, T));
-    float* gram = reinterpret_cast<float*>(smem + Geo::gram_off(W, T));
-    float* coef = reinterpret_cast<float*>(smem + Geo::coef_off(W, T));
-    float* dsm = reinterpret_cast<float*>(smem + Geo::dsm_off(W, T)) + warp * (kChunk * 16);
     volatile int* stage_slot = reinterpret_cast<volatile int*>(smem + Geo::ctl_off(W, T));
     volatile int* abort_flag = stage_slot + 1;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Geo::ctl_off(W, T) + 8);
@@ -358,7 +338,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                         qk[t * 2 * DK + lc] = sv;
                     } else {
                         const int v_h = (lc - 2 * DK) / DV, v_j = lc - 2 * DK - v_h * DV;
-                        vs[(v_h * TP + t) * DV + v_j] = sv;
+                        vs[(v_h * T + t) * DV + v_j] = sv;
                     }
                 }
             }
@@ -382,64 +362,34 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                     *reinterpret_cast<const uint4*>(rows + (ntok + r) * NCH + lc);
             }
         }
-        // ---- steps 4, 5: decay and write strength per v-head and token. The tokens that pad
-        // the last chunk get decay 1 and strength 0, and zero q, k and v: they change nothing.
-        const int ntp = (ntok + kChunk - 1) / kChunk * kChunk;
-        if (tid < ntp * NH) {
+        // ---- steps 4, 5: decay and write strength per v-head and token
+        if (tid < ntok * NH) {
             const int t = tid / NH, k = tid - t * NH;
-            TokenScalars& st = sc[t * Geo::NHC + k];
-            if (t < ntok) {
-                gate_and_beta(g_a, g_b, g_A, g_dt, st.alpha, st.beta);
-            } else {
-                st.alpha = 1.f;
-                st.beta = 0.f;
-            }
-        }
-        for (int i = tid; i < (ntp - ntok) * 2 * DK; i += Geo::NT) qk[ntok * 2 * DK + i] = 0.f;
-        for (int i = tid; i < NH * (ntp - ntok) * DV; i += Geo::NT) {
-            const int h = i / ((ntp - ntok) * DV), r = i - h * (ntp - ntok) * DV;
-            vs[(h * TP + ntok) * DV + r] = 0.f;
+            gate_and_beta(g_a, g_b, g_A, g_dt, sc[t * Geo::NHC + k].alpha, sc[t * Geo::NHC + k].beta);
         }
         __syncthreads();  // the stage is empty; k, q, v are in
         prefetch(u + 1, next_slot, next_tok0, next_ntok);
-        // ---- step 3's L2 norms, as factors on the raw q and k, and the raw dot products
-        // the chunked recurrence needs: a warp per token t, against the tokens of its chunk
-        for (int t = warp; t < ntp; t += Geo::NW) {
-            const int c0t = t - t % kChunk;
-            const float* qt = qk + t * 2 * DK;
-            const float* kt = qt + DK;
-            float acc[kGramFloats - 3];  // k_i.k_t (4), k_i.q_t (4), q_t.q_t
-#pragma unroll
-            for (int i = 0; i < kGramFloats - 3; ++i) acc[i] = 0.f;
+        // ---- L2 norms of q and k (step 3) as factors on the raw values, and k.q: a warp per token
+        for (int t = warp; t < ntok; t += Geo::NW) {
+            float sq = 0.f, sk = 0.f, dot = 0.f;
             for (int r = lane; r < DK; r += 32) {
-                const float qv = qt[r], kv = kt[r];
-#pragma unroll
-                for (int i = 0; i < kChunk; ++i) {
-                    const float ki = qk[(c0t + i) * 2 * DK + DK + r];
-                    acc[i] = fmaf(ki, kv, acc[i]);
-                    acc[kChunk + i] = fmaf(ki, qv, acc[kChunk + i]);
-                }
-                acc[2 * kChunk] = fmaf(qv, qv, acc[2 * kChunk]);
+                const float a = qk[t * 2 * DK + r], b = qk[t * 2 * DK + DK + r];
+                sq = fmaf(a, a, sq);
+                sk = fmaf(b, b, sk);
+                dot = fmaf(a, b, dot);
             }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-                for (int i = 0; i < kGramFloats - 3; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-            if (lane < kGramFloats - 3) {
-                float v = acc[0];
-#pragma unroll
-                for (int i = 1; i < kGramFloats - 3; ++i) v = lane == i ? acc[i] : v;
-                gram[t * kGramFloats + lane] = v;
+            for (int off = 16; off > 0; off >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                dot += __shfl_xor_sync(0xffffffffu, dot, off);
             }
-            const float nq = t < ntok ? rsqrtf(acc[2 * kChunk] + p.sh.l2_eps) * p.sh.q_scale : 0.f;
-            float kk = acc[0];  // k_t . k_t
-#pragma unroll
-            for (int i = 1; i < kChunk; ++i) kk = t - c0t == i ? acc[i] : kk;
-            const float nk = t < ntok ? rsqrtf(kk + p.sh.l2_eps) : 0.f;
+            const float nq = rsqrtf(sq + p.sh.l2_eps) * p.sh.q_scale, nk = rsqrtf(sk + p.sh.l2_eps);
             for (int k = lane; k < NH; k += 32) {
                 TokenScalars& st = sc[t * Geo::NHC + k];
                 st.nq = nq;
                 st.nk = nk;
+                st.kq = dot * nq * nk;
             }
         }
         __syncthreads();
@@ -454,271 +404,108 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                 p.spec_alpha[((size_t)tok0 + t) * Hv + h0 + k] = sc[t * Geo::NHC + k].alpha;
             }
         }
-        // ---- the scalars of each (v-head, chunk). With the chunk's
-        // decays a_j (j = 0..3), Gamma_j = a_0 ... a_j and A_ji = a_{i+1} ... a_j (A_jj = 1),
-        // S0 = c0 S~ the state at the chunk's start and normalised k_j = nk_j k~_j,
-        // q_j = nq_j q~_j (k~, q~ raw), the tokens of the chunk give
-        //   delta_j = b_j v_j - b_j c0 Gamma_j nk_j (S~^T k~_j) - sum_{i<j} b_j A_ji (k_i.k_j) delta_i
-        //   o_j     = c0 Gamma_j nq_j (S~^T q~_j) + sum_{i<=j} A_ji (k_i.q_j) delta_i
-        //   S_end   = Gamma_3 S0 + sum_i A_3i k_i delta_i^T.
-        // The registers keep S~ = S / c with c the running product of the decays; when c
-        // would fall below 2^-64 it is folded into the registers (S~ <- c S~, c <- 1).
-        // Block layout: b[4], ek[4] (on S~^T k~), eq[4] (on S~^T q~), L[6] (row j, i < j),
-        // Q[10] (row j, i <= j), f[4] (factor of delta_i on k~_i in the update), the fold
-        // multiplier, the fold flag and the running scale after the chunk.
-        const int nchunk = ntp / kChunk;
-        // A thread per coefficient: the running scale at its chunk's start (a scan over
-        // the chunks before it), then the one entry.
-        for (int e = tid; e < NH * nchunk * kCoefFloats; e += Geo::NT) {
-            const int k = e / (nchunk * kCoefFloats), rem = e - k * nchunk * kCoefFloats;
-            const int m = rem / kCoefFloats, idx = rem - m * kCoefFloats;
-            const TokenScalars* sk = sc + k;  // token t of v-head k: sk[t * NHC]
-            float c0 = 1.f;
-            for (int mm = 0; mm < m; ++mm) {
-                float gl = 1.f;
-#pragma unroll
-                for (int j = 0; j < kChunk; ++j) gl *= sk[(mm * kChunk + j) * Geo::NHC].alpha;
-                const float cn = c0 * gl;
-                c0 = cn < 0x1p-64f ? 1.f : cn;
-            }
-            const TokenScalars* s0 = sk + m * kChunk * Geo::NHC;
-            auto al = [&](int j) { return s0[j * Geo::NHC].alpha; };
-            auto gam = [&](int j) {  // decays of tokens 0..j of the chunk
-                float r = 1.f;
-                for (int x = 0; x <= j; ++x) r *= al(x);
-                return r;
-            };
-            auto A = [&](int j, int i) {  // decays of tokens i+1..j of the chunk
-                float r = 1.f;
-                for (int x = i + 1; x <= j; ++x) r *= al(x);
-                return r;
-            };
-            const float* gr = gram + m * kChunk * kGramFloats;  // row j: k_i.k_j (i < 4), k_i.q_j, q_j.q_j
-            float v;
-            if (idx < 4) {
-                v = s0[idx * Geo::NHC].beta;
-            } else if (idx < 8) {
-                const int j = idx - 4;
-                v = s0[j * Geo::NHC].beta * c0 * gam(j) * s0[j * Geo::NHC].nk;
-            } else if (idx < 12) {
-                const int j = idx - 8;
-                v = c0 * gam(j) * s0[j * Geo::NHC].nq;
-            } else if (idx < 18) {  // L, row j, i < j
-                const int l = idx - 12, j = l < 1 ? 1 : (l < 3 ? 2 : 3), i = l - j * (j - 1) / 2;
-                v = s0[j * Geo::NHC].beta * A(j, i) * s0[i * Geo::NHC].nk * s0[j * Geo::NHC].nk * gr[j * kGramFloats + i];
-            } else if (idx < 28) {  // Q, row j, i <= j
-                const int l = idx - 18, j = l < 1 ? 0 : (l < 3 ? 1 : (l < 6 ? 2 : 3)), i = l - j * (j + 1) / 2;
-                v = A(j, i) * s0[i * Geo::NHC].nk * s0[j * Geo::NHC].nq * gr[j * kGramFloats + kChunk + i];
-            } else {
-                const float cn = c0 * gam(kChunk - 1);
-                const bool fold = cn < 0x1p-64f;
-                if (idx < 32) {
-                    const int j = idx - 28;
-                    v = fold ? A(kChunk - 1, j) * s0[j * Geo::NHC].nk : __fdividef(s0[j * Geo::NHC].nk, c0 * gam(j));
-                } else if (idx == 32) {
-                    v = fold ? cn : 1.f;
-                } else if (idx == 33) {
-                    v = fold ? 1.f : 0.f;
-                } else if (idx == 34) {
-                    v = fold ? 1.f : cn;
-                } else {
-                    v = 0.f;
-                }
-            }
-            coef[(k * (TP / kChunk) + m) * kCoefFloats + idx] = v;
-        }
-        __syncthreads();
 
-        // ---- steps 6, 7: the recurrence, a chunk of tokens at a time, on this warp's columns
+        // ---- steps 6, 7: the recurrence, token by token, on this warp's columns
         if (active) {
-            float cfin = 1.f;  // the running scale after the last chunk
-            for (int m = 0; m < nchunk; ++m) {
-                const float* cf = coef + (hh * (TP / kChunk) + m) * kCoefFloats;
-                const float* qk0 = qk + m * kChunk * 2 * DK;  // raw q then raw k of the chunk's tokens
-                // S~^T k~_j for the chunk's tokens, two at a time, over this lane's rows (even and
-                // odd rows apart), then summed over the row groups (lanes with the same columns)
-                float mk[kChunk][4];
+            float c = 1.f;  // S = c * S~ (the registers hold S~)
+            for (int t = 0; t < ntok; ++t) {
+                const float* qr = qk + t * 2 * DK;
+                const float* kr = qr + DK;
+                f2 ak[4], aq[4];  // per column: S~^T k and S~^T q over the even and the odd rows
 #pragma unroll
-                for (int h2 = 0; h2 < kChunk; h2 += 2) {
-                    f2 ak[2][4];
+                for (int cc = 0; cc < 4; ++cc) ak[cc] = aq[cc] = 0ull;
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) ak[j][cc] = 0ull;
-#pragma unroll
-                    for (int jb = 0; jb < NB; ++jb) {
-                        const int r0 = mt_row<RPL>(jb, rg, 0);
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const float* kr = qk0 + (h2 + j) * 2 * DK + DK;
-                            f2 kp[EPB / 2];
-                            if constexpr (EPB == 4) {
-                                const ulonglong2 k2 = *reinterpret_cast<const ulonglong2*>(kr + r0);
-                                kp[0] = k2.x; kp[1] = k2.y;
-                            } else {
-                                kp[0] = *reinterpret_cast<const f2*>(kr + r0);
-                            }
-#pragma unroll
-                            for (int e = 0; e < EPB / 2; ++e) {
-                                const f2* pr = P[jb * (EPB / 2) + e];
-#pragma unroll
-                                for (int cc = 0; cc < 4; ++cc) ak[j][cc] = f2_fma(pr[cc], kp[e], ak[j][cc]);
-                            }
-                        }
+                for (int j = 0; j < NB; ++j) {
+                    const int r0 = mt_row<RPL>(j, rg, 0);
+                    f2 kp[EPB / 2], qp[EPB / 2];  // (k_r, k_r+1) and (q_r, q_r+1) of this block's row pairs
+                    if constexpr (EPB == 4) {
+                        const ulonglong2 k2 = *reinterpret_cast<const ulonglong2*>(kr + r0);
+                        const ulonglong2 q2 = *reinterpret_cast<const ulonglong2*>(qr + r0);
+                        kp[0] = k2.x; kp[1] = k2.y; qp[0] = q2.x; qp[1] = q2.y;
+                    } else {
+                        kp[0] = *reinterpret_cast<const f2*>(kr + r0);
+                        qp[0] = *reinterpret_cast<const f2*>(qr + r0);
                     }
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
+                    for (int e = 0; e < EPB / 2; ++e) {
+                        const f2* pr = P[j * (EPB / 2) + e];
 #pragma unroll
                         for (int cc = 0; cc < 4; ++cc) {
-                            const float2 x = f2_unpack(ak[j][cc]);
-                            mk[h2 + j][cc] = x.x + x.y;
-                        }
-#pragma unroll
-                    for (int off = Geo::CG; off < 32; off <<= 1)
-#pragma unroll
-                        for (int j = 0; j < 2; ++j)
-#pragma unroll
-                            for (int cc = 0; cc < 4; ++cc)
-                                mk[h2 + j][cc] += __shfl_xor_sync(0xffffffffu, mk[h2 + j][cc], off);
-                }
-                // delta of every token of the chunk (forward substitution), per column; the row
-                // group 0 lanes keep it in this warp's shared buffer for the readout and update
-                {
-                    float d[kChunk][4];
-                    int li = 12;
-#pragma unroll
-                    for (int j = 0; j < kChunk; ++j) {
-                        const float4 v4 = *reinterpret_cast<const float4*>(vs + (hh * TP + m * kChunk + j) * DV + col);
-                        const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-                        const float bj = cf[j], ekj = cf[4 + j];
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) d[j][cc] = fmaf(-ekj, mk[j][cc], bj * vv[cc]);
-#pragma unroll
-                        for (int i = 0; i < j; ++i, ++li) {
-                            const float l = cf[li];
-#pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) d[j][cc] = fmaf(-l, d[i][cc], d[j][cc]);
-                        }
-                    }
-                    if (rg == 0) {
-#pragma unroll
-                        for (int j = 0; j < kChunk; ++j) {
-                            const float4 dj = make_float4(d[j][0], d[j][1], d[j][2], d[j][3]);
-                            reinterpret_cast<float4*>(dsm + j * 16)[cg] = dj;
-                            if (spec && m * kChunk + j < ntok)
-                                *reinterpret_cast<float4*>(p.spec_delta +
-                                                           (((size_t)tok0 + m * kChunk + j) * Hv + h0 + hh) * DV + col) = dj;
+                            ak[cc] = f2_fma(pr[cc], kp[e], ak[cc]);
+                            aq[cc] = f2_fma(pr[cc], qp[e], aq[cc]);
                         }
                     }
                 }
-                __syncwarp();  // every lane has read v of these columns before o replaces it, and delta is in
-                auto delta = [&](int j) { return reinterpret_cast<const float4*>(dsm + j * 16)[cg]; };
-                // S~^T q~_j two tokens at a time, then o_j
+                float mk[4], mq[4];
 #pragma unroll
-                for (int h2 = 0; h2 < kChunk; h2 += 2) {
-                    f2 aq[2][4];
+                for (int cc = 0; cc < 4; ++cc) {
+                    const float2 x = f2_unpack(ak[cc]), y = f2_unpack(aq[cc]);
+                    mk[cc] = x.x + x.y;
+                    mq[cc] = y.x + y.y;
+                }
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
+                for (int off = Geo::CG; off < 32; off <<= 1) {  // over the row groups (lanes with the same columns)
 #pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) aq[j][cc] = 0ull;
-#pragma unroll
-                    for (int jb = 0; jb < NB; ++jb) {
-                        const int r0 = mt_row<RPL>(jb, rg, 0);
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const float* qr = qk0 + (h2 + j) * 2 * DK;
-                            f2 qp[EPB / 2];
-                            if constexpr (EPB == 4) {
-                                const ulonglong2 q2 = *reinterpret_cast<const ulonglong2*>(qr + r0);
-                                qp[0] = q2.x; qp[1] = q2.y;
-                            } else {
-                                qp[0] = *reinterpret_cast<const f2*>(qr + r0);
-                            }
-#pragma unroll
-                            for (int e = 0; e < EPB / 2; ++e) {
-                                const f2* pr = P[jb * (EPB / 2) + e];
-#pragma unroll
-                                for (int cc = 0; cc < 4; ++cc) aq[j][cc] = f2_fma(pr[cc], qp[e], aq[j][cc]);
-                            }
-                        }
-                    }
-                    float mq[2][4];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const float2 x = f2_unpack(aq[j][cc]);
-                            mq[j][cc] = x.x + x.y;
-                        }
-#pragma unroll
-                    for (int off = Geo::CG; off < 32; off <<= 1)
-#pragma unroll
-                        for (int j = 0; j < 2; ++j)
-#pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) mq[j][cc] += __shfl_xor_sync(0xffffffffu, mq[j][cc], off);
-                    if (rg == 0) {
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int jj = h2 + j;
-                            const int q0 = 18 + jj * (jj + 1) / 2;  // row jj of Q
-                            float o[4];
-#pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) o[cc] = cf[8 + jj] * mq[j][cc];
-#pragma unroll
-                            for (int i = 0; i <= jj; ++i) {
-                                const float qc = cf[q0 + i];
-                                const float4 di = delta(i);
-                                o[0] = fmaf(qc, di.x, o[0]); o[1] = fmaf(qc, di.y, o[1]);
-                                o[2] = fmaf(qc, di.z, o[2]); o[3] = fmaf(qc, di.w, o[3]);
-                            }
-                            *reinterpret_cast<float4*>(os + (hh * TP + m * kChunk + jj) * DV + col) =
-                                make_float4(o[0], o[1], o[2], o[3]);
-                        }
+                    for (int cc = 0; cc < 4; ++cc) {
+                        mk[cc] += __shfl_xor_sync(0xffffffffu, mk[cc], off);
+                        mq[cc] += __shfl_xor_sync(0xffffffffu, mq[cc], off);
                     }
                 }
-                // the rank-4 update S~ <- s S~ + sum_j k~_j (f_j delta_j)^T (s = 1 unless the
-                // running scale is folded in)
-                if (cf[33] != 0.f) {
-                    const f2 s2 = f2_pack(cf[32], cf[32]);
+                const TokenScalars st = sc[t * Geo::NHC + hh];
+                const float4 v4 = *reinterpret_cast<const float4*>(vs + (hh * T + t) * DV + col);
+                const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+                const float c1 = c * st.alpha;  // S after this token's decay is c1 * S~
+                const float am = c1 * st.nk, aqs = c1 * st.nq;
+                float d[4], o[4];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    d[cc] = st.beta * fmaf(-am, mk[cc], vv[cc]);
+                    o[cc] = fmaf(aqs, mq[cc], d[cc] * st.kq);
+                }
+                if (spec && rg == 0)
+                    *reinterpret_cast<float4*>(p.spec_delta + (((size_t)tok0 + t) * Hv + h0 + hh) * DV + col) =
+                        make_float4(d[0], d[1], d[2], d[3]);
+                __syncwarp();  // every lane has read v_t of these columns before o_t replaces it
+                if (rg == 0) *reinterpret_cast<float4*>(os + (hh * T + t) * DV + col) = make_float4(o[0], o[1], o[2], o[3]);
+                float f;  // the update's factor on the raw k: nk delta / c, with c the new scale
+                if (c1 < 0x1p-64f) {  // fold the scale into the registers before it underflows
+                    const f2 cc2 = f2_pack(c1, c1);
 #pragma unroll
                     for (int i = 0; i < NPR; ++i)
 #pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) P[i][cc] = f2_mul(P[i][cc], s2);
+                        for (int cc = 0; cc < 4; ++cc) P[i][cc] = f2_mul(P[i][cc], cc2);
+                    c = 1.f;
+                    f = st.nk;
+                } else {
+                    c = c1;
+                    f = __fdividef(st.nk, c1);
                 }
-#pragma unroll 1
-                for (int j = 0; j < kChunk; ++j) {  // rolled: one token's k rows in flight at a time
-                    const float fj = cf[28 + j];
-                    const float* kr = qk0 + j * 2 * DK + DK;
-                    const float4 dj = delta(j);
-                    f2 dn[4];
-                    dn[0] = f2_pack(dj.x * fj, dj.x * fj); dn[1] = f2_pack(dj.y * fj, dj.y * fj);
-                    dn[2] = f2_pack(dj.z * fj, dj.z * fj); dn[3] = f2_pack(dj.w * fj, dj.w * fj);
+                f2 dn[4];
 #pragma unroll
-                    for (int jb = 0; jb < NB; ++jb) {
-                        const int r0 = mt_row<RPL>(jb, rg, 0);
-                        f2 kp[EPB / 2];
-                        if constexpr (EPB == 4) {
-                            const ulonglong2 k2 = *reinterpret_cast<const ulonglong2*>(kr + r0);
-                            kp[0] = k2.x; kp[1] = k2.y;
-                        } else {
-                            kp[0] = *reinterpret_cast<const f2*>(kr + r0);
-                        }
+                for (int cc = 0; cc < 4; ++cc) dn[cc] = f2_pack(d[cc] * f, d[cc] * f);
+                // S~ += k (nk delta / c)^T on this lane's rows
 #pragma unroll
-                        for (int e = 0; e < EPB / 2; ++e) {
-                            f2* pr = P[jb * (EPB / 2) + e];
+                for (int j = 0; j < NB; ++j) {
+                    const int r0 = mt_row<RPL>(j, rg, 0);
+                    f2 kp[EPB / 2];
+                    if constexpr (EPB == 4) {
+                        const ulonglong2 k2 = *reinterpret_cast<const ulonglong2*>(kr + r0);
+                        kp[0] = k2.x; kp[1] = k2.y;
+                    } else {
+                        kp[0] = *reinterpret_cast<const f2*>(kr + r0);
+                    }
 #pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) pr[cc] = f2_fma(kp[e], dn[cc], pr[cc]);
-                        }
+                    for (int e = 0; e < EPB / 2; ++e) {
+                        f2* pr = P[j * (EPB / 2) + e];
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) pr[cc] = f2_fma(kp[e], dn[cc], pr[cc]);
                     }
                 }
-                cfin = cf[34];
             }
-            const float c = cfin;
             // the state back to the pool, scale applied (streaming: nothing here reads it again)
-            if (!spec) {
             float* Sg = p.state_pool + ((size_t)slot * Hv + h0 + hh) * (size_t)(DK * DV) + col;
 #pragma unroll
-            for (int j = 0; j < NB; ++j)
+            for (int j = 0; j < (spec ? 0 : NB); ++j)
 #pragma unroll
                 for (int e = 0; e < EPB; e += 2) {
                     const f2* pr = P[(j * EPB + e) / 2];
@@ -728,7 +515,6 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
                     __stcs(reinterpret_cast<float4*>(Sg + (size_t)mt_row<RPL>(j, rg, e + 1) * DV),
                            make_float4(x0.y * c, x1.y * c, x2.y * c, x3.y * c));
                 }
-            }
         }
         __syncthreads();
 
@@ -745,7 +531,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         ++zphase;
         for (int task = warp; task < ntok * NH; task += Geo::NW) {
             const int t = task / NH, k = task - t * NH;
-            const float4 o = has_cols ? reinterpret_cast<const float4*>(os + (k * TP + t) * DV)[lane]
+            const float4 o = has_cols ? reinterpret_cast<const float4*>(os + (k * T + t) * DV)[lane]
                                       : make_float4(0.f, 0.f, 0.f, 0.f);
             float ss = o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
 #pragma unroll

@@ -18,30 +18,16 @@ def geometry(dk, dv):
     return dict(NWH=nwh, NHC=nhc, NW=nwh * nhc, RPL=dk // 8, NCHC=2 * dk + nhc * dv, TILE=dk * dv * 4)
 
 
-CHUNK_TOKENS = 4   # tokens the recurrence takes together
-COEF_FLOATS = 36   # scalars per (v-head, chunk)
-GRAM_FLOATS = 12   # raw dot products per token
-
-
-def padded(T):
-    return (T + CHUNK_TOKENS - 1) // CHUNK_TOKENS * CHUNK_TOKENS
-
-
 def layout(dk, dv, W, T):
     g = geometry(dk, dv)
-    TP = padded(T)
     rows = g["NHC"] * g["TILE"]
     wts = rows + R16((W - 1 + T) * g["NCHC"] * 2)
     qk = wts + R16(g["NCHC"] * W * 2)
-    vs = qk + TP * 2 * dk * 4
-    zb = vs + TP * g["NHC"] * dv * 4
+    vs = qk + T * 2 * dk * 4
+    zb = vs + T * g["NHC"] * dv * 4
     sc = zb + T * g["NHC"] * dv * 2
-    gram = R16(sc + TP * g["NHC"] * 20)
-    coef = gram + TP * GRAM_FLOATS * 4
-    dsm = coef + g["NHC"] * (TP // CHUNK_TOKENS) * COEF_FLOATS * 4
-    ctl = dsm + g["NW"] * CHUNK_TOKENS * 16 * 4  # per warp: delta of the chunk's tokens on its 16 columns
-    return dict(rows=rows, wts=wts, qk=qk, vs=vs, zb=zb, sc=sc, gram=gram, coef=coef, dsm=dsm, ctl=ctl,
-                total=ctl + 32)
+    ctl = R16(sc + T * g["NHC"] * 20)
+    return dict(rows=rows, wts=wts, qk=qk, vs=vs, zb=zb, sc=sc, ctl=ctl, total=ctl + 32)
 
 
 def heads_per_pass(G, nhc):
@@ -58,7 +44,7 @@ def test_multitoken_kernel_copies_stay_in_bounds(dk, dv, W, T, G):
     C = 2 * Hk * dk + Hv * dv
     g, L = geometry(dk, dv), layout(dk, dv, W, T)
     assert L["total"] <= SMEM_LIMIT
-    for k in ("rows", "wts", "qk", "vs", "zb", "gram", "coef", "dsm", "ctl"):
+    for k in ("rows", "wts", "qk", "vs", "zb"):
         assert L[k] % 16 == 0
     assert (L["ctl"] + 8) % 8 == 0
     NH = heads_per_pass(G, g["NHC"])
@@ -88,19 +74,6 @@ def test_multitoken_kernel_copies_stay_in_bounds(dk, dv, W, T, G):
             c0 = ch[run] + lc - (0, dk, 2 * dk)[run]
             assert (c0 * W + (i * 8 - lc * W)) % 8 == 0 and (c0 + (last - lc) + 1) * W <= C * W
             assert (i * 8 + 8) * 2 <= L["qk"] - L["wts"]
-        # the chunked recurrence: pad rows, Gram rows, per-token scalars, coefficient blocks
-        TP, ntp = padded(T), padded(ntok)
-        assert ntp <= TP
-        assert ntp * 2 * dk * 4 <= L["vs"] - L["qk"]                      # q/k rows incl. the zero pads
-        assert (NH * TP * dv) * 4 <= L["zb"] - L["vs"]                     # v (then o) of the pass's heads
-        for t in range(ntp):                                               # a warp per token: its chunk's k rows
-            c0t = t - t % CHUNK_TOKENS
-            assert (c0t + CHUNK_TOKENS) * 2 * dk * 4 <= L["vs"] - L["qk"]
-            assert (t * GRAM_FLOATS + GRAM_FLOATS - 3) * 4 <= L["coef"] - L["gram"]
-            assert ((t * g["NHC"] + NH) * 20) <= L["gram"] - L["sc"]
-        for k, m in itertools.product(range(NH), range(ntp // CHUNK_TOKENS)):
-            assert ((k * (TP // CHUNK_TOKENS) + m + 1) * COEF_FLOATS) * 4 <= L["dsm"] - L["coef"]
-        assert NH * (ntp // CHUNK_TOKENS) <= 32 * g["NW"] and ntp * NH <= 32 * g["NW"]
         # z rows of the pass and the history write
         assert ntok * NH * dv * 2 <= L["sc"] - L["zb"] and (NH * dv * 2) % 16 == 0
         lc0 = 0 if ps == npass - 1 else 2 * dk

@@ -79,7 +79,11 @@ def run_rounds(wl, rounds=2):
                                     w["dt_bias"], w["norm_w"], o.conv, o.state, o.local, n)
         compare_out(sb.out, sb.out32, r["out"], rows, f"{wl.name} round {rnd} verify")
         np.testing.assert_allclose(sb.k.cpu().numpy(), r["k"], rtol=0, atol=2e-6)
-        np.testing.assert_allclose(sb.alpha.cpu().numpy(), r["alpha"], rtol=2e-6, atol=1e-30)
+        # alpha = exp(g): an error e in g is a relative error e in alpha, and g carries a few
+        # fp32 roundings of its own size, so the bound grows with |g| = -ln(alpha)
+        ga, ra = sb.alpha.cpu().numpy().astype(np.float64), r["alpha"]
+        lim = 1e-6 * (1.0 + np.abs(np.log(np.maximum(ra, 1e-300)))) * ra + 1e-37
+        assert np.all(np.abs(ga - ra) <= lim), f"{wl.name}: recorded decays"
         commit(g, x, sb, n)
         torch.cuda.synchronize()
         assert int(g.err.item()) == 0

@@ -26,10 +26,12 @@ GDN_ERR_CUDA = 5
 GDN_DEVICE_ERR_SLOT_RANGE = 1
 GDN_DEVICE_ERR_TIMEOUT = 2
 GDN_DEVICE_ERR_SEQLEN = 4
+GDN_DEVICE_ERR_BATCH = 8
 
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
            "gdn_decode_workspace_bytes", "gdn_decode_step_varlen", "gdn_decode_step_static_scratch",
            "gdn_decode_static_scratch_bytes", "gdn_spec_verify", "gdn_spec_commit", "gdn_in_proj", "gdn_out_proj",
+           "gdn_decode_step_device_batch",
            "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
 
 
@@ -81,6 +83,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_static_scratch_bytes.restype = ctypes.c_size_t
         L.gdn_spec_verify.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32] + [vp] * 8
         L.gdn_spec_commit.argtypes = [cfgp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_decode_step_device_batch.argtypes = [cfgp, vp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp, vp]
         L.gdn_in_proj.argtypes = [cfgp, i32, i32] + [vp] * 9
         L.gdn_out_proj.argtypes = [cfgp, i32, i32] + [vp] * 6
         L.gdn_check_slots_host.argtypes = [vp, i32, i32]
@@ -89,7 +92,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_abi_version.argtypes = []
         for f in ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
                   "gdn_decode_step_varlen", "gdn_spec_verify", "gdn_spec_commit", "gdn_in_proj", "gdn_out_proj",
-                  "gdn_check_slots_host",
+                  "gdn_decode_step_device_batch", "gdn_check_slots_host",
                   "gdn_abi_version"):
             getattr(L, f).restype = ctypes.c_int32
         _lib = L
@@ -172,6 +175,22 @@ def gdn_decode_step(cfg: GdnConfig, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w
                                  _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
                                  _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"),
                                  _ptr(workspace, _WS, "workspace"), _stream(stream, qkv)), "gdn_decode_step")
+
+
+def gdn_decode_step_device_batch(cfg: GdnConfig, B_dev, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool,
+                                 state_pool, slots, out, out_f32=None, err_flag=None, workspace=None,
+                                 stream=None) -> None:
+    """gdn_decode_step sized for B_max = qkv.shape[0] sequences that runs the first
+    B_dev[0] of them (B_dev: a one-element int32 CUDA tensor read on the device), so a
+    captured CUDA graph serves any batch up to B_max."""
+    B, T = qkv.shape[0], qkv.shape[1]
+    _check(lib().gdn_decode_step_device_batch(
+        ctypes.byref(cfg), _ptr(B_dev, _I32, "B_dev"), B, T, _ptr(qkv, _BF16, "qkv"), _ptr(a, _BF16, "a"),
+        _ptr(b, _BF16, "b"), _ptr(z, _BF16, "z"), _ptr(conv_w, _BF16, "conv_w"), _ptr(A_log, _F32, "A_log"),
+        _ptr(dt_bias, _F32, "dt_bias"), _ptr(norm_w, _BF16, "norm_w"), _ptr(conv_pool, _BF16, "conv_pool"),
+        _ptr(state_pool, _F32, "state_pool"), state_pool.shape[0], _ptr(slots, _I32, "slots"), _ptr(out, _BF16, "out"),
+        _ptr(out_f32, _F32, "out_f32"), _ptr(err_flag, _I32, "err_flag"), _ptr(workspace, _WS, "workspace"),
+        _stream(stream, qkv)), "gdn_decode_step_device_batch")
 
 
 def gdn_decode_step_varlen(cfg: GdnConfig, cu_seqlens, T_max: int, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w,

@@ -181,6 +181,22 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
 
 size_t gdn_decode_workspace_bytes(void) { return 64; }
 
+gdn_status gdn_decode_step_device_batch(const gdn_config* cfg, const int32_t* B_dev, int32_t B_max, int32_t T,
+                                        const uint16_t* qkv, const uint16_t* a, const uint16_t* b, const uint16_t* z,
+                                        const uint16_t* conv_w, const float* A_log, const float* dt_bias,
+                                        const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                                        int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16, float* out_f32,
+                                        int32_t* err_flag, void* workspace, void* stream) {
+    gdn::DecodeArgs d;
+    gdn_status st = check_decode(cfg, B_max, T, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, conv_pool, state_pool,
+                                 pool_slots, slots, out_bf16, out_f32, err_flag, workspace, &d);
+    if (st != GDN_OK || B_max == 0) return st;
+    if (!B_dev) return GDN_ERR_INVALID_ARGUMENT;
+    if (((uintptr_t)B_dev & 3u) != 0) return GDN_ERR_MISALIGNED;
+    d.B_dev = B_dev;
+    return from_cuda(gdn::launch_decode_fused(d, (cudaStream_t)stream));
+}
+
 gdn_status gdn_decode_step_varlen(const gdn_config* cfg, int32_t B, const int32_t* cu_seqlens, int32_t T_max,
                                   int32_t total_tokens, const uint16_t* qkv, const uint16_t* a, const uint16_t* b,
                                   const uint16_t* z, const uint16_t* conv_w, const float* A_log,

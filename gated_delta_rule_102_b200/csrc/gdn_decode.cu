@@ -108,6 +108,8 @@ decode_fused_tma_kernel(const DecodeArgs p) {
     // drains: nothing is read before that grid has completed.
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    // a sequence past the launch's batch count: the whole cluster leaves (seq is the cluster's)
+    if (seq >= launch_batch(p.B_dev, p.B, p.err_flag, blockIdx.x == 0 && tid == 0)) return;
     const int slot = __ldg(p.slots + seq);
     if (slot < 0 || slot >= p.P) {
         if (tid == 0 && rank == 0 && p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);

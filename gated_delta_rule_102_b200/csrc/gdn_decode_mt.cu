@@ -124,7 +124,8 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     // T: the most tokens a sequence has in this launch (it sizes the shared buffers)
     const int T = p.T, W = p.sh.W, C = p.sh.C, Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk;
     const int npass = G / NH, NCH = 2 * DK + NH * DV;
-    const int ngroups = p.B * Hk;
+    const int ngroups_max = p.B * Hk;  // the launch's bound; the batch itself is read after the grid dependency
+    int ngroups = ngroups_max;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float* stage = reinterpret_cast<float*>(smem);
     uint16_t* rows = reinterpret_cast<uint16_t*>(smem + Geo::rows_off());
@@ -228,7 +229,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     // tiles are prefetched into L2 now. The slot read here may be stale: it only steers
     // the hint, and L2 stays coherent with whatever that grid still writes. Nothing is
     // read for use before that grid has completed.
-    if (warp == 0 && blockIdx.x < ngroups) {
+    if (warp == 0 && blockIdx.x < ngroups_max) {
         const int seq0 = (int)blockIdx.x / Hk, h00 = ((int)blockIdx.x - seq0 * Hk) * G;
         const int sl = __ldcg(p.slots + seq0);
         if (sl >= 0 && sl < p.P) {
@@ -239,6 +240,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     }
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    ngroups = launch_batch(p.B_dev, p.B, p.err_flag, blockIdx.x == 0 && tid == 0) * Hk;
     {
         int tok0 = 0, ntok = 0;
         tokens_of(0, tok0, ntok);

@@ -143,7 +143,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
 
     const int Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk, C = p.sh.C, W = p.sh.W;
     const int rank = (int)cluster_ctarank(), cid = blockIdx.x / G;
-    const int ngroups = p.B * Hk;
+    const int ngroups_max = p.B * Hk;  // the launch's bound; the batch itself is read after the grid dependency
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     if (tid == 0) {
@@ -200,7 +200,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     // before that grid has completed.
     if (warp == 0 && lane < 4 * kFixedUnits) {
         const int g = cid + (lane >> 2) * ncl;
-        if (g < ngroups) {
+        if (g < ngroups_max) {
             const int sl = __ldcg(p.slots + g / Hk);
             if (sl >= 0 && sl < p.P) {
                 const char* t = reinterpret_cast<const char*>(
@@ -211,6 +211,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     }
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    const int ngroups = launch_batch(p.B_dev, p.B, p.err_flag, blockIdx.x == 0 && tid == 0) * Hk;
     // lane u of the loader: the slot of fixed unit u, loaded while the cluster barrier completes
     const int slot_fixed =
         warp == 0 && lane < kFixedUnits && cid + lane * ncl < ngroups ? __ldg(p.slots + (cid + lane * ncl) / Hk) : -1;

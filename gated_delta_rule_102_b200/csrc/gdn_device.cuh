@@ -16,6 +16,19 @@ namespace gdn {
 constexpr int GDN_DEVICE_ERR_SLOT_RANGE_BIT = 1;
 constexpr int GDN_DEVICE_ERR_TIMEOUT_BIT = 2;
 constexpr int GDN_DEVICE_ERR_SEQLEN_BIT = 4;
+constexpr int GDN_DEVICE_ERR_BATCH_BIT = 8;
+
+// The batch count of a launch: B_max, or the value a device batch count holds when
+// one is given. A value outside [0, B_max] runs no sequence; `report` threads flag it.
+__device__ __forceinline__ int launch_batch(const int32_t* B_dev, int B_max, int32_t* err_flag, bool report) {
+    if (!B_dev) return B_max;
+    const int b = *reinterpret_cast<const volatile int32_t*>(B_dev);
+    if (b < 0 || b > B_max) {
+        if (report && err_flag) atomicOr(err_flag, GDN_DEVICE_ERR_BATCH_BIT);
+        return 0;
+    }
+    return b;
+}
 
 // Longest conv supported (taps) and most tokens per launch.
 constexpr int kMaxConvWidth = 8;

@@ -46,6 +46,9 @@ struct DecodeArgs {
     float* spec_k;
     float* spec_delta;
     float* spec_alpha;
+    // nullable: device int32 holding this launch's batch count (0..B); B then only
+    // bounds it and sizes the launch, so one captured launch serves any smaller batch
+    const int32_t* B_dev;
 };
 
 // Commit of the accepted prefix of a speculative verify call.

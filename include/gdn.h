@@ -67,6 +67,7 @@ typedef enum {
 #define GDN_DEVICE_ERR_SLOT_RANGE 1 /* a sequence's slot is outside [0, pool_slots) */
 #define GDN_DEVICE_ERR_TIMEOUT 2    /* a bounded wait inside the kernel ran out */
 #define GDN_DEVICE_ERR_SEQLEN 4     /* a token count (varlen) or accepted count (spec commit) out of range */
+#define GDN_DEVICE_ERR_BATCH 8      /* gdn_decode_step_device_batch: *B_dev outside [0, B_max] */
 
 typedef struct {
     int32_t num_k_heads; /* Hk */
@@ -159,6 +160,30 @@ gdn_status gdn_decode_step(const gdn_config* cfg, int32_t B, int32_t T, const ui
 
 /* Bytes of the optional workspace of gdn_decode_step (a multiple of 16). */
 size_t gdn_decode_workspace_bytes(void);
+
+/*
+ * gdn_decode_step with the batch count in DEVICE memory, for CUDA-graph replay. The
+ * launch is sized for B_max sequences; each kernel reads *B_dev (int32, 4-byte
+ * aligned) after the work before it in the stream has completed and processes
+ * sequences 0 .. *B_dev - 1 only, exactly as gdn_decode_step with B = *B_dev would
+ * (the results may differ from that call in the last bits where B_max selects
+ * another kernel than B would). Sequences *B_dev .. B_max - 1: pools and outputs
+ * untouched. A captured call therefore serves every batch up to B_max: before each
+ * replay write the count to *B_dev and the inputs and slots of that many sequences
+ * to the captured buffers (the counterpart of the layer graph hooks on the page
+ * "metrale_model_arch/glm5next_dsa/layer.rs", which read the replayed step's
+ * positions from device memory). All other arguments are those of gdn_decode_step
+ * with B = B_max (tensors sized for B_max). A value of *B_dev outside [0, B_max]
+ * runs no sequence and ORs GDN_DEVICE_ERR_BATCH into *err_flag. The host-side
+ * kernel choice and device queries happen on the first call per shape: make it
+ * before the capture.
+ */
+gdn_status gdn_decode_step_device_batch(const gdn_config* cfg, const int32_t* B_dev, int32_t B_max, int32_t T,
+                                        const uint16_t* qkv, const uint16_t* a, const uint16_t* b, const uint16_t* z,
+                                        const uint16_t* conv_w, const float* A_log, const float* dt_bias,
+                                        const uint16_t* norm_w, uint16_t* conv_pool, float* state_pool,
+                                        int32_t pool_slots, const int32_t* slots, uint16_t* out_bf16, float* out_f32,
+                                        int32_t* err_flag, void* workspace, void* stream);
 
 /*
  * The fused decode step for a batch whose sequences bring different numbers of tokens
@@ -316,7 +341,7 @@ gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t po
 const char* gdn_status_string(gdn_status status);
 
 /* ABI version of this header: (major << 16) | minor. */
-#define GDN_ABI_VERSION ((1 << 16) | 2)
+#define GDN_ABI_VERSION ((1 << 16) | 3)
 int32_t gdn_abi_version(void);
 
 #ifdef __cplusplus

@@ -53,7 +53,7 @@ def test_status_codes_match_header(L):
         m = re.search(rf"\b{name} = (\d+)", HEADER)
         assert m and int(m.group(1)) == getattr(gdn, name)
         assert gdn.status_string(getattr(gdn, name))
-    for name in ("GDN_DEVICE_ERR_SLOT_RANGE", "GDN_DEVICE_ERR_TIMEOUT", "GDN_DEVICE_ERR_SEQLEN"):
+    for name in ("GDN_DEVICE_ERR_SLOT_RANGE", "GDN_DEVICE_ERR_TIMEOUT", "GDN_DEVICE_ERR_SEQLEN", "GDN_DEVICE_ERR_BATCH"):
         m = re.search(rf"#define {name} (\d+)", HEADER)
         assert int(m.group(1)) == getattr(gdn, name)
 
@@ -187,6 +187,24 @@ def test_spec_entry_points_check_every_argument_before_touching_the_device(L):
         assert spec_commit(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
         ptrs[i] = FAKE_ODD
         assert spec_commit(L, cfg, ptrs=ptrs) == gdn.GDN_ERR_MISALIGNED, i
+
+
+def test_device_batch_entry_point_checks_arguments_on_the_host(L):
+    cfg = good_cfg()
+
+    def call(bdev=FAKE, B=4, T=1, ptrs=None, ws=None):
+        p = [FAKE] * 10 if ptrs is None else ptrs
+        return L.gdn_decode_step_device_batch(ctypes.byref(cfg), bdev, B, T, *p, 8, FAKE, FAKE, None, None, ws, None)
+    assert call(bdev=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert call(bdev=ctypes.c_void_p((1 << 20) + 2)) == gdn.GDN_ERR_MISALIGNED
+    assert call(bdev=ctypes.c_void_p((1 << 20) + 4)) != gdn.GDN_ERR_MISALIGNED  # 4-byte aligned is enough
+    assert call(B=0, bdev=None, ptrs=[None] * 10) == gdn.GDN_OK           # B_max = 0: nothing to launch
+    assert call(T=17) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(ws=FAKE_ODD) == gdn.GDN_ERR_MISALIGNED
+    for i in range(10):
+        ptrs = [FAKE] * 10
+        ptrs[i] = None
+        assert call(ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
 
 
 def test_empty_batch_is_a_no_op(L):

@@ -98,27 +98,8 @@ gdn_status check_proj_sizes(int32_t hidden, int32_t rows) {
     return GDN_OK;
 }
 
-// The SM count of the current device, queried once per device.
-gdn_status sm_count(int* out) {
-    static std::atomic<int> cache[gdn::kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-    if (dev < 0 || dev >= gdn::kMaxDevices) return GDN_ERR_UNSUPPORTED;
-    int n = cache[dev].load(std::memory_order_relaxed);
-    if (n <= 0) {
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            return GDN_ERR_CUDA;
-        cache[dev].store(n, std::memory_order_relaxed);
-    }
-    *out = n;
-    return GDN_OK;
-}
-
 gdn_status launch_proj(gdn::ProjArgs& p, cudaStream_t stream) {
-    int sms = 0;
-    gdn_status st = sm_count(&sms);
-    if (st != GDN_OK) return st;
-    p.slices = gdn::proj_slices(p.N, p.K, sms);
+    if (gdn::proj_slices(p.N, p.K, p.R, &p.slices) != cudaSuccess) return GDN_ERR_CUDA;
     return from_cuda(gdn::launch_proj_gemm(p, stream));
 }
 

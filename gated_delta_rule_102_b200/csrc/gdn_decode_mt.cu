@@ -99,9 +99,10 @@ struct MtGeo {
     static __host__ __device__ int ctl_off(int W, int T) {
         return (sc_off(W, T) + T * NHC * (int)sizeof(TokenScalars) + 15) / 16 * 16;
     }
-    static __host__ __device__ int total(int W, int T) { return ctl_off(W, T) + 32; }
+    static __host__ __device__ int total(int W, int T) { return ctl_off(W, T) + 48; }
     // the control block: the stage's slot, the abort flag, the stage and z barriers,
-    // the stage's first packed row and token count
+    // the stage's first packed row and token count, and the stage and z phases a CTA
+    // that gives up waits for before it leaves
 };
 
 template <int K>
@@ -125,7 +126,6 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     const int T = p.T, W = p.sh.W, C = p.sh.C, Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk;
     const int npass = G / NH, NCH = 2 * DK + NH * DV;
     const int ngroups_max = p.B * Hk;  // the launch's bound; the batch itself is read after the grid dependency
-    int ngroups = ngroups_max;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float* stage = reinterpret_cast<float*>(smem);
     uint16_t* rows = reinterpret_cast<uint16_t*>(smem + Geo::rows_off());
@@ -141,6 +141,33 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
     uint64_t* zbar = full + 1;
     volatile int* stage_tok0 = reinterpret_cast<volatile int*>(zbar + 1);  // the stage's first packed row
     volatile int* stage_ntok = stage_tok0 + 1;                             // and its token count
+    volatile int* drain = stage_ntok + 1;  // [2]: stage phase, z phase still in flight (-1: none)
+
+    if (tid == 0) {
+        mbar_init(full, Geo::NT + 1);  // every thread's copies, and the tile bytes
+        mbar_init(zbar, Geo::NT);      // every thread's copies
+        *abort_flag = 0;
+        drain[0] = drain[1] = -1;
+        mbar_init_fence();
+    }
+    __syncthreads();
+    // With programmatic dependent launch this grid may start while the previous one
+    // drains (on the SMs its early finishers have left), so the first pass's state
+    // tiles are prefetched into L2 now. The slot read here may be stale: it only steers
+    // the hint, and L2 stays coherent with whatever that grid still writes. Nothing is
+    // read for use before that grid has completed.
+    if (warp == 0 && blockIdx.x < ngroups_max) {
+        const int seq0 = (int)blockIdx.x / Hk, h00 = ((int)blockIdx.x - seq0 * Hk) * G;
+        const int sl = __ldcg(p.slots + seq0);
+        if (sl >= 0 && sl < p.P) {
+            const char* t0 = reinterpret_cast<const char*>(p.state_pool + ((size_t)sl * Hv + h00) * (size_t)(DK * DV));
+            for (int c = lane * kMtChunk; c < NH * Geo::TILE; c += 32 * kMtChunk)
+                bulk_prefetch_l2(t0 + c, (uint32_t)min(kMtChunk, NH * Geo::TILE - c));
+        }
+    }
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    const int ngroups = launch_batch(p.B_dev, p.B, p.err_flag, blockIdx.x == 0 && tid == 0) * Hk;
 
     auto item_group = [&](int u) { return (int)blockIdx.x + (u / npass) * (int)gridDim.x; };
     // Every thread: the copies of pass u into the stage (or, past the last pass,
@@ -217,30 +244,6 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         const int group = item_group(u);
         return group < ngroups ? __ldg(p.slots + group / Hk) : -1;
     };
-    if (tid == 0) {
-        mbar_init(full, Geo::NT + 1);  // every thread's copies, and the tile bytes
-        mbar_init(zbar, Geo::NT);      // every thread's copies
-        *abort_flag = 0;
-        mbar_init_fence();
-    }
-    __syncthreads();
-    // With programmatic dependent launch this grid may start while the previous one
-    // drains (on the SMs its early finishers have left), so the first pass's state
-    // tiles are prefetched into L2 now. The slot read here may be stale: it only steers
-    // the hint, and L2 stays coherent with whatever that grid still writes. Nothing is
-    // read for use before that grid has completed.
-    if (warp == 0 && blockIdx.x < ngroups_max) {
-        const int seq0 = (int)blockIdx.x / Hk, h00 = ((int)blockIdx.x - seq0 * Hk) * G;
-        const int sl = __ldcg(p.slots + seq0);
-        if (sl >= 0 && sl < p.P) {
-            const char* t0 = reinterpret_cast<const char*>(p.state_pool + ((size_t)sl * Hv + h00) * (size_t)(DK * DV));
-            for (int c = lane * kMtChunk; c < NH * Geo::TILE; c += 32 * kMtChunk)
-                bulk_prefetch_l2(t0 + c, (uint32_t)min(kMtChunk, NH * Geo::TILE - c));
-        }
-    }
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-    ngroups = launch_batch(p.B_dev, p.B, p.err_flag, blockIdx.x == 0 && tid == 0) * Hk;
     {
         int tok0 = 0, ntok = 0;
         tokens_of(0, tok0, ntok);
@@ -260,8 +263,8 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         if (!__syncthreads_and(ok)) {
             if (tid == 0) {
                 *abort_flag = 1;
+                drain[0] = u & 1;  // pass u's copies were issued and never waited for
                 if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_TIMEOUT_BIT);
-                for (int i = 0; i < 1024; ++i) __nanosleep(64);  // copies in flight land before the CTA leaves
             }
             break;
         }
@@ -527,6 +530,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         if (!mbar_wait_deadline(zbar, (uint32_t)(zphase & 1), kWaitTimeoutNs, [&] { return *abort_flag != 0; })) {
             if (lane == 0) {
                 *abort_flag = 1;
+                drain[1] = zphase & 1;  // this pass's z copies were issued and never waited for
                 if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_TIMEOUT_BIT);
             }
         }
@@ -553,8 +557,15 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
             if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + base) = make_float4(y0, y1, y2, y3);
         }
     }
-    if (*abort_flag && tid == 0) {  // a wait gave up: copies still in flight land before the CTA leaves
-        for (int i = 0; i < 1024; ++i) __nanosleep(64);
+    // A wait gave up: the copies this CTA still has in flight land (or a further bounded
+    // wait runs out) before it leaves. Each barrier phase counts every copy issued into
+    // it, and a phase is armed only once the one before it has been waited for, so at
+    // most the phase whose wait gave up is outstanding on each barrier. (When the z wait
+    // gives up first, the next pass's stage wait then gives up at once and records its
+    // phase; a stage phase never armed is never recorded.)
+    if (*abort_flag && tid == 0) {
+        if (drain[0] >= 0) mbar_wait_bounded(full, (uint32_t)drain[0]);
+        if (drain[1] >= 0) mbar_wait_bounded(zbar, (uint32_t)drain[1]);
     }
 }
 

@@ -123,7 +123,9 @@ struct ProjArgs {
     float* out_f32;  // nullable: [R][N] fp32 before rounding
     int32_t* err_flag;
 };
-int proj_slices(int N, int K, int num_sms);
+// K-slices per weight tile (the cluster size) for a launch; the first call per shape
+// queries the device (sets the kernel attribute, occupancy), later ones hit a cache.
+cudaError_t proj_slices(int N, int K, int R, int* slices);
 int proj_smem_bytes(int R);
 cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream);
 

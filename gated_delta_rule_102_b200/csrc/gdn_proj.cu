@@ -316,12 +316,67 @@ bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows)
 
 }  // namespace
 
-int proj_slices(int N, int K, int num_sms) {
+// Co-resident clusters of `s` CTAs for a launch of R token rows, queried once per
+// (device, s, padded rows) and cached.
+cudaError_t proj_cluster_capacity(int s, int R, int* out) {
+    static std::mutex mu;
+    struct Entry { int dev, s, rp, cap; };
+    static Entry cache[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int rp = rows_padded(R);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (cache[i].dev == dev && cache[i].s == s && cache[i].rp == rp) {
+            *out = cache[i].cap;
+            return cudaSuccess;
+        }
+    if ((e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem_bytes(rows_padded(kProjMaxRows)))) != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)s);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem_bytes(rp);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)s;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int cap = 0;
+    if ((e = cudaOccupancyMaxActiveClusters(&cap, proj_gemm_kernel, &cfg)) != cudaSuccess) return e;
+    if (n < 256) cache[n++] = {dev, s, rp, cap};
+    *out = cap;
+    return cudaSuccess;
+}
+
+// K-slices per weight tile: the most (up to 8, at least two K blocks each) for which
+// every tile's cluster is co-resident, so the launch is one wave; a tile that had to
+// wait for a second wave would double the time of this bandwidth-bound GEMM.
+cudaError_t proj_slices(int N, int K, int R, int* slices) {
     const int tiles = (N + kTileN - 1) / kTileN, nkb = (K + kTileK - 1) / kTileK;
-    int s = (2 * num_sms + tiles / 2) / tiles;  // about two CTAs per SM
-    if (s > kMaxSlices) s = kMaxSlices;
-    if (s > nkb) s = nkb;
-    return s < 1 ? 1 : s;
+#ifdef GDN_PROJ_SLICES_OVERRIDE
+    {  // build-time tuning override, used when the shape allows it
+        const int s = GDN_PROJ_SLICES_OVERRIDE;
+        if (s >= 1 && s <= kMaxSlices && s <= nkb) {
+            *slices = s;
+            return cudaSuccess;
+        }
+    }
+#endif
+    int best = 1;
+    for (int s = 2; s <= kMaxSlices && 2 * s <= nkb; ++s) {
+        int cap = 0;
+        cudaError_t e = proj_cluster_capacity(s, R, &cap);
+        if (e != cudaSuccess) return e;
+        if (cap >= tiles) best = s;
+    }
+    *slices = best;
+    return cudaSuccess;
 }
 
 int proj_smem_bytes(int R) { return smem_bytes(rows_padded(R)); }
@@ -332,13 +387,6 @@ cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
     if (!make_map(&mw, a.w, a.N, a.K, kTileN) || !make_map(&mx, a.x, a.R, a.K, rows_padded(a.R)))
         return cudaErrorInvalidValue;
     const int smem = smem_bytes(rows_padded(a.R));
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        smem_bytes(rows_padded(kProjMaxRows)));
-    });
-    if (attr_err != cudaSuccess) return attr_err;
     const int tiles = (a.N + kTileN - 1) / kTileN;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tiles * a.slices));

@@ -15,7 +15,7 @@
 //
 // One CTA per (sequence, v-head). A thread holds RPT consecutive rows x 4 columns of
 // the dk x dv tile (one float4 per row), the TPR threads of a row segment covering it
-// with whole sectors. The CTA of the first v-head of a k-head group also rolls that
+// with whole sectors; two CTAs share an SM. The CTA of the first v-head of a k-head group also rolls that
 // k-head's q and k channels; every CTA rolls its own v-head's v channels.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -26,10 +26,22 @@
 namespace gdn {
 namespace {
 
+// A thread holds RPT rows x 4 columns (about 32 values): up to 512 threads per tile and
+// two CTAs per SM, so one CTA's loads overlap the other's update and stores.
 template <int DK, int DV>
-__global__ void __launch_bounds__(Tile<DK, DV>::NT)
+struct CommitGeo {
+    static constexpr int TPR = DV / 4;  // threads per row segment
+    static constexpr int NT0 = DK * DV / 32;
+    static constexpr int NT = NT0 < 32 ? 32 : (NT0 > 512 ? 512 : NT0);
+    static constexpr int RPP = NT / TPR;
+    static constexpr int RPT = DK / RPP;
+    static_assert(NT % TPR == 0 && DK % RPP == 0 && RPT >= 1, "commit geometry");
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(CommitGeo<DK, DV>::NT, 2)
 spec_commit_kernel(const SpecCommitArgs p) {
-    using Geo = Tile<DK, DV>;
+    using Geo = CommitGeo<DK, DV>;
     constexpr int RPT = Geo::RPT, NT = Geo::NT;
     extern __shared__ __align__(16) float sm[];  // [T][DK] keys, [T][DV] writes, [T] decays
     const int Hk = p.sh.Hk, Hv = p.sh.Hv, G = Hv / Hk, W = p.sh.W, C = p.sh.C, T = p.T;
@@ -70,6 +82,25 @@ spec_commit_kernel(const SpecCommitArgs p) {
     }
     if (tid < n) as[tid] = p.spec_alpha[((size_t)seq * T + tid) * Hv + h];
 
+    __syncthreads();
+
+    // S <- alpha_t S + k_t delta_t^T for the accepted tokens, in order
+    for (int t = 0; t < n; ++t) {
+        const float al = as[t];
+        const float4 d = reinterpret_cast<const float4*>(ds + t * DV)[cg];
+        const float* kr = ks + t * DK + row0;
+#pragma unroll
+        for (int s = 0; s < RPT; ++s) {
+            const float kv = kr[s];
+            S[s].x = fmaf(al, S[s].x, kv * d.x);
+            S[s].y = fmaf(al, S[s].y, kv * d.y);
+            S[s].z = fmaf(al, S[s].z, kv * d.z);
+            S[s].w = fmaf(al, S[s].w, kv * d.w);
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < RPT; ++s) __stcs(Sg + (size_t)s * (DV / 4), S[s]);
+
     // the conv history of this CTA's channels: v-head h's v channels, and the k-head's
     // q and k channels in the group's first CTA. New row r is element n + r of
     // [history rows 0..W-2, tokens 0..T-1]; every value is read before any is written.
@@ -91,24 +122,6 @@ spec_commit_kernel(const SpecCommitArgs p) {
                 if (r < W - 1) hist[(size_t)r * C + ch] = nv[r];
         }
     }
-    __syncthreads();
-
-    // S <- alpha_t S + k_t delta_t^T for the accepted tokens, in order
-    for (int t = 0; t < n; ++t) {
-        const float al = as[t];
-        const float4 d = reinterpret_cast<const float4*>(ds + t * DV)[cg];
-        const float* kr = ks + t * DK + row0;
-#pragma unroll
-        for (int s = 0; s < RPT; ++s) {
-            const float kv = kr[s];
-            S[s].x = fmaf(al, S[s].x, kv * d.x);
-            S[s].y = fmaf(al, S[s].y, kv * d.y);
-            S[s].z = fmaf(al, S[s].z, kv * d.z);
-            S[s].w = fmaf(al, S[s].w, kv * d.w);
-        }
-    }
-#pragma unroll
-    for (int s = 0; s < RPT; ++s) __stcs(Sg + (size_t)s * (DV / 4), S[s]);
 }
 
 template <int DK, int DV>
@@ -117,7 +130,7 @@ cudaError_t launch_commit(const SpecCommitArgs& a, cudaStream_t stream) {
     const size_t smem = (size_t)a.T * (DK + DV + 1) * sizeof(float);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.B * a.sh.Hv));
-    cfg.blockDim = dim3(Tile<DK, DV>::NT);
+    cfg.blockDim = dim3(CommitGeo<DK, DV>::NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

@@ -235,6 +235,8 @@ gdn_status gdn_decode_step_varlen(const gdn_config* cfg, int32_t B, const int32_
  * decode step's output y (already normalised and gated by SiLU(z)):
  *   y     [rows][Hv*dv] bf16, w_out [hidden][Hv*dv] bf16, out [rows][hidden] bf16
  *   out_f32 [rows][hidden] fp32, nullable
+ * The first call per shape queries the device (kernel attribute, co-resident clusters,
+ * which set how K is split); make it before capturing the call into a CUDA graph.
  * Errors: rows > 256 or hidden not a multiple of 8 give GDN_ERR_UNSUPPORTED; other
  * checks as above, all before anything is enqueued. Every wait inside the kernel is
  * bounded; on expiry GDN_DEVICE_ERR_TIMEOUT is OR-ed into *err_flag (nullable) and

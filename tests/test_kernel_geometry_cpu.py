@@ -27,7 +27,7 @@ def layout(dk, dv, W, T):
     zb = vs + T * g["NHC"] * dv * 4
     sc = zb + T * g["NHC"] * dv * 2
     ctl = R16(sc + T * g["NHC"] * 20)
-    return dict(rows=rows, wts=wts, qk=qk, vs=vs, zb=zb, sc=sc, ctl=ctl, total=ctl + 32)
+    return dict(rows=rows, wts=wts, qk=qk, vs=vs, zb=zb, sc=sc, ctl=ctl, total=ctl + 48)
 
 
 def heads_per_pass(G, nhc):

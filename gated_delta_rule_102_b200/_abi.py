@@ -31,7 +31,7 @@ GDN_DEVICE_ERR_BATCH = 8
 EXPORTS = ("gdn_conv_update", "gdn_recurrent_step", "gdn_gated_rmsnorm", "gdn_decode_step",
            "gdn_decode_workspace_bytes", "gdn_decode_step_varlen", "gdn_decode_step_static_scratch",
            "gdn_decode_static_scratch_bytes", "gdn_spec_verify", "gdn_spec_commit", "gdn_in_proj", "gdn_out_proj",
-           "gdn_decode_step_device_batch",
+           "gdn_decode_step_device_batch", "gdn_selftest_wait_timeout",
            "gdn_check_slots_host", "gdn_status_string", "gdn_abi_version")
 
 
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_spec_verify.argtypes = [cfgp, i32, i32] + [vp] * 10 + [i32] + [vp] * 8
         L.gdn_spec_commit.argtypes = [cfgp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
         L.gdn_decode_step_device_batch.argtypes = [cfgp, vp, i32, i32] + [vp] * 10 + [i32, vp, vp, vp, vp, vp, vp]
+        L.gdn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp, vp]
+        L.gdn_selftest_wait_timeout.restype = ctypes.c_int32
         L.gdn_in_proj.argtypes = [cfgp, i32, i32] + [vp] * 9
         L.gdn_out_proj.argtypes = [cfgp, i32, i32] + [vp] * 6
         L.gdn_check_slots_host.argtypes = [vp, i32, i32]
@@ -279,6 +281,14 @@ def decode_workspace_bytes() -> int:
 def decode_workspace(device) -> torch.Tensor:
     """A zeroed workspace for gdn_decode_step on `device` (keep one per stream)."""
     return torch.zeros(decode_workspace_bytes() // 4, dtype=torch.int32, device=device)
+
+
+def gdn_selftest_wait_timeout(limit_cycles: int, err_flag, cycles=None, stream=None) -> None:
+    """Run the bounded-wait self-test: a wait that nothing completes must give up after
+    about limit_cycles SM cycles and set GDN_DEVICE_ERR_TIMEOUT in err_flag."""
+    _check(lib().gdn_selftest_wait_timeout(int(limit_cycles), _ptr(err_flag, _I32, "err_flag"),
+                                           _ptr(cycles, (torch.int64,), "cycles"), _stream(stream, err_flag)),
+           "gdn_selftest_wait_timeout")
 
 
 def gdn_check_slots_host(slots, pool_slots: int) -> int:

@@ -349,6 +349,13 @@ gdn_status gdn_decode_step_static_scratch(const gdn_config* cfg, int32_t B, int3
 
 size_t gdn_decode_static_scratch_bytes(void) { return kStaticScratchBytes; }
 
+gdn_status gdn_selftest_wait_timeout(uint64_t limit_cycles, int32_t* err_flag, uint64_t* cycles, void* stream) {
+    if (!err_flag || limit_cycles == 0 || limit_cycles > (1ull << 40)) return GDN_ERR_INVALID_ARGUMENT;
+    if (((uintptr_t)err_flag & 3u) != 0 || ((uintptr_t)cycles & 7u) != 0) return GDN_ERR_MISALIGNED;
+    return from_cuda(gdn::launch_wait_selftest(limit_cycles, err_flag, reinterpret_cast<unsigned long long*>(cycles),
+                                               (cudaStream_t)stream));
+}
+
 gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t pool_slots) {
     if (B < 0 || pool_slots < 0 || (B > 0 && !slots_host)) return GDN_ERR_INVALID_ARGUMENT;
     std::vector<unsigned char> seen((size_t)pool_slots, 0);

@@ -259,7 +259,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         if (group >= ngroups) break;
         const int pass = u % npass;
         const int seq = group / Hk, hk = group - seq * Hk, h0 = hk * G + pass * NH;
-        bool ok = mbar_wait_deadline(full, (uint32_t)(u & 1), kWaitTimeoutNs, [&] { return *abort_flag != 0; });
+        bool ok = mbar_wait_deadline(full, (uint32_t)(u & 1), kWaitTimeoutCycles, [&] { return *abort_flag != 0; });
         if (!__syncthreads_and(ok)) {
             if (tid == 0) {
                 *abort_flag = 1;
@@ -527,7 +527,7 @@ decode_mt_kernel(const DecodeArgs p, const int NH) {
         // four columns per lane (DV <= 128)
         const bool has_cols = 4 * lane < DV;
         const uint2 nw = has_cols ? __ldg(reinterpret_cast<const uint2*>(p.norm_w) + lane) : make_uint2(0u, 0u);
-        if (!mbar_wait_deadline(zbar, (uint32_t)(zphase & 1), kWaitTimeoutNs, [&] { return *abort_flag != 0; })) {
+        if (!mbar_wait_deadline(zbar, (uint32_t)(zphase & 1), kWaitTimeoutCycles, [&] { return *abort_flag != 0; })) {
             if (lane == 0) {
                 *abort_flag = 1;
                 drain[1] = zphase & 1;  // this pass's z copies were issued and never waited for

@@ -30,7 +30,7 @@
 // state is read once and written once, and HBM sees a steady stream of TMA loads and
 // row stores instead of alternating load, compute and store phases.
 //
-// Every wait is an mbarrier poll bounded by the global timer. When one expires the
+// Every wait is an mbarrier poll bounded by the SM cycle counter. When one expires the
 // CTA sets the timeout bit of the error flag, all roles leave their loops, the loader
 // gives its copies in flight time to land, and the CTA leaves through the final
 // cluster barrier.
@@ -166,7 +166,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         }
     };
     auto wait = [&](uint64_t* bar, uint32_t parity) {
-        return mbar_wait_deadline(bar, parity, kWaitTimeoutNs, [&] { return *abort_flag != 0; });
+        return mbar_wait_deadline(bar, parity, kWaitTimeoutCycles, [&] { return *abort_flag != 0; });
     };
     auto slot_ok = [&](int s) { return s >= 0 && s < p.P; };
 

@@ -275,11 +275,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
-    return t;
-}
 // Like mbar_try_wait, suspending for at most about `hint_ns` while the phase is open.
 __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
     uint32_t ok;
@@ -290,24 +285,31 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
         : "memory");
     return ok != 0;
 }
-// Bound on every wait inside the kernels, in nanoseconds of the global timer.
-constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
-// Waits for phase `parity` of the barrier; gives up after about `timeout_ns` and
-// returns false. `give_up` is polled now and then so a CTA can stop waiting early.
+// Bound on every wait inside the kernels, in cycles of the SM's own clock (a second at
+// 2 GHz, longer at lower clocks). The SM cycle counter only moves forward while the
+// warp waits; the global timer is not used for this, since it may be adjusted while a
+// kernel runs and a jump would end a healthy wait (an unsigned difference across a
+// backward step reads as an enormous elapsed time).
+constexpr uint64_t kWaitTimeoutCycles = 2000000000ull;
+// Waits for phase `parity` of the barrier; gives up after about `timeout_cycles` SM
+// cycles and returns false. `give_up` is polled now and then so a CTA can stop waiting
+// early.
 template <typename GiveUp>
-__device__ __forceinline__ bool mbar_wait_deadline(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, GiveUp give_up) {
+__device__ __forceinline__ bool mbar_wait_deadline(uint64_t* bar, uint32_t parity, uint64_t timeout_cycles,
+                                                   GiveUp give_up) {
     if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = clock64();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
         if ((i & 15) == 0) {
             if (give_up()) return false;
-            if (globaltimer_ns() - t0 > timeout_ns) return false;
+            if ((uint64_t)clock64() - t0 > timeout_cycles) return false;
         }
     }
 }
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = kWaitTimeoutNs) {
-    return mbar_wait_deadline(bar, parity, timeout_ns, [] { return false; });
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t timeout_cycles = kWaitTimeoutCycles) {
+    return mbar_wait_deadline(bar, parity, timeout_cycles, [] { return false; });
 }
 // One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into
 // this CTA's shared memory, counted on `bar`.

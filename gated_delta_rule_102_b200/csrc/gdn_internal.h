@@ -145,6 +145,8 @@ cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream);
 bool multitoken_supported(const DecodeArgs& a);
 cudaError_t launch_decode_multitoken(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_spec_commit(const SpecCommitArgs& a, cudaStream_t stream);
+cudaError_t launch_wait_selftest(uint64_t limit_cycles, int32_t* err_flag, unsigned long long* cycles,
+                                 cudaStream_t stream);
 cudaError_t launch_conv_update(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_recurrent(const RecurrentArgs& a, cudaStream_t stream);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);

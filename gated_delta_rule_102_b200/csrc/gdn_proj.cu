@@ -21,7 +21,7 @@
 //    32w..32w+31, i.e. weight rows) into shared memory; the cluster then sums its S
 //    partial tiles over distributed shared memory in rank order (deterministic), CTA
 //    rank q taking a band of rows, and stores bf16 (and optionally fp32) outputs.
-// Every mbarrier wait is bounded by the global timer; on expiry the CTA records
+// Every mbarrier wait is bounded by the SM cycle counter; on expiry the CTA records
 // GDN_DEVICE_ERR_TIMEOUT, stops issuing work, lets what it issued complete, frees
 // its TMEM and leaves through the cluster barriers.
 #include <cuda.h>
@@ -174,7 +174,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
         if (p.err_flag) atomicOr(p.err_flag, GDN_DEVICE_ERR_TIMEOUT_BIT);
     };
     auto wait = [&](uint64_t* bar, uint32_t parity) {
-        return mbar_wait_deadline(bar, parity, kWaitTimeoutNs, [&] { return *abort_flag != 0; });
+        return mbar_wait_deadline(bar, parity, kWaitTimeoutCycles, [&] { return *abort_flag != 0; });
     };
 
     int issued = 0;  // stages the loader armed (thread 0)

@@ -40,8 +40,9 @@
  *   library never clears it). Duplicate slots are not detected on the device and
  *   give undefined results; gdn_check_slots_host() checks a host copy. Every wait
  *   inside a kernel is bounded: a CTA whose staged state copy has not landed after
- *   more than a second gives up, ORs GDN_DEVICE_ERR_TIMEOUT into *err_flag and writes
- *   neither that state tile nor its outputs (their values are then unspecified).
+ *   2e9 cycles of its SM's clock (a second at the top clock) gives up, ORs
+ *   GDN_DEVICE_ERR_TIMEOUT into *err_flag and writes neither that state tile nor its
+ *   outputs (their values are then unspecified).
  *   A failed launch returns GDN_ERR_CUDA.
  */
 #ifndef GDN_H_
@@ -333,6 +334,15 @@ gdn_status gdn_decode_step_static_scratch(const gdn_config* cfg, int32_t B, int3
 size_t gdn_decode_static_scratch_bytes(void);
 
 /*
+ * Self-test of the bounded waits inside every kernel of this library (the pages have no
+ * counterpart): one GPU thread waits on a barrier phase that nothing completes, gives up
+ * after limit_cycles cycles of its SM's clock (1 .. 2^40) and ORs GDN_DEVICE_ERR_TIMEOUT
+ * into *err_flag (device int32, required). `cycles` (nullable, device uint64) receives
+ * the cycles the wait took. Nothing else is touched; the context stays usable.
+ */
+gdn_status gdn_selftest_wait_timeout(uint64_t limit_cycles, int32_t* err_flag, uint64_t* cycles, void* stream);
+
+/*
  * Host-side check of a HOST copy of slots[]: GDN_OK when all B values are distinct
  * and in [0, pool_slots), GDN_ERR_SLOT_RANGE otherwise, GDN_ERR_INVALID_ARGUMENT for
  * a null pointer or negative size. Touches no device.
@@ -343,7 +353,7 @@ gdn_status gdn_check_slots_host(const int32_t* slots_host, int32_t B, int32_t po
 const char* gdn_status_string(gdn_status status);
 
 /* ABI version of this header: (major << 16) | minor. */
-#define GDN_ABI_VERSION ((1 << 16) | 3)
+#define GDN_ABI_VERSION ((1 << 16) | 4)
 int32_t gdn_abi_version(void);
 
 #ifdef __cplusplus

@@ -207,6 +207,14 @@ def test_device_batch_entry_point_checks_arguments_on_the_host(L):
         assert call(ptrs=ptrs) == gdn.GDN_ERR_INVALID_ARGUMENT, i
 
 
+def test_selftest_checks_arguments_on_the_host(L):
+    assert L.gdn_selftest_wait_timeout(1000, None, None, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert L.gdn_selftest_wait_timeout(0, FAKE, None, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert L.gdn_selftest_wait_timeout(1 << 41, FAKE, None, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert L.gdn_selftest_wait_timeout(1000, ctypes.c_void_p((1 << 20) + 2), None, None) == gdn.GDN_ERR_MISALIGNED
+    assert L.gdn_selftest_wait_timeout(1000, FAKE, ctypes.c_void_p((1 << 20) + 4), None) == gdn.GDN_ERR_MISALIGNED
+
+
 def test_empty_batch_is_a_no_op(L):
     # B = 0 returns before any pointer is looked at or any launch is made
     assert decode(L, good_cfg(), B=0, ptrs=[None] * 10) == gdn.GDN_OK

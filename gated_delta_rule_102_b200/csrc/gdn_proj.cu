@@ -39,7 +39,10 @@ namespace {
 
 constexpr int kTileN = 128;      // weight rows per tile (the MMA's M)
 constexpr int kTileK = 64;       // bf16 elements per 128-byte swizzled row
-constexpr int kStages = 4;
+#ifndef GDN_PROJ_STAGES
+#define GDN_PROJ_STAGES 4
+#endif
+constexpr int kStages = GDN_PROJ_STAGES;  // stages in flight per CTA (build-time tuning)
 constexpr int kThreads = 128;
 constexpr int kMaxSlices = 8;    // portable cluster size
 constexpr int kWBytes = kTileN * kTileK * 2;  // 16 KiB

@@ -3,6 +3,8 @@ CUDA path (C ABI, device pools) and, for a chosen subset of its sequences, throu
 the FP64 oracle (host pools). Both sides get the same generated bits."""
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, List, Optional, Sequence
 
 import numpy as np
@@ -85,8 +87,23 @@ class OracleRun:
     def step(self, step: int) -> Dict[str, np.ndarray]:
         x = synth.step_inputs(self.wl, step, rows=self.rows)
         w = self.w
-        return oracle.decode_step(self.shape, x["qkv"], x["a"], x["b"], x["z"], w["conv_w"], w["A_log"],
-                                  w["dt_bias"], w["norm_w"], self.conv, self.state, self.local)
+        n = len(self.rows)
+        if n < 8:
+            return oracle.decode_step(self.shape, x["qkv"], x["a"], x["b"], x["z"], w["conv_w"], w["A_log"],
+                                      w["dt_bias"], w["norm_w"], self.conv, self.state, self.local)
+        # Sequences are independent: contiguous shards of rows run in threads (the oracle's C
+        # calls release the interpreter lock), each on its own slice of the pools.
+        nth = min(n // 4, os.cpu_count() or 1, 32)
+        cuts = [n * i // nth for i in range(nth + 1)]
+
+        def shard(i):
+            a, b = cuts[i], cuts[i + 1]
+            return oracle.decode_step(self.shape, x["qkv"][a:b], x["a"][a:b], x["b"][a:b], x["z"][a:b],
+                                      w["conv_w"], w["A_log"], w["dt_bias"], w["norm_w"], self.conv[a:b],
+                                      self.state[a:b], np.arange(b - a, dtype=np.int32))
+        with ThreadPoolExecutor(max_workers=nth) as ex:
+            parts = list(ex.map(shard, range(nth)))
+        return {k: np.concatenate([p[k] for p in parts]) for k in parts[0]}
 
 
 def conv_pool_reference(wl: synth.Workload, steps: int) -> np.ndarray:

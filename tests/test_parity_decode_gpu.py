@@ -49,16 +49,16 @@ def test_single_sequence_256_steps():
     _run(wl, rows=[0])
 
 
-def test_batch64_64_steps_sampled():
+def test_batch64_64_steps_every_sequence():
     wl = synth.WORKLOADS["batch64"]
-    _run(wl, rows=[0, 37, 63], check_every=4)
+    _run(wl, rows=list(range(wl.batch)), check_every=4)
 
 
-def test_pool384_batch256_32_steps_sampled():
+def test_pool384_batch256_32_steps_every_sequence():
     wl = synth.WORKLOADS["pool384_batch256"]
-    _run(wl, rows=[0, 255], check_every=4)
+    _run(wl, rows=list(range(wl.batch)), check_every=4)
 
 
-def test_multitoken_b32_t16_16_launches_sampled():
+def test_multitoken_b32_t16_16_launches_every_sequence():
     wl = synth.WORKLOADS["multitoken_b32_t16"]
-    _run(wl, rows=[0, 31], check_every=2)
+    _run(wl, rows=list(range(wl.batch)), check_every=2)

@@ -319,6 +319,25 @@ bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows)
 
 }  // namespace
 
+// The kernel's dynamic shared-memory limit, raised once per device to what the largest
+// launch (256 token rows) needs.
+cudaError_t proj_kernel_attribute() {
+    static std::mutex mu;
+    static bool set[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!set[dev]) {
+        if ((e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem_bytes(rows_padded(kProjMaxRows)))) != cudaSuccess)
+            return e;
+        set[dev] = true;
+    }
+    return cudaSuccess;
+}
+
 // Co-resident clusters of `s` CTAs for a launch of R token rows, queried once per
 // (device, s, padded rows) and cached.
 cudaError_t proj_cluster_capacity(int s, int R, int* out) {
@@ -330,15 +349,13 @@ cudaError_t proj_cluster_capacity(int s, int R, int* out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const int rp = rows_padded(R);
+    if ((e = proj_kernel_attribute()) != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < n; ++i)
         if (cache[i].dev == dev && cache[i].s == s && cache[i].rp == rp) {
             *out = cache[i].cap;
             return cudaSuccess;
         }
-    if ((e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem_bytes(rows_padded(kProjMaxRows)))) != cudaSuccess)
-        return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)s);
     cfg.blockDim = dim3(kThreads);
@@ -390,6 +407,8 @@ cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
     if (!make_map(&mw, a.w, a.N, a.K, kTileN) || !make_map(&mx, a.x, a.R, a.K, rows_padded(a.R)))
         return cudaErrorInvalidValue;
     const int smem = smem_bytes(rows_padded(a.R));
+    cudaError_t e = proj_kernel_attribute();
+    if (e != cudaSuccess) return e;
     const int tiles = (a.N + kTileN - 1) / kTileN;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tiles * a.slices));

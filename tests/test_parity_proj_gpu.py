@@ -104,3 +104,24 @@ def test_proj_is_deterministic_and_rejects_oversize():
     o = lambda n: torch.zeros(257, n, dtype=torch.bfloat16, device="cuda")  # noqa: E731
     with pytest.raises(gdn.GdnError):
         gdn.gdn_in_proj(cfg, x, w, o(wl.channels), o(128), o(4), o(4))
+
+
+def test_first_call_in_a_fresh_process_with_a_short_k():
+    # K below four 64-element blocks skips the occupancy query; the kernel's shared-memory
+    # limit must still be raised before the first launch of the process
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys, torch; sys.path.insert(0, 'tests'); import gated_delta_rule_102_b200 as gdn\n"
+        "from gated_delta_rule_102_b200 import synth\n"
+        "from gdn_harness import cfg_of\n"
+        "wl = synth.WORKLOADS['tiny_d16'].replace(num_k_heads=1, num_v_heads=2, head_k_dim=64, head_v_dim=16)\n"
+        "cfg = cfg_of(wl); rows, hidden = 33, 8\n"
+        "x = torch.randn(rows, hidden, device='cuda').to(torch.bfloat16)\n"
+        "w = torch.randn(wl.channels + 2 * 16 + 4, hidden, device='cuda').to(torch.bfloat16)\n"
+        "o = lambda n: torch.empty(rows, n, dtype=torch.bfloat16, device='cuda')\n"
+        "gdn.gdn_in_proj(cfg, x, w, o(wl.channels), o(32), o(2), o(2)); torch.cuda.synchronize(); print('ok')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stderr[-2000:]

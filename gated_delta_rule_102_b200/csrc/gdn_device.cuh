@@ -294,13 +294,22 @@ constexpr uint64_t kWaitTimeoutCycles = 2000000000ull;
 // Waits for phase `parity` of the barrier; gives up after about `timeout_cycles` SM
 // cycles and returns false. `give_up` is polled now and then so a CTA can stop waiting
 // early.
+// Suspend-time hint of each poll, in nanoseconds (0: polls without a hint). A build-time
+// tuning constant.
+#ifndef GDN_WAIT_HINT_NS
+#define GDN_WAIT_HINT_NS 1000
+#endif
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
+    if (GDN_WAIT_HINT_NS > 0) return mbar_try_wait_hint(bar, parity, GDN_WAIT_HINT_NS);
+    return mbar_try_wait(bar, parity);
+}
 template <typename GiveUp>
 __device__ __forceinline__ bool mbar_wait_deadline(uint64_t* bar, uint32_t parity, uint64_t timeout_cycles,
                                                    GiveUp give_up) {
-    if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
+    if (mbar_poll(bar, parity)) return true;
     const uint64_t t0 = clock64();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
+        if (mbar_poll(bar, parity)) return true;
         if ((i & 15) == 0) {
             if (give_up()) return false;
             if ((uint64_t)clock64() - t0 > timeout_cycles) return false;

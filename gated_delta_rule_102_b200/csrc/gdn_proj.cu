@@ -330,8 +330,12 @@ cudaError_t proj_kernel_attribute() {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (!set[dev]) {
+        int optin = 0;
+        if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+            return e;
+        const int want = smem_bytes(rows_padded(kProjMaxRows));
         if ((e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem_bytes(rows_padded(kProjMaxRows)))) != cudaSuccess)
+                                      want < optin ? want : optin)) != cudaSuccess)
             return e;
         set[dev] = true;
     }

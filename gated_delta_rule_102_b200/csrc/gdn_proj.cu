@@ -43,12 +43,20 @@ constexpr int kTileK = 64;       // bf16 elements per 128-byte swizzled row
 #define GDN_PROJ_STAGES 4
 #endif
 constexpr int kStages = GDN_PROJ_STAGES;  // stages in flight per CTA (build-time tuning)
+// 64-element K sub-tiles per stage: a stage reads kSub * 128 contiguous bytes of every
+// weight row it covers (build-time tuning)
+#ifndef GDN_PROJ_SUB
+#define GDN_PROJ_SUB 1
+#endif
+constexpr int kSub = GDN_PROJ_SUB;
+constexpr int kBlockK = kSub * 64;  // K elements per stage
 constexpr int kThreads = 128;
 constexpr int kMaxSlices = 8;    // portable cluster size
 constexpr int kWBytes = kTileN * kTileK * 2;  // 16 KiB
 
 __host__ __device__ constexpr int rows_padded(int R) { return (R + 15) / 16 * 16; }
-__host__ __device__ constexpr int stage_bytes(int Rp) { return kWBytes + Rp * kTileK * 2; }
+__host__ __device__ constexpr int sub_bytes(int Rp) { return kWBytes + Rp * kTileK * 2; }  // one K sub-tile
+__host__ __device__ constexpr int stage_bytes(int Rp) { return kSub * sub_bytes(Rp); }
 // the partial tile of the cluster reduction: [128][Rp + 4] fp32 (padded rows)
 __host__ __device__ constexpr int red_stride(int Rp) { return Rp + 4; }
 __host__ __device__ constexpr int smem_bytes(int Rp) {
@@ -148,7 +156,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
     const uint32_t ncols = Rp <= 32 ? 32 : (Rp <= 64 ? 64 : (Rp <= 128 ? 128 : 256));
 
     // this CTA's K-slice, in 64-element blocks
-    const int nkb = (p.K + kTileK - 1) / kTileK;
+    const int nkb = (p.K + kBlockK - 1) / kBlockK;
     const int kb0 = (int)((long)rank * nkb / S), kb1 = (int)((long)(rank + 1) * nkb / S);
     const int nk = kb1 - kb0;
 
@@ -191,9 +199,12 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
             }
             const uint32_t st = base + s * sbytes;
             mbar_arrive_expect_tx(full + s, (uint32_t)sbytes);
-            const int kx = (kb0 + i) * kTileK;
-            tma_load_2d(st, &map_w, kx, tile * kTileN, smem_addr(full + s));
-            tma_load_2d(st + kWBytes, &map_x, kx, 0, smem_addr(full + s));
+            for (int j = 0; j < kSub; ++j) {  // sub-tile j: the next 64 K elements of the same rows
+                const int kx = (kb0 + i) * kBlockK + j * kTileK;
+                const uint32_t sj = st + j * sub_bytes(Rp);
+                tma_load_2d(sj, &map_w, kx, tile * kTileN, smem_addr(full + s));
+                tma_load_2d(sj + kWBytes, &map_x, kx, 0, smem_addr(full + s));
+            }
             issued = i + 1;
         }
     } else if (tid == 32) {
@@ -208,10 +219,14 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
             }
             tcgen05_fence_after();
             const uint32_t st = base + s * sbytes;
-            const uint64_t da = sw128_desc(st), db = sw128_desc(st + kWBytes);
+            for (int j = 0; j < kSub; ++j) {
+                const uint32_t sj = st + j * sub_bytes(Rp);
+                const uint64_t da = sw128_desc(sj), db = sw128_desc(sj + kWBytes);
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 16; ++kk)  // K = 16 per MMA: 32 bytes along the swizzled row
-                umma_bf16(tmem, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTileK / 16; ++kk)  // K = 16 per MMA: 32 bytes along the swizzled row
+                    umma_bf16(tmem, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc,
+                              (i > 0 || j > 0 || kk > 0) ? 1u : 0u);
+            }
             umma_commit(smem_addr(empty + s));  // the stage is free once these MMAs have read it
         }
         umma_commit(smem_addr(done));  // every MMA issued above has completed
@@ -382,7 +397,7 @@ cudaError_t proj_cluster_capacity(int s, int R, int* out) {
 // every tile's cluster is co-resident, so the launch is one wave; a tile that had to
 // wait for a second wave would double the time of this bandwidth-bound GEMM.
 cudaError_t proj_slices(int N, int K, int R, int* slices) {
-    const int tiles = (N + kTileN - 1) / kTileN, nkb = (K + kTileK - 1) / kTileK;
+    const int tiles = (N + kTileN - 1) / kTileN, nkb = (K + kBlockK - 1) / kBlockK;
 #ifdef GDN_PROJ_SLICES_OVERRIDE
     {  // build-time tuning override, used when the shape allows it
         const int s = GDN_PROJ_SLICES_OVERRIDE;

@@ -393,9 +393,11 @@ cudaError_t proj_cluster_capacity(int s, int R, int* out) {
     return cudaSuccess;
 }
 
-// K-slices per weight tile: the most (up to 8, at least two K blocks each) for which
-// every tile's cluster is co-resident, so the launch is one wave; a tile that had to
-// wait for a second wave would double the time of this bandwidth-bound GEMM.
+// K-slices per weight tile. With at least half as many weight tiles as SMs (in_proj's
+// 97 at the benchmark shape) two slices measured fastest (17.7 against 20.6 µs unsplit;
+// three and more did not fit one wave of clusters). With fewer tiles, the most slices (up
+// to 8, at least two K blocks each) for which every tile's cluster is co-resident, so
+// the launch is one wave (out_proj's 16 tiles: 6).
 cudaError_t proj_slices(int N, int K, int R, int* slices) {
     const int tiles = (N + kTileN - 1) / kTileN, nkb = (K + kBlockK - 1) / kBlockK;
 #ifdef GDN_PROJ_SLICES_OVERRIDE
@@ -407,6 +409,14 @@ cudaError_t proj_slices(int N, int K, int R, int* slices) {
         }
     }
 #endif
+    int dev = 0, sms = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e0 != cudaSuccess) return e0;
+    if (2 * tiles >= sms && nkb >= 4) {
+        *slices = 2;
+        return cudaSuccess;
+    }
     int best = 1;
     for (int s = 2; s <= kMaxSlices && 2 * s <= nkb; ++s) {
         int cap = 0;

@@ -32,8 +32,8 @@
 //
 // Every wait is an mbarrier poll bounded by the SM cycle counter. When one expires the
 // CTA sets the timeout bit of the error flag, all roles leave their loops, the loader
-// gives its copies in flight time to land, and the CTA leaves through the final
-// cluster barrier.
+// waits (bounded) for the copies of the stages it armed, and the CTA leaves through the
+// final cluster barrier.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -133,6 +133,9 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
     float* qkb = reinterpret_cast<float*>(smem + L::QK);
     float* part = reinterpret_cast<float*>(smem + L::PART);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::FLAG);
+    // the last unit whose full barrier the first finisher warp has arrived on (for a CTA
+    // that gives up: the arrivals that never came)
+    volatile int* fin_full = abort_flag + 1;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
     uint64_t* empty = full + NSTAGE;
     uint64_t* cbar = empty + NSTAGE;
@@ -156,9 +159,11 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         for (int q = 0; q < QB; ++q) mbar_init(qkbar + q, 1);
         for (int r = 0; r < kRing; ++r) mbar_init(rbar + r, 1);
         *abort_flag = 0;
+        *fin_full = -1;
         mbar_init_fence();
     }
     __syncthreads();
+    int armed = 0;  // loader: units whose full and conv barriers it has armed
     auto fail = [&]() {
         if (lane == 0) {
             *abort_flag = 1;
@@ -297,6 +302,7 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                     mbar_arrive(cbar + s);
                 }
             }
+            armed = v + 1;
             __syncwarp();
             if (valid) {
                 constexpr int nchunk = (L::TILE_BYTES + kTileChunk - 1) / kTileChunk;
@@ -340,9 +346,6 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
             g_next = receive(v + 1);
             slot_next = v + 1 < kFixedUnits ? __shfl_sync(0xffffffffu, slot_fixed, v + 1)
                                             : (g_next >= 0 ? __ldg(p.slots + g_next / Hk) : -1);
-        }
-        if (*abort_flag && lane == 0) {  // give copies this CTA may still have in flight time to land
-            for (int i = 0; i < 1024; ++i) __nanosleep(64);
         }
         // The last loader through leaves the counters at zero for the next call: every
         // fetch of every cluster has returned (its value was relayed) before its CTA
@@ -439,7 +442,10 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
                 fail();  // the other finisher warps see the abort at the next agreement
                 continue;
             }
-            if (lane == 0) mbar_arrive(full + s);  // the raw q/k and v are in: pass 1 may start
+            if (lane == 0) {
+                mbar_arrive(full + s);  // the raw q/k and v are in: pass 1 may start
+                *fin_full = v;
+            }
             if (valid) {
                 const float* qr = qkb + q * 2 * DK;
                 float sq = 0.f, sk = 0.f, dot = 0.f;
@@ -584,6 +590,21 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         }
     }
     __syncthreads();
+    // A wait gave up: before the CTA leaves, the copies it still has in flight land (or a
+    // further bounded wait runs out). Every role has left its loop, so nothing else arrives
+    // on these barriers now. A stage is re-armed only after its previous phase completed,
+    // so only the last NSTAGE armed units can be outstanding; the conv barrier counts the
+    // loader's arrival and its copies, the full barrier also the first finisher warp's
+    // arrival, which is made here where it never came.
+    if (warp == 0 && lane == 0 && *abort_flag) {
+        for (int v = armed > NSTAGE ? armed - NSTAGE : 0; v < armed; ++v) {
+            const int s = v % NSTAGE;
+            const uint32_t par = (uint32_t)((v / NSTAGE) & 1);
+            mbar_wait_bounded(cbar + s, par);
+            if (v > *fin_full) mbar_arrive(full + s);
+            mbar_wait_bounded(full + s, par);
+        }
+    }
     // No CTA leaves while a peer may still send to it. Every message a CTA expects has
     // been waited for, so the arrival needs no release ordering of this CTA's stores.
     cluster_arrive_relaxed();

@@ -86,10 +86,16 @@ def kernel_for(wl, num_sms: int) -> str:
     (one CTA per SM, G CTAs per cluster), else the cluster-per-group kernels."""
     G = wl.num_v_heads // wl.num_k_heads
     if wl.ragged:
-        return "decode_mt_kernel"
+        return multitoken_kernel_for(wl)
     if wl.tokens == 1 and wl.batch * wl.num_k_heads >= 2 * (num_sms // G):
         return "decode_ws_kernel"
-    return "decode_fused_tma_kernel" if wl.tokens == 1 else "decode_mt_kernel"
+    return "decode_fused_tma_kernel" if wl.tokens == 1 else multitoken_kernel_for(wl)
+
+
+def multitoken_kernel_for(wl) -> str:
+    """Several tokens per sequence (and every speculative verify): the chunked
+    tensor-core kernel for dk = dv = 128, the register-tile kernel otherwise."""
+    return "decode_chunk_kernel" if wl.head_k_dim == 128 and wl.head_v_dim == 128 else "decode_mt_kernel"
 
 
 def algorithmic_flops(wl) -> int:
@@ -102,8 +108,9 @@ def algorithmic_flops(wl) -> int:
 KERNEL_SOURCES = {
     "decode_ws_kernel": ("gdn_decode_persistent.cu",),
     "decode_mt_kernel": ("gdn_decode_mt.cu",),
+    "decode_chunk_kernel": ("gdn_decode_chunk.cu", "gdn_tcgen05.cuh"),
     "decode_fused_tma_kernel": ("gdn_decode.cu",),
-    "proj_gemm_kernel": ("gdn_proj.cu",),
+    "proj_gemm_kernel": ("gdn_proj.cu", "gdn_tcgen05.cuh"),
     "spec_commit_kernel": ("gdn_spec.cu",),
 }
 SHARED_SOURCES = ("gdn_device.cuh", "gdn_internal.h")
@@ -535,7 +542,7 @@ def run_extra(args, name, rank, world):
                   acc * (2 * S + 4) + ntok_acc * (wl.num_k_heads * wl.head_k_dim + Z + Hv) * 4)
         flops = 7 * B * T * Hv * wl.head_k_dim * wl.head_v_dim
         tokens_per_step = B * T
-        kernel = "decode_mt_kernel"
+        kernel = multitoken_kernel_for(wl)
         note = f"{sets} state pools x {pool_bytes >> 20} MiB cycled (inputs larger than L2)"
         desc = (f"{name}: verify {B} sequences x {T} drafted tokens, then commit a seeded accepted count "
                 f"(0..{T}, mean {ntok_acc / B:.1f}) per sequence; Hk={wl.num_k_heads}, Hv={Hv}, "

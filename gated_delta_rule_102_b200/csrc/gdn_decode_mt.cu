@@ -70,9 +70,6 @@ __device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-// SiLU with the hardware exponential and an approximate division (relative error a
-// few ulp; evaluated for every conv channel and every output element of every token).
-__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 template <int DK, int DV>
 struct MtGeo {
@@ -656,6 +653,7 @@ bool multitoken_supported(const DecodeArgs& a) {
 }
 
 cudaError_t launch_decode_multitoken(const DecodeArgs& a, cudaStream_t stream) {
+    if (chunk_supported(a)) return launch_decode_chunk(a, stream);  // the tensor-core chunk form
     switch (a.sh.dk) {
         case 16: return mt_dispatch<16>(a, stream);
         case 32: return mt_dispatch<32>(a, stream);

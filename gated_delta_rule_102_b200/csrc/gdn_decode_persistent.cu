@@ -105,21 +105,6 @@ struct WS {
     static_assert(TOTAL <= 232448, "shared memory");
 };
 
-__device__ __forceinline__ void named_barrier(int id, int threads) {
-    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
-}
-// Named barrier that also returns whether `pred` held in every participating thread:
-// warps sharing later named barriers leave a loop together or not at all.
-__device__ __forceinline__ bool named_barrier_and(int id, int threads, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(threads)
-        : "memory");
-    return r != 0;
-}
-
 template <int DK, int DV>
 __global__ void __launch_bounds__(WS<DK, DV>::NT, 1)
 decode_ws_kernel(const DecodeArgs p, const int ncl) {

@@ -46,6 +46,9 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 __device__ __forceinline__ float sigmoid(float x) { return 1.0f / (1.0f + expf(-x)); }
+// SiLU with the hardware exponential and an approximate division (relative error a
+// few ulp), for the multi-token kernels' per-channel and per-output evaluations.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 // log(1 + e^x) without overflow: max(x, 0) + log1p(e^-|x|).
 __device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x))); }
 
@@ -438,6 +441,30 @@ __device__ __forceinline__ uint32_t cluster_map_u32(uint32_t smem_cta_addr, int 
 __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];\n" ::"r"(remote_addr),
                  "r"(__float_as_uint(v)), "r"(remote_bar)
+                 : "memory");
+}
+// Named barrier over `threads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+// Named barrier that also returns whether `pred` held in every participating thread:
+// warps sharing later named barriers leave a loop together or not at all.
+__device__ __forceinline__ bool named_barrier_and(int id, int threads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
+// One bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from this
+// CTA's shared memory into the shared memory of the cluster CTA that owns `dst`, counted
+// on that CTA's mbarrier `bar` (dst and bar: shared::cluster addresses).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     dst),
+                 "r"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -126,7 +126,7 @@ struct ProjArgs {
 // K-slices per weight tile (the cluster size) for a launch; the first call per shape
 // queries the device (sets the kernel attribute, occupancy), later ones hit a cache.
 cudaError_t proj_slices(int N, int K, int R, int* slices);
-int proj_smem_bytes(int R);
+int proj_smem_bytes(int R, int slices);
 cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream);
 
 // Column slices per v-head for the fused kernel: the cluster of one (sequence,
@@ -141,9 +141,12 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
 bool persistent_supported(const DecodeArgs& a);
 cudaError_t persistent_capacity(const DecodeArgs& a, int* max_clusters);
 cudaError_t launch_decode_persistent(const DecodeArgs& a, cudaStream_t stream);
-// Multi-token kernel (state in registers across the launch's tokens).
+// Multi-token kernel (state in registers across the launch's tokens); for dk = dv = 128
+// it hands the launch to the chunked tensor-core kernel.
 bool multitoken_supported(const DecodeArgs& a);
 cudaError_t launch_decode_multitoken(const DecodeArgs& a, cudaStream_t stream);
+bool chunk_supported(const DecodeArgs& a);
+cudaError_t launch_decode_chunk(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_spec_commit(const SpecCommitArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint64_t limit_cycles, int32_t* err_flag, unsigned long long* cycles,
                                  cudaStream_t stream);

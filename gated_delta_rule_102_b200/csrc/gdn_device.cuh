@@ -458,15 +458,6 @@ __device__ __forceinline__ bool named_barrier_and(int id, int threads, bool pred
         : "memory");
     return r != 0;
 }
-// One bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from this
-// CTA's shared memory into the shared memory of the cluster CTA that owns `dst`, counted
-// on that CTA's mbarrier `bar` (dst and bar: shared::cluster addresses).
-__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     dst),
-                 "r"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }

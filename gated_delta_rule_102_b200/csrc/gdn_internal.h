@@ -126,7 +126,7 @@ struct ProjArgs {
 // K-slices per weight tile (the cluster size) for a launch; the first call per shape
 // queries the device (sets the kernel attribute, occupancy), later ones hit a cache.
 cudaError_t proj_slices(int N, int K, int R, int* slices);
-int proj_smem_bytes(int R, int slices);
+int proj_smem_bytes(int R);
 cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream);
 
 // Column slices per v-head for the fused kernel: the cluster of one (sequence,

@@ -18,11 +18,9 @@
 //  * thread 32 issues tcgen05.mma (kind::f16, bf16 in, fp32 accumulate in TMEM), four
 //    K=16 steps per stage, and frees each stage with tcgen05.commit;
 //  * after the last MMA all four warps read the accumulator (warp w owns TMEM lanes
-//    32w..32w+31, i.e. weight rows) into shared memory; CTA rank q owns a band of rows
-//    and every CTA pushes each other rank's band of its partial tile into that rank's
-//    shared memory with one bulk copy (distributed shared memory, completed on the
-//    receiver's mbarrier); the owner adds the S bands in rank order (deterministic) and
-//    stores bf16 (and optionally fp32) outputs.
+//    32w..32w+31, i.e. weight rows) into shared memory; the cluster then sums its S
+//    partial tiles over distributed shared memory in rank order (deterministic), CTA
+//    rank q taking a band of rows, and stores bf16 (and optionally fp32) outputs.
 // Every mbarrier wait is bounded by the SM cycle counter; on expiry the CTA records
 // GDN_DEVICE_ERR_TIMEOUT, stops issuing work, lets what it issued complete, frees
 // its TMEM and leaves through the cluster barriers.
@@ -31,7 +29,6 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "gdn_device.cuh"
@@ -61,14 +58,11 @@ constexpr int kWBytes = kTileN * kTileK * 2;  // 16 KiB
 __host__ __device__ constexpr int rows_padded(int R) { return (R + 15) / 16 * 16; }
 __host__ __device__ constexpr int sub_bytes(int Rp) { return kWBytes + Rp * kTileK * 2; }  // one K sub-tile
 __host__ __device__ constexpr int stage_bytes(int Rp) { return kSub * sub_bytes(Rp); }
-// the partial tile of the cluster reduction: [128][Rp + 4] fp32 (padded rows), followed by
-// the bands the S-1 other CTAs send: S-1 slots of ceil(128/S) rows
+// the partial tile of the cluster reduction: [128][Rp + 4] fp32 (padded rows)
 __host__ __device__ constexpr int red_stride(int Rp) { return Rp + 4; }
-__host__ __device__ constexpr int band_rows(int S) { return (kTileN + S - 1) / S; }
-__host__ __device__ constexpr int recv_rows(int S) { return S > 1 ? (S - 1) * band_rows(S) : 0; }
-__host__ __device__ constexpr int smem_bytes(int Rp, int S) {
+__host__ __device__ constexpr int smem_bytes(int Rp) {
     const int ring = kStages * stage_bytes(Rp);
-    const int red = (kTileN + recv_rows(S)) * red_stride(Rp) * 4;
+    const int red = kTileN * red_stride(Rp) * 4;
     return 1024 + (ring > red ? ring : red) + 128;  // alignment slack, ring (reused), barriers
 }
 
@@ -79,6 +73,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "[%4];\n" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 // Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = n.
@@ -97,13 +99,12 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - smem_addr(smem_raw));
     const int sbytes = stage_bytes(Rp);
-    const int ring = kStages * sbytes, red = (kTileN + recv_rows(S)) * red_stride(Rp) * 4;
+    const int ring = kStages * sbytes, red = kTileN * red_stride(Rp) * 4;
     unsigned char* ctl = gbase + (ring > red ? ring : red);
     uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
     uint64_t* empty = full + kStages;
     uint64_t* done = empty + kStages;
-    uint64_t* recv_bar = done + 1;  // the other CTAs' bands of this CTA's rows have landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const uint32_t ncols = Rp <= 32 ? 32 : (Rp <= 64 ? 64 : (Rp <= 128 ? 128 : 256));
 
@@ -118,7 +119,6 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
             mbar_init(empty + s, 1);
         }
         mbar_init(done, 1);
-        mbar_init(recv_bar, 1);
         *abort_flag = 0;
         mbar_init_fence();
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
@@ -214,42 +214,24 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
             if (i >= issued - kStages) wait(full + s, (i / kStages) & 1);
         }
     }
-    // ---- the cluster's sum: rank q owns rows [q*128/S, (q+1)*128/S). Every CTA sends the
-    // band of each other rank to that rank's shared memory with one bulk copy (completed
-    // on the receiver's barrier); the owner adds the S partial bands in rank order.
-    const int r0 = rank * kTileN / S, r1 = (rank + 1) * kTileN / S, nr = r1 - r0;
-    float* recv = redp + kTileN * rs;  // slot j: the band from rank j (j < rank) or j + 1
-    if (tid == 0 && S > 1) mbar_arrive_expect_tx(recv_bar, (uint32_t)((S - 1) * nr * rs * 4));
-    fence_proxy_async_smem();  // the partial tile is read by the bulk copies
     tcgen05_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, ncols);
-    cluster_arrive_release();  // every partial tile is written, every receiver armed
+    cluster_arrive_release();  // every CTA's partial tile is in its shared memory
     cluster_wait_acquire();
-    if (tid == 0)
-        for (int q = 0; q < S; ++q) {
-            if (q == rank) continue;
-            const int b0 = q * kTileN / S, b1 = (q + 1) * kTileN / S;
-            const int slot = rank < q ? rank : rank - 1;  // this CTA's slot at rank q
-            const uint32_t dst = cluster_map_u32(smem_addr(recv + slot * band_rows(S) * rs), q);
-            bulk_copy_to_cluster(dst, smem_addr(redp + b0 * rs), (uint32_t)((b1 - b0) * rs * 4),
-                                 cluster_map_u32(smem_addr(recv_bar), q));
-        }
-    bool got_bands = true;
-    if (S > 1) {
-        got_bands = mbar_wait_bounded(recv_bar, 0);
-        if (!got_bands) fail();
-    }
+
+    // ---- the cluster's sum, rank order; rank q stores rows [q*128/S, (q+1)*128/S)
+    const int r0 = rank * kTileN / S, r1 = (rank + 1) * kTileN / S;
     const int nq = Rp / 4;  // float4 groups of token rows
-    for (int t = tid; got_bands && t < nr * nq; t += kThreads) {
-        const int g = t / nr, rr = t - g * nr, row = r0 + rr;
+    const uint32_t red_local = smem_addr(redp);
+    for (int t = tid; t < (r1 - r0) * nq; t += kThreads) {
+        const int g = t / (r1 - r0), row = r0 + (t - g * (r1 - r0));
         const int n = tile * kTileN + row;
         const int c = 4 * g;
         if (n >= p.N || c >= p.R) continue;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int q = 0; q < S; ++q) {
-            const float* src = q == rank ? redp + row * rs : recv + ((q < rank ? q : q - 1) * band_rows(S) + rr) * rs;
-            const float4 v = *reinterpret_cast<const float4*>(src + c);
+            const float4 v = ld_cluster_f4(cluster_map_u32(red_local + (uint32_t)(row * rs + c) * 4u, q));
             acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
         int width = p.seg_width[0], start = p.seg_start[0];
@@ -272,9 +254,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
             }
         }
     }
-    // no CTA leaves while a bulk copy may still read its partial tile: every copy has
-    // landed once its receiver passes this barrier
-    cluster_arrive_release();
+    cluster_arrive_release();  // no CTA leaves while a peer may still read its partial tile
     cluster_wait_acquire();
 }
 
@@ -307,20 +287,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows)
 
 }  // namespace
 
-// The device's opt-in shared-memory limit per block, found once per device.
-int proj_smem_limit(int dev) {
-    static std::atomic<int> limit[kMaxDevices];
-    if (dev < 0 || dev >= kMaxDevices) return 0;
-    int v = limit[dev].load(std::memory_order_relaxed);
-    if (v == 0) {
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
-        limit[dev].store(v, std::memory_order_relaxed);
-    }
-    return v;
-}
-
-// The kernel's dynamic shared-memory limit, raised once per device to the opt-in maximum
-// (a launch asks for its own size, which depends on the token rows and the slices).
+// The kernel's dynamic shared-memory limit, raised once per device to what the largest
+// launch (256 token rows) needs.
 cudaError_t proj_kernel_attribute() {
     static std::mutex mu;
     static bool set[kMaxDevices];
@@ -330,10 +298,12 @@ cudaError_t proj_kernel_attribute() {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (!set[dev]) {
-        const int optin = proj_smem_limit(dev);
-        if (optin <= 0) return cudaErrorInvalidValue;
-        if ((e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) !=
-            cudaSuccess)
+        int optin = 0;
+        if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+            return e;
+        const int want = smem_bytes(rows_padded(kProjMaxRows));
+        if ((e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      want < optin ? want : optin)) != cudaSuccess)
             return e;
         set[dev] = true;
     }
@@ -358,14 +328,10 @@ cudaError_t proj_cluster_capacity(int s, int R, int* out) {
             *out = cache[i].cap;
             return cudaSuccess;
         }
-    if (smem_bytes(rp, s) > proj_smem_limit(dev)) {  // the receive slots do not fit
-        *out = 0;
-        return cudaSuccess;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)s);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)smem_bytes(rp, s);
+    cfg.dynamicSmemBytes = (size_t)smem_bytes(rp);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)s;
@@ -400,7 +366,7 @@ cudaError_t proj_slices(int N, int K, int R, int* slices) {
     cudaError_t e0 = cudaGetDevice(&dev);
     if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e0 != cudaSuccess) return e0;
-    if (2 * tiles >= sms && nkb >= 4 && smem_bytes(rows_padded(R), 2) <= proj_smem_limit(dev)) {
+    if (2 * tiles >= sms && nkb >= 4) {
         *slices = 2;
         return cudaSuccess;
     }
@@ -415,14 +381,14 @@ cudaError_t proj_slices(int N, int K, int R, int* slices) {
     return cudaSuccess;
 }
 
-int proj_smem_bytes(int R, int slices) { return smem_bytes(rows_padded(R), slices); }
+int proj_smem_bytes(int R) { return smem_bytes(rows_padded(R)); }
 
 cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
     if (a.R <= 0 || a.N <= 0) return cudaSuccess;
     CUtensorMap mw, mx;
     if (!make_map(&mw, a.w, a.N, a.K, kTileN) || !make_map(&mx, a.x, a.R, a.K, rows_padded(a.R)))
         return cudaErrorInvalidValue;
-    const int smem = smem_bytes(rows_padded(a.R), a.slices);
+    const int smem = smem_bytes(rows_padded(a.R));
     cudaError_t e = proj_kernel_attribute();
     if (e != cudaSuccess) return e;
     const int tiles = (a.N + kTileN - 1) / kTileN;

@@ -120,9 +120,12 @@ def test_varlen_rows_past_the_end_are_skipped_and_flagged():
     assert torch.equal(g.state[s2], state0[s2])
 
 
-def test_varlen_equals_uniform_launch():
-    # every sequence with T tokens: the ragged entry point gives the uniform one's bits
-    wl = wl_of("varlen_uniform", 2, 4, 128, 128, 4, 4, 6).replace(tokens=5)
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_equals_uniform_launch(d):
+    # every sequence with T tokens: the ragged entry point gives the uniform one's bits when
+    # both run the register kernel (d = 64); at d = 128 the uniform launch takes the chunked
+    # tensor-core kernel (another summation order): both within the parity bars of each other
+    wl = wl_of(f"varlen_uniform_d{d}", 2, 4, d, d, 4, 4, 6).replace(tokens=5)
     a, b = DeviceRun(wl), DeviceRun(wl)
     x = a.inputs(0)
     out_u, out_u32 = a.step(x)
@@ -131,5 +134,11 @@ def test_varlen_equals_uniform_launch():
     flat = {k: bf16_host(v).reshape((B * T,) + tuple(v.shape[2:])) for k, v in x.items()}
     out_v, out_v32 = launch(b, wl, cu, T, flat)
     torch.cuda.synchronize()
-    assert torch.equal(out_u32.reshape(out_v32.shape), out_v32)
-    assert torch.equal(a.state, b.state) and torch.equal(a.conv, b.conv)
+    assert torch.equal(a.conv, b.conv)
+    if d == 64:
+        assert torch.equal(out_u32.reshape(out_v32.shape), out_v32)
+        assert torch.equal(a.state, b.state)
+    else:
+        assert float((out_u32.reshape(out_v32.shape) - out_v32).abs().max()) <= 2 * OUT_ABS_TOL
+        scale = a.state.abs().amax(dim=(-2, -1), keepdim=True).clamp_min(1e-30)
+        assert float(((a.state - b.state).abs() / scale).max()) <= 2e-4

@@ -24,17 +24,16 @@
 // the pool, each warp writing whole 128-byte rows. The state is read and written once
 // per launch, so the step is bound by HBM like the single-token one.
 //
-// Roles (one CTA of 288 threads per SM, walking the (sequence, k-head) groups cid,
+// Roles (one CTA of 384 threads per SM, walking the (sequence, k-head) groups cid,
 // cid + grid, ...; a group's G v-heads are its units):
-//  * warp 8, lane 0, the loader: TMA bulk copies of the units' state tiles, 32 rows
-//    (16 KiB) at a time, into a ring of chunk buffers;
-//  * warps 4-7, the producers: per group the conv + SiLU of its q and k channels, the
-//    L2 norms, the high/low operand tiles of [k | q] (K-major, 128-byte swizzle) and
-//    the Gram products k.k, q.k; per unit the conv of its v channels, SiLU(z), the
-//    gates and the unit's solve coefficients;
+//  * warps 4-11, the producers: per group the conv + SiLU of its q and k channels, the
+//    L2 norms, the high/low operand tiles of [k | q] (K-major, 128-byte swizzle), k^T
+//    and the Gram products k.k, q.k; per unit the conv of its v channels, the gates and
+//    the unit's solve coefficients; raw rows arrive by cp.async into shared memory;
 //  * warps 0-3, the consumers (thread c owns column c and TMEM lane c): state chunks
-//    into TMEM, the two GEMMs (issued by thread 0), the solve, the gated RMSNorm and
-//    the stores.
+//    into TMEM, the two GEMMs and the state copies (issued by thread 0: TMA bulk copies of
+//    32 rows, 16 KiB, into a ring holding one tile), the solve, the gated RMSNorm and the
+//    stores.
 // Groups and units pass from producers to consumers through double buffers guarded by
 // mbarriers. Every wait is bounded by the SM cycle counter; on expiry the CTA sets the
 // timeout bit, all roles leave their loops, and what was issued completes before the
@@ -58,10 +57,10 @@ constexpr int kChunkRows = 32;                       // state rows per ring buff
 constexpr int kChunkBytes = kChunkRows * kDV * 4;    // 16 KiB
 constexpr int kChunksPerTile = kDK / kChunkRows;     // 4
 constexpr int kRing = 4;                             // ring buffers: one state tile in flight
-constexpr int kConsumerWarps = 4, kProducerWarps = 4;
-constexpr int kLoaderWarp = kConsumerWarps + kProducerWarps;
-constexpr int kThreads = 32 * (kLoaderWarp + 1);
-constexpr int kConsumerBar = 1, kProducerBar = 2;    // named barriers (128 threads each)
+constexpr int kConsumerWarps = 4, kProducerWarps = 8;
+constexpr int kProducers = 32 * kProducerWarps;
+constexpr int kThreads = 32 * (kConsumerWarps + kProducerWarps);
+constexpr int kConsumerBar = 1, kProducerBar = 2;    // named barriers (consumers, producers)
 
 // [k_0..k_15 | q_0..q_15] x dk as the B operand of S0^T [k|q]^T: the tf32 high parts in
 // rows 0..31 and the low parts in rows 32..63, K = dk, K-major with the 128-byte swizzle,
@@ -93,8 +92,8 @@ constexpr int OFF_NRM = OFF_GRAW + kGroupRawBytes;       // [16] q factors, [16]
 constexpr int OFF_HEAD = OFF_NRM + 2 * kCT * 4;
 constexpr int OFF_RMS = OFF_HEAD + 2 * kHeadFloats * 4;  // [4 warps][16] partial sums of o^2
 constexpr int OFF_BAR = OFF_RMS + kConsumerWarps * kCT * 4;
-// ring full/empty [kRing] each, group full/empty [2] each, unit full/empty [2] each, mma
-constexpr int kNumBars = 2 * kRing + 8 + 1;
+// ring full [kRing], group full/empty [2] each, unit full/empty [2] each, mma
+constexpr int kNumBars = kRing + 8 + 1;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;  // TMEM address, abort flag
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(OFF_X % 1024 == 0 && OFF_Z % 1024 == 0 && kXRegion % 1024 == 0, "swizzled operand alignment");
@@ -155,8 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
     float* heads = reinterpret_cast<float*>(smem + OFF_HEAD);
     float* rms = reinterpret_cast<float*>(smem + OFF_RMS);
     uint64_t* ring_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* ring_empty = ring_full + kRing;
-    uint64_t* grp_full = ring_empty + kRing;
+    uint64_t* grp_full = ring_full + kRing;
     uint64_t* grp_empty = grp_full + 2;
     uint64_t* unit_full = grp_empty + 2;
     uint64_t* unit_empty = unit_full + 2;
@@ -165,10 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     if (tid == 0) {
-        for (int s = 0; s < kRing; ++s) {
-            mbar_init(ring_full + s, 1);
-            mbar_init(ring_empty + s, kConsumerWarps);
-        }
+        for (int s = 0; s < kRing; ++s) mbar_init(ring_full + s, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(grp_full + b, kProducerWarps);
             mbar_init(grp_empty + b, kConsumerWarps);
@@ -213,52 +208,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         return !bad_slot && !bad_len && n > 0;
     };
 
-    if (warp == kLoaderWarp) {
-        // ---- loader
-        if (lane == 0) {
-            int armed = 0;
-            bool ok = true;
-            for (int g = blockIdx.x; ok && g < ngroups; g += gridDim.x) {
-                int slot, tok0, n;
-                bool bad_slot, bad_len;
-                const bool run = group_info(g, slot, tok0, n, bad_slot, bad_len);
-                if (p.err_flag && bad_slot) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
-                if (p.err_flag && bad_len) atomicOr(p.err_flag, GDN_DEVICE_ERR_SEQLEN_BIT);
-                if (!run) continue;
-                const int hk = g % Hk;
-                for (int j = 0; ok && j < G; ++j) {
-                    const float* tile = p.state_pool + ((size_t)slot * Hv + hk * G + j) * (size_t)(kDK * kDV);
-                    for (int q = 0; q < kChunksPerTile; ++q) {
-                        const int s = armed % kRing;
-                        if (armed >= kRing && !wait(ring_empty + s, (uint32_t)(((armed / kRing) - 1) & 1))) {
-                            fail();
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(ring_full + s, (uint32_t)kChunkBytes);
-                        tma_load_1d(ring + (size_t)s * (kChunkBytes / 4), tile + (size_t)q * kChunkRows * kDV,
-                                    (uint32_t)kChunkBytes, ring_full + s);
-                        ++armed;
-                    }
-                }
-            }
-            // after an abort, the copies still in flight land before the CTA leaves
-            if (*abort_flag)
-                for (int v = armed > kRing ? armed - kRing : 0; v < armed; ++v)
-                    mbar_wait_bounded(ring_full + v % kRing, (uint32_t)((v / kRing) & 1));
-        }
-    } else if (warp >= kConsumerWarps) {
-        // ---- producers: thread i handles channel i of q, k and each unit's v, and column i
+    if (warp >= kConsumerWarps) {
+        // ---- producers: thread i handles conv channel i of the group's q | k (256) and, for
+        // i < 128, channel i of each unit's v; the group's bad slots and token counts are
+        // flagged here
         const int i = tid - 32 * kConsumerWarps, pw = warp - kConsumerWarps;
         int li = 0, hu = 0;  // groups and units produced
         for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
             int slot, tok0, n;
             bool bad_slot, bad_len;
-            if (!group_info(g, slot, tok0, n, bad_slot, bad_len)) continue;
+            const bool run = group_info(g, slot, tok0, n, bad_slot, bad_len);
+            if (i == 0 && p.err_flag && bad_slot) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
+            if (i == 0 && p.err_flag && bad_len) atomicOr(p.err_flag, GDN_DEVICE_ERR_SEQLEN_BIT);
+            if (!run) continue;
             const int gb = li & 1, hk = g % Hk;
             bool ok = li < 2 || wait(grp_empty + gb, (uint32_t)(((li >> 1) - 1) & 1));
             // (also: this group's scratch is free, every producer having read the last one)
-            if (!named_barrier_and(kProducerBar, 128, ok && !*abort_flag)) {
+            if (!named_barrier_and(kProducerBar, kProducers, ok && !*abort_flag)) {
                 if (!ok) fail();
                 break;
             }
@@ -268,35 +234,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             uint16_t* gw = graw + kRawRows * 2 * kDK;  // weights [256][W]
             {  // stage the q and k channels' history and token rows (16-byte pieces: two runs
                // of 128 channels per row) and their weights (two runs of 128 W)
-                for (int e = i; e < nrow * 32; e += 128) {
+                for (int e = i; e < nrow * 32; e += kProducers) {
                     const int r = e >> 5, part = (e >> 4) & 1, off = (e & 15) * 8;
                     const size_t ch = (size_t)(part * Hk + hk) * kDK + off;
                     cp_async_16(graw + r * 2 * kDK + part * kDK + off,
                                 r < W - 1 ? hist + (size_t)r * C + ch : x + (size_t)(r - (W - 1)) * C + ch);
                 }
                 const int wpieces = kDK * W / 8;
-                for (int e = i; e < 2 * wpieces; e += 128) {
+                for (int e = i; e < 2 * wpieces; e += kProducers) {
                     const int part = e >= wpieces, o = e - part * wpieces;
                     cp_async_16(gw + part * kDK * W + o * 8, p.conv_w + (size_t)(part * Hk + hk) * kDK * W + o * 8);
                 }
                 cp_async_wait_all();
             }
-            named_barrier(kProducerBar, 128);
-#pragma unroll 1
-            for (int part = 0; part < 2; ++part) {  // step 3 for q (then k) channel i: conv + SiLU into the scratch
+            named_barrier(kProducerBar, kProducers);
+            {  // step 3 for channel i of q | k: conv + SiLU into the scratch
                 float qk[kCT];
-                const int lc = part * kDK + i;
+                const int lc = i, part = i / kDK;
                 conv_staged(graw + lc, 2 * kDK, gw + lc * W, W, n, qk);
 #pragma unroll
                 for (int t = 0; t < kCT; ++t) scr[t * kScrStride + lc] = qk[t];
                 if (!spec)  // the new history: the last W-1 raw inputs
                     for (int r = 0; r < W - 1; ++r)
-                        hist[(size_t)r * C + (size_t)(part * Hk + hk) * kDK + i] = graw[(n + r) * 2 * kDK + lc];
+                        hist[(size_t)r * C + (size_t)(part * Hk + hk) * kDK + (i - part * kDK)] =
+                            graw[(n + r) * 2 * kDK + lc];
             }
-            named_barrier(kProducerBar, 128);
+            named_barrier(kProducerBar, kProducers);
             // L2 norms of q and k per token (step 3): factors on the raw values
 #pragma unroll
-            for (int m = 0; m < kCT / kProducerWarps; ++m) {
+            for (int m = 0; m < kCT / kProducerWarps; ++m) {  // a warp per token
                 const int t = pw + kProducerWarps * m;
                 float sq = 0.f, sk = 0.f;
 #pragma unroll
@@ -315,17 +281,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     nrm[kCT + t] = rsqrtf(sk + p.sh.l2_eps);
                 }
             }
-            named_barrier(kProducerBar, 128);
+            named_barrier(kProducerBar, kProducers);
             {  // the operand tiles: row r < 16 the normalised k_r, row 16 + t the scaled q_t
-                const int row = i >> 2;
+                const int row = i >> 3;
                 const bool isk = row < kCT;
                 const int t = isk ? row : row - kCT;
                 const float f = isk ? nrm[kCT + t] : nrm[t];
                 const float* src = scr + t * kScrStride + (isk ? kDK : 0);
                 unsigned char* xh = xbuf + gb * kXBuf;  // high parts in rows 0..31, low in 32..63
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int j = (i & 3) + 4 * m;  // 16-byte group: dk 4j .. 4j+3
+                for (int m = 0; m < 4; ++m) {
+                    const int j = (i & 7) + 8 * m;  // 16-byte group: dk 4j .. 4j+3
                     float4 v = *reinterpret_cast<const float4*>(src + 4 * j);
                     v.x *= f; v.y *= f; v.z *= f; v.w *= f;
                     const uint4 h = make_uint4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
@@ -340,46 +306,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         *reinterpret_cast<float4*>(p.spec_k + (((size_t)tok0 + t) * Hk + hk) * kDK + 4 * j) = v;
                 }
             }
-            {  // k^T for the update: row i = dk index i, high then low parts of k_0..k_15 [i]
-                unsigned char* zr = zbuf + gb * kZBuf + i * 128;
+            {  // k^T for the update: row r = dk index, high then low parts of k_0..k_15 [r]; thread
+               // i takes row i % 128 and the token quads 2 (i / 128) and 2 (i / 128) + 1
+                const int zrow = i & (kDK - 1);
+                unsigned char* zr = zbuf + gb * kZBuf + zrow * 128;
 #pragma unroll
-                for (int j = 0; j < kCT / 4; ++j) {
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int j = 2 * (i / kDK) + jj;
                     float kx[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) kx[e] = scr[(4 * j + e) * kScrStride + kDK + i] * nrm[kCT + 4 * j + e];
+                    for (int e = 0; e < 4; ++e)
+                        kx[e] = scr[(4 * j + e) * kScrStride + kDK + zrow] * nrm[kCT + 4 * j + e];
                     const uint4 h = make_uint4(tf32_hi(kx[0]), tf32_hi(kx[1]), tf32_hi(kx[2]), tf32_hi(kx[3]));
                     const uint4 l = make_uint4(__float_as_uint(kx[0] - __uint_as_float(h.x)),
                                                __float_as_uint(kx[1] - __uint_as_float(h.y)),
                                                __float_as_uint(kx[2] - __uint_as_float(h.z)),
                                                __float_as_uint(kx[3] - __uint_as_float(h.w)));
-                    *reinterpret_cast<uint4*>(zr + ((j ^ (i & 7)) << 4)) = h;
-                    *reinterpret_cast<uint4*>(zr + (((j + 4) ^ (i & 7)) << 4)) = l;
+                    *reinterpret_cast<uint4*>(zr + ((j ^ (zrow & 7)) << 4)) = h;
+                    *reinterpret_cast<uint4*>(zr + (((j + 4) ^ (zrow & 7)) << 4)) = l;
                 }
             }
-            {  // Gram products of the normalised vectors: k_t.k_s and q_t.k_s
-                const int t = i >> 3, s0 = (i & 7) * 2;
+            {  // Gram products of the normalised vectors: k_t.k_s and q_t.k_s, thread i one (t, s)
+                const int t = i >> 4, s0 = i & 15;
                 const float* qt = scr + t * kScrStride;
                 const float* kt = qt + kDK;
                 const float* k0 = scr + s0 * kScrStride + kDK;
-                const float* k1 = k0 + kScrStride;
-                float kk0 = 0.f, kk1 = 0.f, qk0 = 0.f, qk1 = 0.f;
+                float kk0 = 0.f, qk0 = 0.f;
 #pragma unroll 8
                 for (int r = 0; r < kDK; r += 4) {
                     const float4 a = *reinterpret_cast<const float4*>(kt + r);
                     const float4 b = *reinterpret_cast<const float4*>(qt + r);
                     const float4 c0 = *reinterpret_cast<const float4*>(k0 + r);
-                    const float4 c1 = *reinterpret_cast<const float4*>(k1 + r);
                     kk0 = fmaf(a.x, c0.x, fmaf(a.y, c0.y, fmaf(a.z, c0.z, fmaf(a.w, c0.w, kk0))));
-                    kk1 = fmaf(a.x, c1.x, fmaf(a.y, c1.y, fmaf(a.z, c1.z, fmaf(a.w, c1.w, kk1))));
                     qk0 = fmaf(b.x, c0.x, fmaf(b.y, c0.y, fmaf(b.z, c0.z, fmaf(b.w, c0.w, qk0))));
-                    qk1 = fmaf(b.x, c1.x, fmaf(b.y, c1.y, fmaf(b.z, c1.z, fmaf(b.w, c1.w, qk1))));
                 }
-                const float nkt = nrm[kCT + t], nqt = nrm[t], nk0 = nrm[kCT + s0], nk1 = nrm[kCT + s0 + 1];
                 float* gr = gram + gb * 2 * kCT * kCT;
-                gr[t * kCT + s0] = kk0 * nkt * nk0;
-                gr[t * kCT + s0 + 1] = kk1 * nkt * nk1;
-                gr[kCT * kCT + t * kCT + s0] = qk0 * nqt * nk0;
-                gr[kCT * kCT + t * kCT + s0 + 1] = qk1 * nqt * nk1;
+                gr[t * kCT + s0] = kk0 * nrm[kCT + t] * nrm[kCT + s0];
+                gr[kCT * kCT + t * kCT + s0] = qk0 * nrm[t] * nrm[kCT + s0];
             }
             fence_proxy_async_smem();  // the operand tiles are read by the tensor core
             __syncwarp();
@@ -393,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             for (int j = 0; j < G; ++j, ++hu) {
                 const int hb = hu & 1, h = hk * G + j;
                 ok = hu < 2 || wait(unit_empty + hb, (uint32_t)(((hu >> 1) - 1) & 1));
-                if (!named_barrier_and(kProducerBar, 128, ok && !*abort_flag)) {
+                if (!named_barrier_and(kProducerBar, kProducers, ok && !*abort_flag)) {
                     if (!ok) fail();
                     stop = true;
                     break;
@@ -409,47 +372,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 const size_t chv = (size_t)2 * Hk * kDK + (size_t)h * kDV;
                 uint16_t* uw = uraw + kRawRows * kDV;  // weights [128][W]
                 // the gate inputs of this head's tokens, loaded now and used after the staging
+                const int gi = i - kDK;  // threads 128..143: the gates of token gi
                 uint16_t ga = 0, gbb = 0;
-                if (i < kCT && i < n) {
-                    const size_t ai = ((size_t)tok0 + i) * Hv + h;
+                if (gi >= 0 && gi < kCT && gi < n) {
+                    const size_t ai = ((size_t)tok0 + gi) * Hv + h;
                     ga = p.a[ai];
                     gbb = p.b[ai];
                 }
                 {  // stage the v channels' rows and weights, and the z rows (straight into the unit's buffer)
-                    for (int e = i; e < nrow * 16; e += 128) {
+                    for (int e = i; e < nrow * 16; e += kProducers) {
                         const int r = e >> 4, off = (e & 15) * 8;
                         cp_async_16(uraw + r * kDV + off, r < W - 1 ? hist + (size_t)r * C + chv + off
                                                                     : x + (size_t)(r - (W - 1)) * C + chv + off);
                     }
-                    for (int e = i; e < kDV * W / 8; e += 128) cp_async_16(uw + e * 8, p.conv_w + chv * W + e * 8);
-                    for (int e = i; e < n * 16; e += 128) {
+                    for (int e = i; e < kDV * W / 8; e += kProducers) cp_async_16(uw + e * 8, p.conv_w + chv * W + e * 8);
+                    for (int e = i; e < n * 16; e += kProducers) {
                         const int t = e >> 4, off = (e & 15) * 8;
                         cp_async_16(hz + t * kDV + off, p.z + (((size_t)tok0 + t) * Hv + h) * kDV + off);
                     }
                     cp_async_wait_all();
                 }
-                if (i < kCT) {  // steps 4, 5 per token (no decay and no write past the sequence's tokens)
-                    float al = 1.f, be = 0.f;
-                    if (i < n) {
-                        gate_and_beta(ga, gbb, p.A_log[h], p.dt_bias[h], al, be);
-                        if (spec) p.spec_alpha[((size_t)tok0 + i) * Hv + h] = al;
-                    }
-                    ha[i] = al;
-                    hbeta[i] = be;
-                }
-                named_barrier(kProducerBar, 128);
-                {  // v channel i of this head (step 3)
+                named_barrier(kProducerBar, kProducers);
+                if (i < kDV) {  // v channel i of this head (step 3)
                     float vv[kCT];
                     conv_staged(uraw + i, kDV, uw + i * W, W, n, vv);
 #pragma unroll
                     for (int t = 0; t < kCT; ++t) hv[t * kDV + i] = vv[t];
                     if (!spec)
                         for (int r = 0; r < W - 1; ++r) hist[(size_t)r * C + chv + i] = uraw[(n + r) * kDV + i];
+                } else if (gi < kCT) {  // steps 4, 5 per token (no decay and no write past the tokens)
+                    float al = 1.f, be = 0.f;
+                    if (gi < n) {
+                        gate_and_beta(ga, gbb, p.A_log[h], p.dt_bias[h], al, be);
+                        if (spec) p.spec_alpha[((size_t)tok0 + gi) * Hv + h] = al;
+                    }
+                    ha[gi] = al;
+                    hbeta[gi] = be;
                 }
+                named_barrier(kProducerBar, kProducers);
                 // the solve's coefficients: A_ts = beta_t g_ts k_t.k_s (s < t), M_ts = g_ts q_t.k_s (s <= t)
-#pragma unroll
-                for (int e = i; e < kCT * kCT; e += 128) {
-                    const int t = e >> 4, s = e & 15;
+                {
+                    const int e = i, t = e >> 4, s = e & 15;  // one coefficient pair per thread
                     float gts = 1.f;
                     for (int u = s + 1; u <= t; ++u) gts *= ha[u];
                     hA[e] = s < t ? hbeta[t] * gts * KK[e] : 0.f;
@@ -486,6 +449,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
 #pragma unroll
             for (int r = 0; r < 32; ++r) __stcs(pend + (size_t)(32 * q + r) * kDV, col[r]);
         };
+        // Thread 0 also issues the state copies: the ring holds one tile (kRing = 4 chunks),
+        // and a unit's chunk q is copied into buffer q as soon as the unit before it has
+        // taken its own chunk q into TMEM (after that chunk's consumer barrier).
+        static_assert(kRing == kChunksPerTile, "one tile in the ring");
+        constexpr size_t kTileElems = (size_t)kDK * kDV;
+        int issued = 0;                    // chunks thread 0 has armed
+        const float* next_tile = nullptr;  // the state tile of the unit after the current one
+        auto next_group = [&](int from, int& sl) {  // the first group >= from this CTA runs
+            int gg = from, t0, nn;
+            bool bs, bl;
+            while (gg < ngroups && !group_info(gg, sl, t0, nn, bs, bl)) gg += (int)gridDim.x;
+            return gg;
+        };
+        auto issue_chunk = [&](const float* tile, int q) {
+            fence_proxy_async_smem();  // the buffer's last reads (generic proxy) before the copy
+            mbar_arrive_expect_tx(ring_full + q, (uint32_t)kChunkBytes);
+            tma_load_1d(ring + (size_t)q * (kChunkBytes / 4), tile + (size_t)q * kChunkRows * kDV,
+                        (uint32_t)kChunkBytes, ring_full + q);
+            ++issued;
+        };
+        if (c == 0) {
+            int sl = 0;
+            const int g0 = next_group(blockIdx.x, sl);
+            if (g0 < ngroups)
+                for (int q = 0; q < kChunksPerTile; ++q)
+                    issue_chunk(p.state_pool + ((size_t)sl * Hv + (g0 % Hk) * G) * kTileElems, q);
+        }
         for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
             int slot, tok0, n;
             bool bad_slot, bad_len;
@@ -508,6 +498,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 const float* hA = hw + kCT;
                 const float* hM = hA + kCT * kCT;
                 const uint16_t* hz = reinterpret_cast<const uint16_t*>(hM + kCT * kCT);
+                if (c == 0) {
+                    int sl2 = slot;
+                    const int g2 = j + 1 < G ? g : next_group(g + (int)gridDim.x, sl2);
+                    next_tile = g2 < ngroups
+                                    ? p.state_pool + ((size_t)sl2 * Hv + (g2 % Hk) * G + (g2 == g ? j + 1 : 0)) * kTileElems
+                                    : nullptr;
+                }
                 bool w = wait(unit_full + hb, (uint32_t)((hu >> 1) & 1));
                 const float gC = hgam[n - 1];
                 // ---- the state tile into TMEM chunk by chunk (S0^T high and low parts, and
@@ -536,7 +533,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         if (!spec) tmem_st16(lane_base + TM_D2 + col, dd);
                     }
                     w = __all_sync(0xffffffffu, w);
-                    if (lane == 0 && w) mbar_arrive(ring_empty + s);  // this warp has read the buffer
                     tmem_wait_st();
                     tcgen05_fence_before();
                     if (!named_barrier_and(kConsumerBar, 128, w && !*abort_flag)) {
@@ -544,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         break;
                     }
                     if (c == 0) {
+                        if (next_tile) issue_chunk(next_tile, q);  // every consumer has read buffer q
                         tcgen05_fence_after();
                         constexpr uint32_t idesc64 = idesc_tf32(4 * kCT, 0), idesc32 = idesc_tf32(2 * kCT, 0);
                         const uint64_t bx = sw128_desc(xb + q * kXRegion);
@@ -703,8 +700,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         }
         if (!ok) {
             fail();
-            // an MMA batch that was issued and never waited for completes before TMEM is freed
+            // an MMA batch that was issued and never waited for completes before TMEM is freed,
+            // and the state copies still in flight land before the CTA leaves
             if (c == 0 && mma_issued > mma_seen) mbar_wait_bounded(mma_bar, mma_seen & 1u);
+            if (c == 0)
+                for (int v = chunk; v < issued; ++v) mbar_wait_bounded(ring_full + v % kRing, (uint32_t)((v / kRing) & 1));
         }
     }
     tcgen05_fence_before();

@@ -31,9 +31,9 @@
 //    and the Gram products k.k, q.k; per unit the conv of its v channels, the gates and
 //    the unit's solve coefficients; raw rows arrive by cp.async into shared memory;
 //  * warps 0-3, the consumers (thread c owns column c and TMEM lane c): state chunks
-//    into TMEM, the two GEMMs and the state copies (issued by thread 0: TMA bulk copies of
-//    32 rows, 16 KiB, into a ring holding one tile), the solve, the gated RMSNorm and the
-//    stores.
+//    into TMEM, the two GEMMs (issued by threads 0 and 32), the state copies (issued by
+//    thread 64: TMA bulk copies of 32 rows, 16 KiB, into a ring holding one tile), the
+//    solve, the gated RMSNorm and the stores.
 // Groups and units pass from producers to consumers through double buffers guarded by
 // mbarriers. Every wait is bounded by the SM cycle counter; on expiry the CTA sets the
 // timeout bit, all roles leave their loops, and what was issued completes before the
@@ -92,8 +92,9 @@ constexpr int OFF_NRM = OFF_GRAW + kGroupRawBytes;       // [16] q factors, [16]
 constexpr int OFF_HEAD = OFF_NRM + 2 * kCT * 4;
 constexpr int OFF_RMS = OFF_HEAD + 2 * kHeadFloats * 4;  // [4 warps][16] partial sums of o^2
 constexpr int OFF_BAR = OFF_RMS + kConsumerWarps * kCT * 4;
-// ring full [kRing], group full/empty [2] each, unit full/empty [2] each, mma
-constexpr int kNumBars = kRing + 8 + 1;
+// ring full [kRing], group full/empty [2] each, unit full/empty [2] each, the update's
+// MMAs, the first GEMM's MMAs (two issuing threads)
+constexpr int kNumBars = kRing + 8 + 2;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;  // TMEM address, abort flag
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(OFF_X % 1024 == 0 && OFF_Z % 1024 == 0 && kXRegion % 1024 == 0, "swizzled operand alignment");
@@ -104,8 +105,9 @@ static_assert(kSmemBytes <= 232448, "shared memory");
 // TMEM columns (one fp32 per column per lane)
 constexpr uint32_t TM_AHI = 0, TM_ALO = 128;  // S0^T high and low parts (K = dk)
 constexpr uint32_t TM_D2 = 256;               // the update's accumulator: S_n^T
-constexpr uint32_t TM_D1 = 384;               // S0^T [k | q]^T: 64 columns (two partial sums)
-constexpr uint32_t TM_YHI = 448, TM_YLO = 464;  // A of the update: g_{n-1,t} delta_t (K = 16 tokens)
+constexpr uint32_t TM_D1 = 384;   // S0_hi^T [k | q]_hi^T and S0_hi^T [k | q]_lo^T: 2 x 32 columns
+constexpr uint32_t TM_D1B = 448;  // S0_lo^T [k | q]_hi^T: 32 columns (issued by another thread)
+constexpr uint32_t TM_YHI = 480, TM_YLO = 496;  // A of the update: g_{n-1,t} delta_t (K = 16 tokens)
 constexpr uint32_t kTmemCols = 512;
 static_assert(TM_YLO + kCT <= kTmemCols, "TMEM columns");
 
@@ -158,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
     uint64_t* grp_empty = grp_full + 2;
     uint64_t* unit_full = grp_empty + 2;
     uint64_t* unit_empty = unit_full + 2;
-    uint64_t* mma_bar = unit_empty + 2;
+    uint64_t* mma_bar = unit_empty + 2;  // the update GEMM (thread 0)
+    uint64_t* g1_bar = mma_bar + 1;      // the first GEMM (threads 0 and 32)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -171,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             mbar_init(unit_empty + b, kConsumerWarps);
         }
         mbar_init(mma_bar, 1);
+        mbar_init(g1_bar, 2);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -440,7 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         const float nwc = bf16_bits_to_float(p.norm_w[c]);
         int li = 0, hu = 0, chunk = 0;
-        uint32_t mma_issued = 0, mma_seen = 0;  // commits issued (counted by all) and waited for (own)
+        uint32_t mma_issued = 0, mma_seen = 0;  // update commits issued (counted by all) and waited for (own)
+        uint32_t g1_seen = 0;                   // first-GEMM phases waited for (own)
+        bool g1_open = false;                   // (threads 0, 32) MMAs issued since their last commit
         float* pend = nullptr;                  // column c of the state tile still in the accumulator
         bool ok = true;
         auto store_chunk = [&](int q) {         // rows 32q .. 32q+31 of the pending tile
@@ -449,12 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
 #pragma unroll
             for (int r = 0; r < 32; ++r) __stcs(pend + (size_t)(32 * q + r) * kDV, col[r]);
         };
-        // Thread 0 also issues the state copies: the ring holds one tile (kRing = 4 chunks),
-        // and a unit's chunk q is copied into buffer q as soon as the unit before it has
-        // taken its own chunk q into TMEM (after that chunk's consumer barrier).
+        // Thread 64 issues the state copies: the ring holds one tile (kRing = 4 chunks), and
+        // a unit's chunk q is copied into buffer q as soon as the unit before it has taken
+        // its own chunk q into TMEM (after that chunk's consumer barrier).
         static_assert(kRing == kChunksPerTile, "one tile in the ring");
         constexpr size_t kTileElems = (size_t)kDK * kDV;
-        int issued = 0;                    // chunks thread 0 has armed
+        constexpr int kCopier = 64;        // the thread (warp 2) that issues the state copies
+        int issued = 0;                    // chunks the copier has armed
         const float* next_tile = nullptr;  // the state tile of the unit after the current one
         auto next_group = [&](int from, int& sl) {  // the first group >= from this CTA runs
             int gg = from, t0, nn;
@@ -469,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         (uint32_t)kChunkBytes, ring_full + q);
             ++issued;
         };
-        if (c == 0) {
+        if (c == kCopier) {
             int sl = 0;
             const int g0 = next_group(blockIdx.x, sl);
             if (g0 < ngroups)
@@ -498,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 const float* hA = hw + kCT;
                 const float* hM = hA + kCT * kCT;
                 const uint16_t* hz = reinterpret_cast<const uint16_t*>(hM + kCT * kCT);
-                if (c == 0) {
+                if (c == kCopier) {
                     int sl2 = slot;
                     const int g2 = j + 1 < G ? g : next_group(g + (int)gridDim.x, sl2);
                     next_tile = g2 < ngroups
@@ -539,39 +546,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         ok = false;
                         break;
                     }
-                    if (c == 0) {
-                        if (next_tile) issue_chunk(next_tile, q);  // every consumer has read buffer q
+                    // the chunk's MMAs from two threads of different warps, each into its own
+                    // accumulator (a fixed order per accumulator), and the next unit's chunk q
+                    // from a third
+                    if (c == kCopier && next_tile) issue_chunk(next_tile, q);  // every consumer has read buffer q
+                    if (c == 0 || c == 32) {
                         tcgen05_fence_after();
-                        constexpr uint32_t idesc64 = idesc_tf32(4 * kCT, 0), idesc32 = idesc_tf32(2 * kCT, 0);
                         const uint64_t bx = sw128_desc(xb + q * kXRegion);
+                        if (c == 0) {
+                            constexpr uint32_t idesc64 = idesc_tf32(4 * kCT, 0);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_tf32_ts(tmem + TM_D1, tmem + TM_AHI + 32 * q + 8 * kk, bx + (uint64_t)(2 * kk),
-                                         idesc64, (q | kk) != 0 ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_tf32_ts(tmem + TM_D1, tmem + TM_AHI + 32 * q + 8 * kk, bx + (uint64_t)(2 * kk),
+                                             idesc64, (q | kk) != 0 ? 1u : 0u);
+                        } else {
+                            constexpr uint32_t idesc32 = idesc_tf32(2 * kCT, 0);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_tf32_ts(tmem + TM_D1, tmem + TM_ALO + 32 * q + 8 * kk, bx + (uint64_t)(2 * kk),
-                                         idesc32, 1u);
-                        if (q == kChunksPerTile - 1) umma_commit(smem_addr(mma_bar));
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_tf32_ts(tmem + TM_D1B, tmem + TM_ALO + 32 * q + 8 * kk, bx + (uint64_t)(2 * kk),
+                                             idesc32, (q | kk) != 0 ? 1u : 0u);
+                        }
+                        g1_open = true;
+                        if (q == kChunksPerTile - 1) {
+                            umma_commit(smem_addr(g1_bar));
+                            g1_open = false;
+                        }
                     }
                 }
                 if (!ok) break;
                 pend = nullptr;
-                ++mma_issued;
                 float vv[kCT];
 #pragma unroll
                 for (int t = 0; t < kCT; ++t) vv[t] = hv[t * kDV + c];
-                w = wait(mma_bar, mma_seen & 1u);
-                if (w) ++mma_seen;
+                w = wait(g1_bar, g1_seen & 1u);
+                if (w) ++g1_seen;
                 tcgen05_fence_after();
-                float d1[32];  // [S0^T k_t]_c for t < 16, then [S0^T q_t]_c: the two partial sums added
+                float d1[32];  // [S0^T k_t]_c for t < 16, then [S0^T q_t]_c: the three partial sums added
 #pragma unroll
-                for (int h16 = 0; h16 < 2; ++h16) {
-                    float pa[16], pb[16];
-                    tmem_ld16(lane_base + TM_D1 + 16 * h16, pa);
-                    tmem_ld16(lane_base + TM_D1 + 32 + 16 * h16, pb);
+                for (int part = 0; part < 6; ++part) {  // 16 columns of one partial sum at a time
+                    float pa[16];
+                    const int h16 = part & 1, which = part >> 1;
+                    tmem_ld16(lane_base + (which == 0 ? TM_D1 : which == 1 ? TM_D1 + 32 : TM_D1B) + 16 * h16, pa);
 #pragma unroll
-                    for (int j2 = 0; j2 < 16; ++j2) d1[16 * h16 + j2] = pa[j2] + pb[j2];
+                    for (int j2 = 0; j2 < 16; ++j2) d1[16 * h16 + j2] = which == 0 ? pa[j2] : d1[16 * h16 + j2] + pa[j2];
                 }
                 // ---- steps 6, 7: the triangular solve for delta and the outputs, column c
                 // (the coefficients of token t read as one row of float4s)
@@ -624,21 +641,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     ok = false;
                     break;
                 }
-                if (!spec) {
-                    if (c == 0) {  // S_n^T = gamma S0^T + (w delta)^T k, B = k^T (K = tokens)
-                        tcgen05_fence_after();
-                        constexpr uint32_t idesc = idesc_tf32(kDK, 0);
-                        const uint64_t bz = sw128_desc(zb);
-#pragma unroll
-                        for (int kk = 0; kk < kCT / 8; ++kk) {  // 8 tokens per MMA; low parts of k at 64 bytes
-                            umma_tf32_ts(tmem + TM_D2, tmem + TM_YHI + 8 * kk, bz + (uint64_t)(2 * kk), idesc, 1u);
-                            umma_tf32_ts(tmem + TM_D2, tmem + TM_YHI + 8 * kk, bz + (uint64_t)(2 * (kk + 2)), idesc, 1u);
-                            umma_tf32_ts(tmem + TM_D2, tmem + TM_YLO + 8 * kk, bz + (uint64_t)(2 * kk), idesc, 1u);
-                        }
-                        umma_commit(smem_addr(mma_bar));
-                    }
-                    ++mma_issued;
-                }
                 // ---- step 8 and the gate: RMSNorm over the head's 128 columns, per token.
                 // Butterfly over the warp, halving the tokens each round: lane L ends with
                 // the warp's sum for token (L >> 1) & 15.
@@ -664,6 +666,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     if ((lane & 1) == 0) rms[warp * kCT + ((lane >> 1) & 15)] = sq[0];
                 }
                 named_barrier(kConsumerBar, 128);
+                if (!spec) {  // issued here so that no warp waits for the issue
+                    if (c == 0) {  // S_n^T = gamma S0^T + (w delta)^T k, B = k^T (K = tokens)
+                        tcgen05_fence_after();
+                        constexpr uint32_t idesc = idesc_tf32(kDK, 0);
+                        const uint64_t bz = sw128_desc(zb);
+#pragma unroll
+                        for (int kk = 0; kk < kCT / 8; ++kk) {  // 8 tokens per MMA; low parts of k at 64 bytes
+                            umma_tf32_ts(tmem + TM_D2, tmem + TM_YHI + 8 * kk, bz + (uint64_t)(2 * kk), idesc, 1u);
+                            umma_tf32_ts(tmem + TM_D2, tmem + TM_YHI + 8 * kk, bz + (uint64_t)(2 * (kk + 2)), idesc, 1u);
+                            umma_tf32_ts(tmem + TM_D2, tmem + TM_YLO + 8 * kk, bz + (uint64_t)(2 * kk), idesc, 1u);
+                        }
+                        umma_commit(smem_addr(mma_bar));
+                    }
+                    ++mma_issued;
+                }
 #pragma unroll
                 for (int t = 0; t < kCT; ++t) {
                     if (t >= n) continue;
@@ -703,7 +720,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             // an MMA batch that was issued and never waited for completes before TMEM is freed,
             // and the state copies still in flight land before the CTA leaves
             if (c == 0 && mma_issued > mma_seen) mbar_wait_bounded(mma_bar, mma_seen & 1u);
-            if (c == 0)
+            if ((c == 0 || c == 32) && g1_open) {  // a first GEMM left half-issued: close it and wait
+                umma_commit(smem_addr(g1_bar));
+                mbar_wait_bounded(g1_bar, g1_seen & 1u);
+            }
+            if (c == kCopier)
                 for (int v = chunk; v < issued; ++v) mbar_wait_bounded(ring_full + v % kRing, (uint32_t)((v / kRing) & 1));
         }
     }

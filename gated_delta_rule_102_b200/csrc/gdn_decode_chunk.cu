@@ -77,9 +77,10 @@ constexpr int kRawRows = kMaxConvWidth - 1 + kCT;  // staged conv input rows: hi
 constexpr int kGroupRawBytes = kRawRows * 2 * kDK * 2 + 2 * kDK * kMaxConvWidth * 2;
 // per unit (producers only, in the scratch's place): the v channels' raw rows and weights
 constexpr int kUnitRawBytes = kRawRows * kDV * 2 + kDV * kMaxConvWidth * 2;
-// per unit (double-buffered): v [16][128] f32, alpha, beta, gamma, w [16], the solve's
-// coefficients A [16][16] and M [16][16], then z [16][128] bf16
-constexpr int kHeadFloats = kCT * kDV + 4 * kCT + 2 * kCT * kCT + kCT * kDV / 2;
+// per unit (double-buffered): v [16][128] f32 (replaced by o once the consumers have solved),
+// alpha, beta, gamma, w [16], the solve's coefficients A [16][16] and M [16][16], z [16][128]
+// bf16, and the unit's first packed row, v-head and token count (ints)
+constexpr int kHeadFloats = kCT * kDV + 4 * kCT + 2 * kCT * kCT + kCT * kDV / 2 + 4;
 
 // shared-memory byte offsets from a 1024-byte aligned base
 constexpr int OFF_RING = 0;
@@ -90,8 +91,7 @@ constexpr int OFF_SCR = OFF_GRAM + 2 * 2 * kCT * kCT * 4;
 constexpr int OFF_GRAW = OFF_SCR + kCT * kScrStride * 4;
 constexpr int OFF_NRM = OFF_GRAW + kGroupRawBytes;       // [16] q factors, [16] k factors
 constexpr int OFF_HEAD = OFF_NRM + 2 * kCT * 4;
-constexpr int OFF_RMS = OFF_HEAD + 2 * kHeadFloats * 4;  // [4 warps][16] partial sums of o^2
-constexpr int OFF_BAR = OFF_RMS + kConsumerWarps * kCT * 4;
+constexpr int OFF_BAR = OFF_HEAD + 2 * kHeadFloats * 4;
 // ring full [kRing], group full/empty [2] each, unit full/empty [2] each, the update's
 // MMAs, the first GEMM's MMAs (two issuing threads)
 constexpr int kNumBars = kRing + 8 + 2;
@@ -154,7 +154,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
     uint16_t* graw = reinterpret_cast<uint16_t*>(smem + OFF_GRAW);
     float* nrm = reinterpret_cast<float*>(smem + OFF_NRM);
     float* heads = reinterpret_cast<float*>(smem + OFF_HEAD);
-    float* rms = reinterpret_cast<float*>(smem + OFF_RMS);
     uint64_t* ring_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* grp_full = ring_full + kRing;
     uint64_t* grp_empty = grp_full + 2;
@@ -218,6 +217,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         // flagged here
         const int i = tid - 32 * kConsumerWarps, pw = warp - kConsumerWarps;
         int li = 0, hu = 0;  // groups and units produced
+        // step 8 and the SiLU(z) gate of a solved unit in buffer ub: a warp per token, four
+        // columns per lane
+        auto emit_unit = [&](int ub) {
+            const uint2 nw4 = __ldg(reinterpret_cast<const uint2*>(p.norm_w) + lane);
+            const float nw[4] = {bf16_bits_to_float(nw4.x & 0xffffu), bf16_bits_to_float(nw4.x >> 16),
+                                 bf16_bits_to_float(nw4.y & 0xffffu), bf16_bits_to_float(nw4.y >> 16)};
+            const float* ov = heads + ub * kHeadFloats;
+            const uint16_t* oz = reinterpret_cast<const uint16_t*>(ov + kCT * kDV + 4 * kCT + 2 * kCT * kCT);
+            const int* meta = reinterpret_cast<const int*>(ov + kHeadFloats - 4);
+            const int ut0 = meta[0], uh = meta[1], un = meta[2];
+            for (int t = pw; t < un; t += kProducerWarps) {
+                const float4 o4 = reinterpret_cast<const float4*>(ov + t * kDV)[lane];
+                float ss = o4.x * o4.x + o4.y * o4.y + o4.z * o4.z + o4.w * o4.w;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float inv = rsqrtf(ss * (1.0f / (float)kDV) + p.sh.rms_eps);
+                const uint2 z2 = reinterpret_cast<const uint2*>(oz + t * kDV)[lane];
+                const float y0 = o4.x * inv * nw[0] * silu_fast(bf16_bits_to_float(z2.x & 0xffffu));
+                const float y1 = o4.y * inv * nw[1] * silu_fast(bf16_bits_to_float(z2.x >> 16));
+                const float y2 = o4.z * inv * nw[2] * silu_fast(bf16_bits_to_float(z2.y & 0xffffu));
+                const float y3 = o4.w * inv * nw[3] * silu_fast(bf16_bits_to_float(z2.y >> 16));
+                const size_t oi = (((size_t)ut0 + t) * Hv + uh) * kDV + 4 * lane;
+                uint2 packed;
+                packed.x = (uint32_t)float_to_bf16_bits(y0) | ((uint32_t)float_to_bf16_bits(y1) << 16);
+                packed.y = (uint32_t)float_to_bf16_bits(y2) | ((uint32_t)float_to_bf16_bits(y3) << 16);
+                *reinterpret_cast<uint2*>(p.out + oi) = packed;
+                if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + oi) = make_float4(y0, y1, y2, y3);
+            }
+        };
         for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
             int slot, tok0, n;
             bool bad_slot, bad_len;
@@ -365,6 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     stop = true;
                     break;
                 }
+                if (hu >= 2) {  // the unit solved two units ago leaves the buffer first
+                    emit_unit(hb);
+                    named_barrier(kProducerBar, kProducers);
+                }
                 float* hv = heads + hb * kHeadFloats;  // v [16][128]
                 float* ha = hv + kCT * kDV;            // alpha [16], beta, gamma, w, A [16][16], M [16][16]
                 float* hbeta = ha + kCT;
@@ -373,6 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 float* hA = hw + kCT;
                 float* hM = hA + kCT * kCT;
                 uint16_t* hz = reinterpret_cast<uint16_t*>(hM + kCT * kCT);  // z [16][128] bf16
+                if (i == 0) {
+                    int* meta = reinterpret_cast<int*>(hv + kHeadFloats - 4);
+                    meta[0] = tok0;
+                    meta[1] = h;
+                    meta[2] = n;
+                }
                 const size_t chv = (size_t)2 * Hk * kDK + (size_t)h * kDV;
                 uint16_t* uw = uraw + kRawRows * kDV;  // weights [128][W]
                 // the gate inputs of this head's tokens, loaded now and used after the staging
@@ -434,6 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             }
             if (stop) break;
         }
+        // the last two units' outputs (every producer takes the same decision)
+        if (named_barrier_and(kProducerBar, kProducers, !*abort_flag))
+            for (int u = hu >= 2 ? hu - 2 : 0; u < hu; ++u) {
+                const bool got = wait(unit_empty + (u & 1), (uint32_t)((u >> 1) & 1));
+                if (!named_barrier_and(kProducerBar, kProducers, got && !*abort_flag)) {
+                    if (!got) fail();
+                    break;
+                }
+                emit_unit(u & 1);
+            }
     } else {
         // ---- consumers: thread c owns state column c (TMEM lane c). A wait that gives
         // up is agreed on at the next consumer barrier, where all four warps leave
@@ -442,7 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         // the accumulator is stored just before the next unit's chunk q overwrites it.
         const int c = tid;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        const float nwc = bf16_bits_to_float(p.norm_w[c]);
         int li = 0, hu = 0, chunk = 0;
         uint32_t mma_issued = 0, mma_seen = 0;  // update commits issued (counted by all) and waited for (own)
         uint32_t g1_seen = 0;                   // first-GEMM phases waited for (own)
@@ -497,14 +544,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             const uint32_t zb = smem_addr(zbuf + gb * kZBuf);
             for (int j = 0; j < G; ++j, ++hu) {
                 const int hb = hu & 1, h = hk * G + j;
-                const float* hv = heads + hb * kHeadFloats;
+                float* hv = heads + hb * kHeadFloats;  // v, then o
                 const float* ha = hv + kCT * kDV;
                 const float* hbeta = ha + kCT;
                 const float* hgam = hbeta + kCT;
                 const float* hw = hgam + kCT;
                 const float* hA = hw + kCT;
                 const float* hM = hA + kCT * kCT;
-                const uint16_t* hz = reinterpret_cast<const uint16_t*>(hM + kCT * kCT);
                 if (c == kCopier) {
                     int sl2 = slot;
                     const int g2 = j + 1 < G ? g : next_group(g + (int)gridDim.x, sl2);
@@ -620,6 +666,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     dl[t] = t < n ? xd : 0.f;
                     o[t] = fmaf(mv[t], dl[t], xo);
                 }
+                // o of column c replaces v_c (this thread has read it) for the producers'
+                // gated RMSNorm
+#pragma unroll
+                for (int t = 0; t < kCT; ++t) hv[t * kDV + c] = o[t];
                 if (spec) {
 #pragma unroll
                     for (int t = 0; t < kCT; ++t)
@@ -641,32 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     ok = false;
                     break;
                 }
-                // ---- step 8 and the gate: RMSNorm over the head's 128 columns, per token.
-                // Butterfly over the warp, halving the tokens each round: lane L ends with
-                // the warp's sum for token (L >> 1) & 15.
-                {
-                    float sq[kCT];
-#pragma unroll
-                    for (int t = 0; t < kCT; ++t) sq[t] = o[t] * o[t];
-                    auto fold = [&](auto half_c) {  // lanes 2*half apart swap halves and add
-                        constexpr int half = decltype(half_c)::value;
-                        const bool upper = (lane & (2 * half)) != 0;
-#pragma unroll
-                        for (int t = 0; t < half; ++t) {
-                            const float send = upper ? sq[t] : sq[t + half];
-                            const float keep = upper ? sq[t + half] : sq[t];
-                            sq[t] = keep + __shfl_xor_sync(0xffffffffu, send, 2 * half);
-                        }
-                    };
-                    fold(std::integral_constant<int, 8>{});
-                    fold(std::integral_constant<int, 4>{});
-                    fold(std::integral_constant<int, 2>{});
-                    fold(std::integral_constant<int, 1>{});
-                    sq[0] += __shfl_xor_sync(0xffffffffu, sq[0], 1);
-                    if ((lane & 1) == 0) rms[warp * kCT + ((lane >> 1) & 15)] = sq[0];
-                }
-                named_barrier(kConsumerBar, 128);
-                if (!spec) {  // issued here so that no warp waits for the issue
+                if (!spec) {
                     if (c == 0) {  // S_n^T = gamma S0^T + (w delta)^T k, B = k^T (K = tokens)
                         tcgen05_fence_after();
                         constexpr uint32_t idesc = idesc_tf32(kDK, 0);
@@ -681,18 +706,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     }
                     ++mma_issued;
                 }
-#pragma unroll
-                for (int t = 0; t < kCT; ++t) {
-                    if (t >= n) continue;
-                    const float ss = rms[t] + rms[kCT + t] + rms[2 * kCT + t] + rms[3 * kCT + t];
-                    const float inv = rsqrtf(ss * (1.0f / (float)kDV) + p.sh.rms_eps);
-                    const float y = o[t] * inv * nwc * silu_fast(bf16_bits_to_float(hz[t * kDV + c]));
-                    const size_t oi = (((size_t)tok0 + t) * Hv + h) * kDV + c;
-                    p.out[oi] = float_to_bf16_bits(y);
-                    if (p.out_f32) p.out_f32[oi] = y;
-                }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(unit_empty + hb);  // the unit's inputs are consumed
+                if (lane == 0) mbar_arrive(unit_empty + hb);  // inputs consumed, o written
                 if (!spec) {  // the update is done: the tile is stored during the next unit's chunks
                     w = wait(mma_bar, mma_seen & 1u);
                     if (w) ++mma_seen;
@@ -700,7 +715,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     pend = p.state_pool + ((size_t)slot * Hv + h) * (size_t)(kDK * kDV) + c;
                 }
                 tcgen05_fence_before();
-                // (the rms partials are rewritten by the next unit only after this barrier)
                 if (!named_barrier_and(kConsumerBar, 128, w && !*abort_flag)) {
                     ok = false;
                     break;

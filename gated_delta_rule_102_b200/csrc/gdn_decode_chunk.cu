@@ -217,6 +217,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         // flagged here
         const int i = tid - 32 * kConsumerWarps, pw = warp - kConsumerWarps;
         int li = 0, hu = 0;  // groups and units produced
+        int gstaged = -1;    // the group whose q/k rows and weights are in (or on their way to) graw
+        int emitted = -1;    // the last unit whose outputs are written
+        int ustaged = -1;    // the unit whose v rows, weights and z rows are staged
+        // cp.async of group gg's q and k channels: their history and token rows (16-byte
+        // pieces, two runs of 128 channels per row) and weights (two runs of 128 W)
+        auto stage_group = [&](int gg, int sl, int t0, int nn) {
+            const int kh = gg % Hk, nr = W - 1 + nn;
+            const uint16_t* hs = p.conv_pool + (size_t)sl * (W - 1) * C;
+            const uint16_t* xs = p.qkv + (size_t)t0 * C;
+            for (int e = i; e < nr * 32; e += kProducers) {
+                const int r = e >> 5, part = (e >> 4) & 1, off = (e & 15) * 8;
+                const size_t ch = (size_t)(part * Hk + kh) * kDK + off;
+                cp_async_16(graw + r * 2 * kDK + part * kDK + off,
+                            r < W - 1 ? hs + (size_t)r * C + ch : xs + (size_t)(r - (W - 1)) * C + ch);
+            }
+            const int wpieces = kDK * W / 8;
+            uint16_t* gwt = graw + kRawRows * 2 * kDK;
+            for (int e = i; e < 2 * wpieces; e += kProducers) {
+                const int part = e >= wpieces, o = e - part * wpieces;
+                cp_async_16(gwt + part * kDK * W + o * 8, p.conv_w + (size_t)(part * Hk + kh) * kDK * W + o * 8);
+            }
+            gstaged = gg;
+        };
         // step 8 and the SiLU(z) gate of a solved unit in buffer ub: a warp per token, four
         // columns per lane
         auto emit_unit = [&](int ub) {
@@ -264,21 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             const uint16_t* x = p.qkv + (size_t)tok0 * C;
             const int nrow = W - 1 + n;
             uint16_t* gw = graw + kRawRows * 2 * kDK;  // weights [256][W]
-            {  // stage the q and k channels' history and token rows (16-byte pieces: two runs
-               // of 128 channels per row) and their weights (two runs of 128 W)
-                for (int e = i; e < nrow * 32; e += kProducers) {
-                    const int r = e >> 5, part = (e >> 4) & 1, off = (e & 15) * 8;
-                    const size_t ch = (size_t)(part * Hk + hk) * kDK + off;
-                    cp_async_16(graw + r * 2 * kDK + part * kDK + off,
-                                r < W - 1 ? hist + (size_t)r * C + ch : x + (size_t)(r - (W - 1)) * C + ch);
-                }
-                const int wpieces = kDK * W / 8;
-                for (int e = i; e < 2 * wpieces; e += kProducers) {
-                    const int part = e >= wpieces, o = e - part * wpieces;
-                    cp_async_16(gw + part * kDK * W + o * 8, p.conv_w + (size_t)(part * Hk + hk) * kDK * W + o * 8);
-                }
-                cp_async_wait_all();
+            // the next group this CTA runs, looked up now (its loads travel during the conv)
+            int g2 = g + (int)gridDim.x, s2 = 0, t2 = 0, n2 = 0;
+            {
+                bool b2s, b2l;
+                while (g2 < ngroups && !group_info(g2, s2, t2, n2, b2s, b2l)) g2 += (int)gridDim.x;
             }
+            if (gstaged != g) stage_group(g, slot, tok0, n);  // (normally staged while the group before ran)
+            cp_async_wait_all();
             named_barrier(kProducerBar, kProducers);
             {  // step 3 for channel i of q | k: conv + SiLU into the scratch
                 float qk[kCT];
@@ -292,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                             graw[(n + r) * 2 * kDK + lc];
             }
             named_barrier(kProducerBar, kProducers);
+            if (g2 < ngroups) stage_group(g2, s2, t2, n2);  // the staging buffer is free: the next group's rows
             // L2 norms of q and k per token (step 3): factors on the raw values
 #pragma unroll
             for (int m = 0; m < kCT / kProducerWarps; ++m) {  // a warp per token
@@ -363,15 +380,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 const float* qt = scr + t * kScrStride;
                 const float* kt = qt + kDK;
                 const float* k0 = scr + s0 * kScrStride + kDK;
-                float kk0 = 0.f, qk0 = 0.f;
+                float4 kk4 = make_float4(0.f, 0.f, 0.f, 0.f), qk4 = kk4;  // four independent chains each
 #pragma unroll 8
                 for (int r = 0; r < kDK; r += 4) {
                     const float4 a = *reinterpret_cast<const float4*>(kt + r);
                     const float4 b = *reinterpret_cast<const float4*>(qt + r);
                     const float4 c0 = *reinterpret_cast<const float4*>(k0 + r);
-                    kk0 = fmaf(a.x, c0.x, fmaf(a.y, c0.y, fmaf(a.z, c0.z, fmaf(a.w, c0.w, kk0))));
-                    qk0 = fmaf(b.x, c0.x, fmaf(b.y, c0.y, fmaf(b.z, c0.z, fmaf(b.w, c0.w, qk0))));
+                    kk4.x = fmaf(a.x, c0.x, kk4.x); kk4.y = fmaf(a.y, c0.y, kk4.y);
+                    kk4.z = fmaf(a.z, c0.z, kk4.z); kk4.w = fmaf(a.w, c0.w, kk4.w);
+                    qk4.x = fmaf(b.x, c0.x, qk4.x); qk4.y = fmaf(b.y, c0.y, qk4.y);
+                    qk4.z = fmaf(b.z, c0.z, qk4.z); qk4.w = fmaf(b.w, c0.w, qk4.w);
                 }
+                const float kk0 = (kk4.x + kk4.y) + (kk4.z + kk4.w), qk0 = (qk4.x + qk4.y) + (qk4.z + qk4.w);
                 float* gr = gram + gb * 2 * kCT * kCT;
                 gr[t * kCT + s0] = kk0 * nrm[kCT + t] * nrm[kCT + s0];
                 gr[kCT * kCT + t * kCT + s0] = qk0 * nrm[t] * nrm[kCT + s0];
@@ -393,8 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     stop = true;
                     break;
                 }
-                if (hu >= 2) {  // the unit solved two units ago leaves the buffer first
+                if (hu >= 2 && emitted < hu - 2) {  // the unit solved two units ago leaves the buffer first
                     emit_unit(hb);
+                    emitted = hu - 2;
                     named_barrier(kProducerBar, kProducers);
                 }
                 float* hv = heads + hb * kHeadFloats;  // v [16][128]
@@ -404,7 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 float* hw = hgam + kCT;
                 float* hA = hw + kCT;
                 float* hM = hA + kCT * kCT;
-                uint16_t* hz = reinterpret_cast<uint16_t*>(hM + kCT * kCT);  // z [16][128] bf16
                 if (i == 0) {
                     int* meta = reinterpret_cast<int*>(hv + kHeadFloats - 4);
                     meta[0] = tok0;
@@ -421,19 +441,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     ga = p.a[ai];
                     gbb = p.b[ai];
                 }
-                {  // stage the v channels' rows and weights, and the z rows (straight into the unit's buffer)
+                // cp.async of head hh's v channel rows and weights (into the staging area) and
+                // z rows (straight into unit buffer ub)
+                auto stage_unit = [&](int hh, int ub) {
+                    const size_t cv = (size_t)2 * Hk * kDK + (size_t)hh * kDV;
+                    uint16_t* zb2 = reinterpret_cast<uint16_t*>(heads + ub * kHeadFloats + kCT * kDV + 4 * kCT +
+                                                                2 * kCT * kCT);
                     for (int e = i; e < nrow * 16; e += kProducers) {
                         const int r = e >> 4, off = (e & 15) * 8;
-                        cp_async_16(uraw + r * kDV + off, r < W - 1 ? hist + (size_t)r * C + chv + off
-                                                                    : x + (size_t)(r - (W - 1)) * C + chv + off);
+                        cp_async_16(uraw + r * kDV + off, r < W - 1 ? hist + (size_t)r * C + cv + off
+                                                                    : x + (size_t)(r - (W - 1)) * C + cv + off);
                     }
-                    for (int e = i; e < kDV * W / 8; e += kProducers) cp_async_16(uw + e * 8, p.conv_w + chv * W + e * 8);
+                    for (int e = i; e < kDV * W / 8; e += kProducers) cp_async_16(uw + e * 8, p.conv_w + cv * W + e * 8);
                     for (int e = i; e < n * 16; e += kProducers) {
                         const int t = e >> 4, off = (e & 15) * 8;
-                        cp_async_16(hz + t * kDV + off, p.z + (((size_t)tok0 + t) * Hv + h) * kDV + off);
+                        cp_async_16(zb2 + t * kDV + off, p.z + (((size_t)tok0 + t) * Hv + hh) * kDV + off);
                     }
-                    cp_async_wait_all();
-                }
+                    ustaged = hu + (hh - h);
+                };
+                if (ustaged != hu) stage_unit(h, hb);  // (later heads were staged while the one before ran)
+                cp_async_wait_all();
                 named_barrier(kProducerBar, kProducers);
                 if (i < kDV) {  // v channel i of this head (step 3)
                     float vv[kCT];
@@ -453,28 +480,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 }
                 named_barrier(kProducerBar, kProducers);
                 // the solve's coefficients: A_ts = beta_t g_ts k_t.k_s (s < t), M_ts = g_ts q_t.k_s (s <= t)
-                {
+                {  // the decays in registers: every product below is a chain of selects and multiplies
+                    float al[kCT];
+#pragma unroll
+                    for (int b4 = 0; b4 < kCT / 4; ++b4) {
+                        const float4 a4 = reinterpret_cast<const float4*>(ha)[b4];
+                        al[4 * b4] = a4.x; al[4 * b4 + 1] = a4.y; al[4 * b4 + 2] = a4.z; al[4 * b4 + 3] = a4.w;
+                    }
                     const int e = i, t = e >> 4, s = e & 15;  // one coefficient pair per thread
-                    float gts = 1.f;
-                    for (int u = s + 1; u <= t; ++u) gts *= ha[u];
+                    float gts = 1.f;                           // alpha_{s+1} .. alpha_t
+#pragma unroll
+                    for (int u = 1; u < kCT; ++u) gts *= (u > s && u <= t) ? al[u] : 1.f;
                     hA[e] = s < t ? hbeta[t] * gts * KK[e] : 0.f;
                     hM[e] = s <= t ? gts * QK[e] : 0.f;
-                }
-                if (i < kCT) {  // gamma_t = alpha_0..alpha_t; w_s = alpha_{s+1}..alpha_{n-1}
-                    float gm = 1.f, w = 1.f;
-                    for (int u = 0; u <= i; ++u) gm *= ha[u];
-                    for (int u = i + 1; u < n; ++u) w *= ha[u];
-                    hgam[i] = gm;
-                    hw[i] = i < n ? w : 0.f;
+                    if (i < kCT) {  // gamma_t = alpha_0..alpha_t; w_s = alpha_{s+1}..alpha_{n-1}
+                        float gm = 1.f, w = 1.f;
+#pragma unroll
+                        for (int u = 0; u < kCT; ++u) {
+                            gm *= u <= i ? al[u] : 1.f;
+                            w *= (u > i && u < n) ? al[u] : 1.f;
+                        }
+                        hgam[i] = gm;
+                        hw[i] = i < n ? w : 0.f;
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(unit_full + hb);
+                if (j + 1 < G) {  // the next head: its buffer's previous unit leaves, its rows start
+                    const int nb = (hu + 1) & 1;
+                    const bool ok2 = hu < 1 || wait(unit_empty + nb, (uint32_t)(((hu - 1) >> 1) & 1));
+                    if (!named_barrier_and(kProducerBar, kProducers, ok2 && !*abort_flag)) {
+                        if (!ok2) fail();
+                        stop = true;
+                        break;
+                    }
+                    if (hu >= 1 && emitted < hu - 1) {
+                        emit_unit(nb);
+                        emitted = hu - 1;
+                    }
+                    named_barrier(kProducerBar, kProducers);  // the buffer and the staging area are free
+                    stage_unit(h + 1, nb);
+                }
             }
             if (stop) break;
         }
         // the last two units' outputs (every producer takes the same decision)
         if (named_barrier_and(kProducerBar, kProducers, !*abort_flag))
-            for (int u = hu >= 2 ? hu - 2 : 0; u < hu; ++u) {
+            for (int u = emitted + 1; u < hu; ++u) {
                 const bool got = wait(unit_empty + (u & 1), (uint32_t)((u >> 1) & 1));
                 if (!named_barrier_and(kProducerBar, kProducers, got && !*abort_flag)) {
                     if (!got) fail();
@@ -482,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 }
                 emit_unit(u & 1);
             }
+        cp_async_wait_all();  // no copy of this thread lands after the CTA has left
     } else {
         // ---- consumers: thread c owns state column c (TMEM lane c). A wait that gives
         // up is agreed on at the next consumer barrier, where all four warps leave

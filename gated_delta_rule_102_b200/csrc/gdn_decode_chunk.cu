@@ -210,6 +210,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         bad_len = n < 0 || n > T || (p.cu_seqlens && (tok0 < 0 || tok0 + n > p.total_rows));
         return !bad_slot && !bad_len && n > 0;
     };
+    // The same, split in two: the loads of a group's slot and offsets (issued one group ahead,
+    // so their latency passes while the group before runs), then the decision.
+    struct GroupRaw {
+        int slot, tok0, end;
+    };
+    auto group_fetch = [&](int g) {
+        GroupRaw r{-1, 0, 0};
+        if (g >= ngroups) return r;
+        const int seq = g / Hk;
+        r.slot = __ldg(p.slots + seq);
+        if (p.cu_seqlens) {
+            r.tok0 = __ldg(p.cu_seqlens + seq);
+            r.end = __ldg(p.cu_seqlens + seq + 1);
+        } else {
+            r.tok0 = seq * T;
+            r.end = r.tok0 + T;
+        }
+        return r;
+    };
+    auto group_eval = [&](const GroupRaw& r, int& slot, int& tok0, int& n, bool& bad_slot, bool& bad_len) {
+        slot = r.slot;
+        tok0 = r.tok0;
+        n = r.end - r.tok0;
+        bad_slot = slot < 0 || slot >= p.P;
+        bad_len = n < 0 || n > T || (p.cu_seqlens && (tok0 < 0 || tok0 + n > p.total_rows));
+        return !bad_slot && !bad_len && n > 0;
+    };
 
     if (warp >= kConsumerWarps) {
         // ---- producers: thread i handles conv channel i of the group's q | k (256) and, for
@@ -269,10 +296,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + oi) = make_float4(y0, y1, y2, y3);
             }
         };
-        for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
+        GroupRaw cur = group_fetch(blockIdx.x), nxt;
+        int gn = 0;
+        for (int g = blockIdx.x; g < ngroups; g = gn, cur = nxt) {
+            gn = g + (int)gridDim.x;
+            nxt = group_fetch(gn);  // used by the next iteration
             int slot, tok0, n;
             bool bad_slot, bad_len;
-            const bool run = group_info(g, slot, tok0, n, bad_slot, bad_len);
+            const bool run = group_eval(cur, slot, tok0, n, bad_slot, bad_len);
             if (i == 0 && p.err_flag && bad_slot) atomicOr(p.err_flag, GDN_DEVICE_ERR_SLOT_RANGE_BIT);
             if (i == 0 && p.err_flag && bad_len) atomicOr(p.err_flag, GDN_DEVICE_ERR_SEQLEN_BIT);
             if (!run) continue;
@@ -287,11 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             const uint16_t* x = p.qkv + (size_t)tok0 * C;
             const int nrow = W - 1 + n;
             uint16_t* gw = graw + kRawRows * 2 * kDK;  // weights [256][W]
-            // the next group this CTA runs, looked up now (its loads travel during the conv)
-            int g2 = g + (int)gridDim.x, s2 = 0, t2 = 0, n2 = 0;
+            // the next group this CTA runs (normally the one fetched ahead)
+            int g2 = gn, s2 = 0, t2 = 0, n2 = 0;
             {
                 bool b2s, b2l;
-                while (g2 < ngroups && !group_info(g2, s2, t2, n2, b2s, b2l)) g2 += (int)gridDim.x;
+                if (g2 < ngroups && !group_eval(nxt, s2, t2, n2, b2s, b2l))
+                    for (g2 += (int)gridDim.x; g2 < ngroups && !group_info(g2, s2, t2, n2, b2s, b2l);)
+                        g2 += (int)gridDim.x;
             }
             if (gstaged != g) stage_group(g, slot, tok0, n);  // (normally staged while the group before ran)
             cp_async_wait_all();
@@ -583,10 +616,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 for (int q = 0; q < kChunksPerTile; ++q)
                     issue_chunk(p.state_pool + ((size_t)sl * Hv + (g0 % Hk) * G) * kTileElems, q);
         }
-        for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
+        GroupRaw cur = group_fetch(blockIdx.x), nxt;
+        int gn = 0;
+        for (int g = blockIdx.x; g < ngroups; g = gn, cur = nxt) {
+            gn = g + (int)gridDim.x;
+            nxt = group_fetch(gn);  // used by the next iteration
             int slot, tok0, n;
             bool bad_slot, bad_len;
-            if (!group_info(g, slot, tok0, n, bad_slot, bad_len)) continue;
+            if (!group_eval(cur, slot, tok0, n, bad_slot, bad_len)) continue;
             const int gb = li & 1, hk = g % Hk;
             const bool got = wait(grp_full + gb, (uint32_t)((li >> 1) & 1));
             if (!named_barrier_and(kConsumerBar, 128, got && !*abort_flag)) {
@@ -605,8 +642,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 const float* hA = hw + kCT;
                 const float* hM = hA + kCT * kCT;
                 if (c == kCopier) {
-                    int sl2 = slot;
-                    const int g2 = j + 1 < G ? g : next_group(g + (int)gridDim.x, sl2);
+                    int sl2 = slot, g2 = g;
+                    if (j + 1 >= G) {  // the next group: normally the one fetched ahead
+                        int t2, n2;
+                        bool b2s, b2l;
+                        g2 = gn;
+                        if (g2 < ngroups && !group_eval(nxt, sl2, t2, n2, b2s, b2l)) g2 = next_group(gn + (int)gridDim.x, sl2);
+                    }
                     next_tile = g2 < ngroups
                                     ? p.state_pool + ((size_t)sl2 * Hv + (g2 % Hk) * G + (g2 == g ? j + 1 : 0)) * kTileElems
                                     : nullptr;

@@ -86,16 +86,15 @@ def kernel_for(wl, num_sms: int) -> str:
     (one CTA per SM, G CTAs per cluster), else the cluster-per-group kernels."""
     G = wl.num_v_heads // wl.num_k_heads
     if wl.ragged:
-        return "decode_mt_kernel"
+        return multitoken_kernel_for(wl)
     if wl.tokens == 1 and wl.batch * wl.num_k_heads >= 2 * (num_sms // G):
         return "decode_ws_kernel"
     return "decode_fused_tma_kernel" if wl.tokens == 1 else multitoken_kernel_for(wl)
 
 
 def multitoken_kernel_for(wl) -> str:
-    """Several tokens per sequence, every sequence the same count (and every speculative
-    verify): the chunked tensor-core kernel for dk = dv = 128, the register-tile kernel
-    otherwise and for ragged launches."""
+    """Several tokens per sequence (ragged launches and every speculative verify included):
+    the chunked tensor-core kernel for dk = dv = 128, the register-tile kernel otherwise."""
     return "decode_chunk_kernel" if wl.head_k_dim == 128 and wl.head_v_dim == 128 else "decode_mt_kernel"
 
 

@@ -870,12 +870,12 @@ cudaError_t chunk_grid_cap(int* cap) {
 
 }  // namespace
 
-// Uniform launches only: the chunk form costs a whole state tile per (sequence, head)
-// whatever its token count, so ragged launches (many short sequences) stay on the
-// register kernel, whose cost follows the tokens (measured 119 against 136 µs on 64
-// sequences of 0..16 tokens; level at 16 tokens each).
+// Every multi-token launch at dk = dv = 128, ragged ones included: a sequence without
+// tokens costs nothing, one with fewer than 16 costs a whole tile like one with 16, and still
+// the chunk form measured ahead of the register kernel on 64 sequences of 0..16 tokens (108
+// against 119 us).
 bool chunk_supported(const DecodeArgs& a) {
-    return a.cu_seqlens == nullptr && a.sh.dk == kDK && a.sh.dv == kDV && a.T >= 1 && a.T <= kCT && a.sh.W >= 1 &&
+    return a.sh.dk == kDK && a.sh.dv == kDV && a.T >= 1 && a.T <= kCT && a.sh.W >= 1 &&
            a.sh.W <= kMaxConvWidth && a.sh.Hk >= 1 && a.sh.Hv % a.sh.Hk == 0;
 }
 

@@ -26,10 +26,10 @@ def test_kernel_choice_per_workload():
     assert b.kernel_for(w["pool384_batch256"], 148) == "decode_ws_kernel"
     assert b.kernel_for(w["single_seq"], 148) == "decode_fused_tma_kernel"
     assert b.kernel_for(w["tiny_d16"], 148) == "decode_fused_tma_kernel"
-    # several tokens per sequence: the chunked tensor-core kernel at dk = dv = 128 for
-    # uniform launches, else (and for ragged ones) the register-tile kernel
+    # several tokens per sequence: the chunked tensor-core kernel at dk = dv = 128, else the
+    # register-tile kernel
     assert b.kernel_for(w["multitoken_b32_t16"], 148) == "decode_chunk_kernel"
-    assert b.kernel_for(w["ragged_b64_t16"], 148) == "decode_mt_kernel"
+    assert b.kernel_for(w["ragged_b64_t16"], 148) == "decode_chunk_kernel"
     assert b.kernel_for(w["multitoken_b32_t16"].replace(head_v_dim=64), 148) == "decode_mt_kernel"
 
 

@@ -104,6 +104,9 @@ def algorithmic_flops(wl) -> int:
     return 7 * wl.batch * wl.tokens * wl.num_v_heads * wl.head_k_dim * wl.head_v_dim
 
 
+# Kernels whose contractions run on the tensor cores: their roofline is HBM, never the FP32 FMA peak.
+TENSOR_CORE_KERNELS = ("decode_chunk_kernel", "proj_gemm_kernel")
+
 # The sources each decode kernel is compiled from (its own file and the shared headers).
 KERNEL_SOURCES = {
     "decode_ws_kernel": ("gdn_decode_persistent.cu",),
@@ -568,7 +571,7 @@ def run_extra(args, name, rank, world):
             "algorithmic_bytes": int(nbytes), "algorithmic_flops": int(flops),
             "tflops_achieved": flops / step_s / 1e12}
     sm_mhz = (clocks or {}).get("sm_mhz")
-    if kind == "spec" and sm_mhz:
+    if kind == "spec" and sm_mhz and kernel not in TENSOR_CORE_KERNELS:
         alu_peak = num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6
         alu = flops / step_s / 1e12
         if alu / alu_peak > roof["frac"]:
@@ -866,7 +869,11 @@ def main():
             "traffic": profiled_traffic(kernel, wl.name), "peak_source": f"{peak_kind} copy bandwidth"}
     flops = whole(statistics.fmean(set_cost[i][1] for i in step_sets))
     sm_mhz = (clocks or {}).get("sm_mhz")
-    if sm_mhz and flops / (kernel_ms / 1e3) / 1e12 / (num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6) > roof["frac"]:
+    if kernel in TENSOR_CORE_KERNELS:
+        # the delta rule's contractions run on the tensor cores (split tf32): the FP32 FMA
+        # roofline does not apply; the kernel is designed against HBM
+        roof["peak_note"] = "contractions on the tensor cores: HBM roofline"
+    elif sm_mhz and flops / (kernel_ms / 1e3) / 1e12 / (num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6) > roof["frac"]:
         # closer to the FP32 FMA peak (SMs x 128 lanes x 2 flops x the median SM clock
         # sampled in the timed region) than to the copy bandwidth: ALU-bound
         alu_peak = num_sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e-6

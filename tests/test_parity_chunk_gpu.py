@@ -36,6 +36,7 @@ CASES = [
     ("c_g2_t16_many_groups", 16, 32, 4, 20, 5, 24, 2, 0.02, "normal"),  # 320 groups: 2-3 per CTA
     ("c_big_state_t16", 2, 4, 4, 3, 16, 4, 2, 1.0, "normal"),
     ("c_wide_decay_t7", 2, 4, 4, 3, 7, 4, 2, 0.02, "decay_wide"),
+    ("c_g8_t6", 1, 8, 4, 3, 6, 4, 2, 0.02, "normal"),        # eight v-heads per k-head
 ]
 
 

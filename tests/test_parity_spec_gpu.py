@@ -106,6 +106,7 @@ SHAPES = [
     ("spec_t1", 2, 4, 32, 32, 2, 4, 1, 5, "normal"),
     ("spec_w8_t7", 2, 4, 32, 64, 8, 4, 7, 5, "normal"),
     ("spec_wide_t16", 2, 4, 128, 128, 4, 4, 16, 5, "decay_wide"),
+    ("spec_d128_t1", 2, 4, 128, 128, 4, 3, 1, 5, "normal"),  # one drafted token, the chunked kernel
 ]
 
 

@@ -114,6 +114,9 @@ static_assert(TM_YLO + kCT <= kTmemCols, "TMEM columns");
 __device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xFFFFE000u; }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// all of this thread's committed copy groups but the newest have landed
+__device__ __forceinline__ void cp_async_wait_all_but_newest() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // conv + SiLU of one channel from its staged inputs: rows[r * stride] for r < W-1 the
 // history, then the n <= 16 tokens; w: its W weights. out[t] for t < n, 0 beyond.
@@ -246,7 +249,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         int li = 0, hu = 0;  // groups and units produced
         int gstaged = -1;    // the group whose q/k rows and weights are in (or on their way to) graw
         int emitted = -1;    // the last unit whose outputs are written
-        int ustaged = -1;    // the unit whose v rows, weights and z rows are staged
         // cp.async of group gg's q and k channels: their history and token rows (16-byte
         // pieces, two runs of 128 channels per row) and weights (two runs of 128 W)
         auto stage_group = [&](int gg, int sl, int t0, int nn) {
@@ -265,14 +267,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 const int part = e >= wpieces, o = e - part * wpieces;
                 cp_async_16(gwt + part * kDK * W + o * 8, p.conv_w + (size_t)(part * Hk + kh) * kDK * W + o * 8);
             }
+            cp_async_commit();
             gstaged = gg;
         };
+        // the RMSNorm weights of this lane's four columns (the same for every unit)
+        const uint2 nw4 = __ldg(reinterpret_cast<const uint2*>(p.norm_w) + lane);
+        const float nw[4] = {bf16_bits_to_float(nw4.x & 0xffffu), bf16_bits_to_float(nw4.x >> 16),
+                             bf16_bits_to_float(nw4.y & 0xffffu), bf16_bits_to_float(nw4.y >> 16)};
         // step 8 and the SiLU(z) gate of a solved unit in buffer ub: a warp per token, four
         // columns per lane
         auto emit_unit = [&](int ub) {
-            const uint2 nw4 = __ldg(reinterpret_cast<const uint2*>(p.norm_w) + lane);
-            const float nw[4] = {bf16_bits_to_float(nw4.x & 0xffffu), bf16_bits_to_float(nw4.x >> 16),
-                                 bf16_bits_to_float(nw4.y & 0xffffu), bf16_bits_to_float(nw4.y >> 16)};
             const float* ov = heads + ub * kHeadFloats;
             const uint16_t* oz = reinterpret_cast<const uint16_t*>(ov + kCT * kDV + 4 * kCT + 2 * kCT * kCT);
             const int* meta = reinterpret_cast<const int*>(ov + kHeadFloats - 4);
@@ -318,14 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             const uint16_t* x = p.qkv + (size_t)tok0 * C;
             const int nrow = W - 1 + n;
             uint16_t* gw = graw + kRawRows * 2 * kDK;  // weights [256][W]
-            // the next group this CTA runs (normally the one fetched ahead)
-            int g2 = gn, s2 = 0, t2 = 0, n2 = 0;
-            {
-                bool b2s, b2l;
-                if (g2 < ngroups && !group_eval(nxt, s2, t2, n2, b2s, b2l))
-                    for (g2 += (int)gridDim.x; g2 < ngroups && !group_info(g2, s2, t2, n2, b2s, b2l);)
-                        g2 += (int)gridDim.x;
-            }
             if (gstaged != g) stage_group(g, slot, tok0, n);  // (normally staged while the group before ran)
             cp_async_wait_all();
             named_barrier(kProducerBar, kProducers);
@@ -341,7 +337,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                             graw[(n + r) * 2 * kDK + lc];
             }
             named_barrier(kProducerBar, kProducers);
-            if (g2 < ngroups) stage_group(g2, s2, t2, n2);  // the staging buffer is free: the next group's rows
+            {  // the staging buffer is free: the rows of the next group this CTA runs (normally the one
+               // fetched ahead, whose slot and offsets have arrived during the conv)
+                int g2 = gn, s2 = 0, t2 = 0, n2 = 0;
+                bool b2s, b2l;
+                if (g2 < ngroups && !group_eval(nxt, s2, t2, n2, b2s, b2l))
+                    for (g2 += (int)gridDim.x; g2 < ngroups && !group_info(g2, s2, t2, n2, b2s, b2l);)
+                        g2 += (int)gridDim.x;
+                if (g2 < ngroups) stage_group(g2, s2, t2, n2);
+            }
             // L2 norms of q and k per token (step 3): factors on the raw values
 #pragma unroll
             for (int m = 0; m < kCT / kProducerWarps; ++m) {  // a warp per token
@@ -438,6 +442,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             const float* KK = gram + gb * 2 * kCT * kCT;
             const float* QK = KK + kCT * kCT;
             bool stop = false;
+            const int gi = i - kDK;  // threads 128..143: the gates of token gi
+            // cp.async of head hh's v channel rows and weights into the staging area (free once every
+            // producer has passed the group's Gram products, or the last head's v conv)
+            uint16_t* uw = uraw + kRawRows * kDV;  // weights [128][W]
+            auto stage_v = [&](int hh) {
+                const size_t cv = (size_t)2 * Hk * kDK + (size_t)hh * kDV;
+                for (int e = i; e < nrow * 16; e += kProducers) {
+                    const int r = e >> 4, off = (e & 15) * 8;
+                    cp_async_16(uraw + r * kDV + off, r < W - 1 ? hist + (size_t)r * C + cv + off
+                                                            : x + (size_t)(r - (W - 1)) * C + cv + off);
+                }
+                for (int e = i; e < kDV * W / 8; e += kProducers) cp_async_16(uw + e * 8, p.conv_w + cv * W + e * 8);
+                cp_async_commit();
+            };
+            // cp.async of head hh's z rows into unit buffer ub (free once its last unit is emitted)
+            auto stage_z = [&](int hh, int ub) {
+                uint16_t* zb2 =
+                    reinterpret_cast<uint16_t*>(heads + ub * kHeadFloats + kCT * kDV + 4 * kCT + 2 * kCT * kCT);
+                for (int e = i; e < n * 16; e += kProducers) {
+                    const int t = e >> 4, off = (e & 15) * 8;
+                    cp_async_16(zb2 + t * kDV + off, p.z + (((size_t)tok0 + t) * Hv + hh) * kDV + off);
+                }
+                cp_async_commit();
+            };
+            // the gate inputs of head hh's tokens (loaded one head ahead within the group)
+            uint16_t ga = 0, gbb = 0;
+            auto load_gates = [&](int hh) {
+                if (gi >= 0 && gi < kCT && gi < n) {
+                    const size_t ai = ((size_t)tok0 + gi) * Hv + hh;
+                    ga = p.a[ai];
+                    gbb = p.b[ai];
+                }
+            };
             for (int j = 0; j < G; ++j, ++hu) {
                 const int hb = hu & 1, h = hk * G + j;
                 ok = hu < 2 || wait(unit_empty + hb, (uint32_t)(((hu >> 1) - 1) & 1));
@@ -445,6 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     if (!ok) fail();
                     stop = true;
                     break;
+                }
+                if (j == 0) {  // the group's first head: its v rows and gate inputs travel under the emit
+                    stage_v(h);
+                    load_gates(h);
                 }
                 if (hu >= 2 && emitted < hu - 2) {  // the unit solved two units ago leaves the buffer first
                     emit_unit(hb);
@@ -465,35 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     meta[2] = n;
                 }
                 const size_t chv = (size_t)2 * Hk * kDK + (size_t)h * kDV;
-                uint16_t* uw = uraw + kRawRows * kDV;  // weights [128][W]
-                // the gate inputs of this head's tokens, loaded now and used after the staging
-                const int gi = i - kDK;  // threads 128..143: the gates of token gi
-                uint16_t ga = 0, gbb = 0;
-                if (gi >= 0 && gi < kCT && gi < n) {
-                    const size_t ai = ((size_t)tok0 + gi) * Hv + h;
-                    ga = p.a[ai];
-                    gbb = p.b[ai];
-                }
-                // cp.async of head hh's v channel rows and weights (into the staging area) and
-                // z rows (straight into unit buffer ub)
-                auto stage_unit = [&](int hh, int ub) {
-                    const size_t cv = (size_t)2 * Hk * kDK + (size_t)hh * kDV;
-                    uint16_t* zb2 = reinterpret_cast<uint16_t*>(heads + ub * kHeadFloats + kCT * kDV + 4 * kCT +
-                                                                2 * kCT * kCT);
-                    for (int e = i; e < nrow * 16; e += kProducers) {
-                        const int r = e >> 4, off = (e & 15) * 8;
-                        cp_async_16(uraw + r * kDV + off, r < W - 1 ? hist + (size_t)r * C + cv + off
-                                                                    : x + (size_t)(r - (W - 1)) * C + cv + off);
-                    }
-                    for (int e = i; e < kDV * W / 8; e += kProducers) cp_async_16(uw + e * 8, p.conv_w + cv * W + e * 8);
-                    for (int e = i; e < n * 16; e += kProducers) {
-                        const int t = e >> 4, off = (e & 15) * 8;
-                        cp_async_16(zb2 + t * kDV + off, p.z + (((size_t)tok0 + t) * Hv + hh) * kDV + off);
-                    }
-                    ustaged = hu + (hh - h);
-                };
-                if (ustaged != hu) stage_unit(h, hb);  // (later heads were staged while the one before ran)
-                cp_async_wait_all();
+                if (j == 0) stage_z(h, hb);  // (later heads' z rows were staged while the one before ran)
+                // this head's v rows have landed; its z rows, the newest copies, may still be on their
+                // way: they are read only by the emit, after another wait of this kind or the drain's
+                cp_async_wait_all_but_newest();
                 named_barrier(kProducerBar, kProducers);
                 if (i < kDV) {  // v channel i of this head (step 3)
                     float vv[kCT];
@@ -512,6 +528,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     hbeta[gi] = be;
                 }
                 named_barrier(kProducerBar, kProducers);
+                if (j + 1 < G) {  // the staging area is free: the next head's v rows and gate inputs
+                    stage_v(h + 1);
+                    load_gates(h + 1);
+                }
                 // the solve's coefficients: A_ts = beta_t g_ts k_t.k_s (s < t), M_ts = g_ts q_t.k_s (s <= t)
                 {  // the decays in registers: every product below is a chain of selects and multiplies
                     float al[kCT];
@@ -539,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(unit_full + hb);
-                if (j + 1 < G) {  // the next head: its buffer's previous unit leaves, its rows start
+                if (j + 1 < G) {  // the next head's buffer: its previous unit leaves, its z rows start
                     const int nb = (hu + 1) & 1;
                     const bool ok2 = hu < 1 || wait(unit_empty + nb, (uint32_t)(((hu - 1) >> 1) & 1));
                     if (!named_barrier_and(kProducerBar, kProducers, ok2 && !*abort_flag)) {
@@ -551,13 +571,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         emit_unit(nb);
                         emitted = hu - 1;
                     }
-                    named_barrier(kProducerBar, kProducers);  // the buffer and the staging area are free
-                    stage_unit(h + 1, nb);
+                    named_barrier(kProducerBar, kProducers);  // the buffer's z rows are read
+                    stage_z(h + 1, nb);
                 }
             }
             if (stop) break;
         }
-        // the last two units' outputs (every producer takes the same decision)
+        // the last two units' outputs (every producer takes the same decision; their z rows have
+        // landed before the barrier)
+        cp_async_wait_all();
         if (named_barrier_and(kProducerBar, kProducers, !*abort_flag))
             for (int u = emitted + 1; u < hu; ++u) {
                 const bool got = wait(unit_empty + (u & 1), (uint32_t)((u >> 1) & 1));
@@ -579,7 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         int li = 0, hu = 0, chunk = 0;
         uint32_t mma_issued = 0, mma_seen = 0;  // update commits issued (counted by all) and waited for (own)
         uint32_t g1_seen = 0;                   // first-GEMM phases waited for (own)
-        bool g1_open = false;                   // (threads 0, 32) MMAs issued since their last commit
         float* pend = nullptr;                  // column c of the state tile still in the accumulator
         bool ok = true;
         auto store_chunk = [&](int q) {         // rows 32q .. 32q+31 of the pending tile
@@ -656,10 +677,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 bool w = wait(unit_full + hb, (uint32_t)((hu >> 1) & 1));
                 const float gC = hgam[n - 1];
                 // ---- the state tile into TMEM chunk by chunk (S0^T high and low parts, and
-                // gamma_{n-1} S0^T in the accumulator); each chunk's MMAs of S0^T [k | q]^T are
-                // issued as soon as it is in: the high part of S0 against the high and low
-                // operand tiles side by side (N = 64), then its low part against the high
-                // tiles (N = 32, into the first 32 columns); K = 8 per MMA
+                // gamma_{n-1} S0^T in the accumulator); after each chunk's barrier the next
+                // unit's chunk q is copied into the buffer just read
                 for (int q = 0; q < kChunksPerTile; ++q, ++chunk) {
                     const int s = chunk % kRing;
                     w = w && wait(ring_full + s, (uint32_t)((chunk / kRing) & 1));
@@ -687,12 +706,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         ok = false;
                         break;
                     }
-                    // the chunk's MMAs from two threads of different warps, each into its own
-                    // accumulator (a fixed order per accumulator), and the next unit's chunk q
-                    // from a third
                     if (c == kCopier && next_tile) issue_chunk(next_tile, q);  // every consumer has read buffer q
-                    if (c == 0 || c == 32) {
-                        tcgen05_fence_after();
+                }
+                if (!ok) break;
+                // the first GEMM, S0^T [k | q]^T, once the whole tile is in (the consumers' barriers
+                // are not held up by its issue): the high part of S0 against the high and low operand
+                // tiles side by side (N = 64) from thread 0, its low part against the high tiles
+                // (N = 32) from thread 32, each into its own accumulator (a fixed order per
+                // accumulator); K = 8 per MMA
+                if (c == 0 || c == 32) {
+                    tcgen05_fence_after();
+#pragma unroll 1
+                    for (int q = 0; q < kChunksPerTile; ++q) {
                         const uint64_t bx = sw128_desc(xb + q * kXRegion);
                         if (c == 0) {
                             constexpr uint32_t idesc64 = idesc_tf32(4 * kCT, 0);
@@ -707,14 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                                 umma_tf32_ts(tmem + TM_D1B, tmem + TM_ALO + 32 * q + 8 * kk, bx + (uint64_t)(2 * kk),
                                              idesc32, (q | kk) != 0 ? 1u : 0u);
                         }
-                        g1_open = true;
-                        if (q == kChunksPerTile - 1) {
-                            umma_commit(smem_addr(g1_bar));
-                            g1_open = false;
-                        }
                     }
+                    umma_commit(smem_addr(g1_bar));
                 }
-                if (!ok) break;
                 pend = nullptr;
                 float vv[kCT];
 #pragma unroll
@@ -829,10 +849,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             // an MMA batch that was issued and never waited for completes before TMEM is freed,
             // and the state copies still in flight land before the CTA leaves
             if (c == 0 && mma_issued > mma_seen) mbar_wait_bounded(mma_bar, mma_seen & 1u);
-            if ((c == 0 || c == 32) && g1_open) {  // a first GEMM left half-issued: close it and wait
-                umma_commit(smem_addr(g1_bar));
-                mbar_wait_bounded(g1_bar, g1_seen & 1u);
-            }
             if (c == kCopier)
                 for (int v = chunk; v < issued; ++v) mbar_wait_bounded(ring_full + v % kRing, (uint32_t)((v / kRing) & 1));
         }

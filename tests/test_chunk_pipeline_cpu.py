@@ -6,11 +6,14 @@ One CTA walks its (sequence, k-head) groups; a group's v-heads are its units. Fo
 share the CTA's buffers:
   * the producers (warps 4-11, one agent: their named barriers keep them together) fill
     the group operand tiles X and Z (double-buffered) and the unit buffers (v, the solve's
-    coefficients, z; double-buffered), and emit each unit's gated RMSNorm from o;
+    coefficients, z; double-buffered), and emit each unit's gated RMSNorm from o; their raw
+    rows arrive by cp.async in committed groups (a group's q|k rows, a head's v rows into
+    the staging area that aliases the group scratch, a head's z rows into its unit buffer)
+    that land at some later time, and at the latest when a wait_group asks for them;
   * the consumers (warps 0-3, one agent) take each unit's state tile from the copy ring
-    into TMEM, issue the two GEMMs, solve, write o, and store the new state while the next
-    unit's tile goes in; thread 64 among them issues the bulk copies of the next unit's
-    chunks into the ring;
+    into TMEM chunk by chunk, issue the first GEMM once the tile is in, solve, write o, issue
+    the update, and store the new state while the next unit's tile goes in; thread 64 among
+    them issues the bulk copy of the next unit's chunk q once chunk q has been read;
   * the bulk-copy engine lands a copy at some later time and completes its ring barrier;
   * the tensor core runs each issuing thread's MMAs and commits in order, at some later time.
 An mbarrier wait with parity P passes when the barrier's completed-phase count has the
@@ -20,7 +23,8 @@ shows up as a premature pass (caught by the data checks) or a deadlock.
 Checked for every schedule: no deadlock; no buffer (ring chunk, operand tile, unit buffer,
 TMEM column block) rewritten before its reader is done with it, asynchronous readers
 included; every read sees the data meant for it (ring chunks by the state tile they hold:
-pool slot and v-head); every unit's outputs emitted once and its state stored once; no
+pool slot and v-head; staged rows by their group or head), no v rows landing in the scratch
+while a group phase uses it; every unit's outputs emitted once and its state stored once; no
 copy or MMA left in flight at the end; each group's and unit's rows staged once (the
 look-ahead always right). Each planted protocol mistake must be caught by some schedule."""
 import collections
@@ -73,17 +77,44 @@ class CTA:
         self.emitted, self.stored = collections.Counter(), collections.Counter()
         self.group_stagings, self.unit_stagings = collections.Counter(), collections.Counter()
         self.graw = None
+        self.uraw = None   # the head whose v rows are in the staging area
+        self.cp = []       # committed cp.async groups in commit order: [kind, landing action, landed]
 
     def tile(self, g, j):
         return (self.slot[g], (g % self.Hk) * self.G + j)
 
     # ---- producer-side data actions
+    def copy(self, kind, action):
+        self.cp.append([kind, action, False])
+
+    def cp_in_flight(self):
+        return [c for c in self.cp if not c[2]]
+
+    def land_group(self, c):
+        c[1]()
+        c[2] = True
+
+    def cp_wait(self, keep):
+        """cp.async.wait_group keep: every committed group but the `keep` most recently
+        committed ones (landed or not) has landed."""
+        for c in self.cp[:len(self.cp) - keep]:
+            if not c[2]:
+                self.land_group(c)
+
     def stage_group(self, g):
         self.group_stagings[g] += 1
-        self.graw = g
+        self.copy("group", lambda: setattr(self, "graw", g))
 
     def conv_group(self, g):
         assert self.graw == g, "conv of a group whose rows are not staged"
+        assert not any(c[0] == "v" for c in self.cp_in_flight()), "v rows landing in the scratch during the group phase"
+
+    def stage_v(self, h):
+        self.uraw = None
+        self.copy("v", lambda: setattr(self, "uraw", h))
+
+    def conv_v(self, h):
+        assert self.uraw == h, "v conv of a head whose rows have not landed"
 
     def write_group(self, gb, li):
         b = self.xz[gb]
@@ -93,11 +124,12 @@ class CTA:
             assert b["z_done"] == (0 if self.spec else self.G), "key tile rewritten before every update read it"
         b.update(tag=li, x_done=0, z_done=0)
 
-    def stage_unit(self, b, u):
+    def stage_z(self, b, u):
         self.unit_stagings[u] += 1
         prev = self.unit[b]["z"]
         assert prev is None or self.emitted[self.p_keys[prev]], "z rows overwritten before their unit was emitted"
-        self.unit[b]["z"] = u
+        self.unit[b]["z"] = None  # (in flight)
+        self.copy("z", lambda: self.unit[b].__setitem__("z", u))
 
     def write_unit(self, b, u):
         prev = self.unit[b]["v"]
@@ -184,6 +216,9 @@ class CTA:
             self.y_out -= 1
             self.d2 = [("upd", u)] * CHUNKS
 
+    def land_copy(self, k):
+        self.land_group(self.cp_in_flight()[k])
+
     def land(self, k):
         q, tile = self.tma.pop(k)
         self.ring[q].update(tile=tile, inflight=False, read=False)
@@ -193,7 +228,7 @@ class CTA:
     def producer(self):
         Hk, G, grid, ng = self.Hk, self.G, self.grid, self.ngroups
         li = hu = 0
-        emitted = ustaged = gstaged = -1
+        emitted = gstaged = -1
         for g in range(self.cta, ng, grid):
             gn = g + grid
             if not self.valid[g]:
@@ -201,15 +236,16 @@ class CTA:
             gb, hk = li & 1, g % Hk
             if li >= 2:
                 yield f"grp_empty{gb}", ((li >> 1) - 1) & 1
-            g2 = gn  # the next group this CTA runs
+            if gstaged != g:
+                self.stage_group(g)
+                gstaged = g
+            self.cp_wait(0)
+            self.conv_group(g)
+            g2 = gn  # the next group this CTA runs: its rows into the staging buffer just read
             if g2 < ng and not self.valid[g2]:
                 g2 += grid
                 while g2 < ng and not self.valid[g2]:
                     g2 += grid
-            if gstaged != g:
-                self.stage_group(g)
-                gstaged = g
-            self.conv_group(g)
             if g2 < ng:
                 self.stage_group(g2)
                 gstaged = g2
@@ -222,27 +258,34 @@ class CTA:
                 if hu >= 2 and self.mistake != "no_unit_empty_wait":
                     par = (hu >> 1) & 1 if self.mistake == "unit_empty_parity" else ((hu >> 1) - 1) & 1
                     yield f"unit_empty{hb}", par
+                if j == 0:
+                    self.stage_v(h)
                 if hu >= 2 and emitted < hu - 2:
                     self.emit(hb, hu - 2)
                     emitted = hu - 2
-                if ustaged != hu:
-                    self.stage_unit(hb, hu)
-                    ustaged = hu
+                if j == 0:
+                    self.stage_z(hb, hu)
+                self.cp_wait(2 if self.mistake == "wait_keeps_two" else 1)
+                self.conv_v(h)
                 self.write_unit(hb, hu)
+                if j + 1 < G:  # the staging area is free: the next head's v rows
+                    self.stage_v(h + 1)
                 self.bars[f"unit_full{hb}"].arrive()
-                if j + 1 < G:  # the next head: its buffer's previous unit leaves, its rows start
+                if j + 1 < G:  # the next head's buffer: its previous unit leaves, its z rows start
                     nb = (hu + 1) & 1
                     if hu >= 1:
                         yield f"unit_empty{nb}", ((hu - 1) >> 1) & 1
                     if hu >= 1 and emitted < hu - 1:
                         self.emit(nb, hu - 1)
                         emitted = hu - 1
-                    self.stage_unit(nb, hu + 1)
-                    ustaged = hu + 1
+                    self.stage_z(nb, hu + 1)
                 hu += 1
+        if self.mistake != "drain_without_wait":
+            self.cp_wait(0)
         for u in range(emitted + 1, hu):  # the last units' outputs
             yield f"unit_empty{u & 1}", (u >> 1) & 1
             self.emit(u & 1, u)
+        self.cp_wait(0)
 
     def consumer(self):
         Hk, G, grid, ng = self.Hk, self.G, self.grid, self.ngroups
@@ -291,6 +334,7 @@ class CTA:
                     if nt is not None and self.mistake != "copy_before_read":  # after the chunk's barrier
                         self.tma_issue(q, nt)
                         issued += 1
+                for q in range(CHUNKS):  # the first GEMM once the whole tile is in (threads 0 and 32)
                     self.gemm1(q, hu, gb, li)
                 pend = None
                 yield "g1", g1_seen & 1
@@ -322,12 +366,15 @@ class CTA:
             self._step(agents, waits, name)
         for _ in range(1_000_000):
             ready = [("agent", n) for n in agents if self.bars[waits[n][0]].passes(waits[n][1])]
-            pending = [("fifo", t) for t in (0, 32) if self.fifo[t]] + [("tma", k) for k in range(len(self.tma))]
+            pending = ([("fifo", t) for t in (0, 32) if self.fifo[t]] + [("tma", k) for k in range(len(self.tma))] +
+                       [("cp", k) for k in range(len(self.cp_in_flight()))])
             if not ready and not pending:
                 if agents:
                     raise Deadlock({n: waits[n] for n in agents})
                 break
-            if policy == "agents_first" and ready:
+            if policy == "late_copies":  # copies land only when a wait needs them or nothing else runs
+                pool = ready + [e for e in pending if e[0] != "cp"] or pending
+            elif policy == "agents_first" and ready:
                 pool = ready
             elif policy == "async_first" and pending:
                 pool = pending
@@ -338,6 +385,8 @@ class CTA:
                 self._step(agents, waits, which)
             elif kind == "fifo":
                 self.complete(self.fifo[which].popleft())
+            elif kind == "cp":
+                self.land_copy(which)
             else:
                 self.land(which)
         else:
@@ -353,7 +402,7 @@ class CTA:
 
     def check_end(self):
         assert self.p_keys == self.c_keys, "producers and consumers ran different units"
-        assert not self.tma and not self.fifo[0] and not self.fifo[32], "work in flight when the CTA leaves"
+        assert not self.tma and not self.fifo[0] and not self.fifo[32] and not self.cp_in_flight(), "work in flight when the CTA leaves"
         assert self.issued == self.chunks, "state chunks copied that no unit took"
         for key in self.p_keys:
             assert self.emitted[key] == 1, key
@@ -391,7 +440,7 @@ SCENARIOS = [
     (7, 2, 1, 3, (1, 2, 6)),
     (2, 1, 3, 4, ()),             # more CTAs than groups
 ]
-POLICIES = ["random", "agents_first", "async_first"]
+POLICIES = ["random", "agents_first", "async_first", "late_copies"]
 
 
 @pytest.mark.parametrize("spec", [False, True], ids=["decode", "verify"])
@@ -404,7 +453,7 @@ def test_pipeline_protocol_under_random_schedules(scenario, spec):
 
 
 @pytest.mark.parametrize("mistake", ["no_unit_empty_wait", "unit_empty_parity", "copier_no_skip",
-                                     "copy_before_read", "no_mma_wait"])
+                                     "copy_before_read", "no_mma_wait", "wait_keeps_two", "drain_without_wait"])
 def test_planted_protocol_mistakes_are_caught(mistake):
     caught = 0
     for scenario in SCENARIOS:

@@ -119,10 +119,11 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all_but_newest() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // conv + SiLU of one channel from its staged inputs: rows[r * stride] for r < W-1 the
-// history, then the n <= 16 tokens; w: its W weights. out[t] for t < n, 0 beyond.
+// history, then the n <= 16 tokens; w: its W <= KW weights. out[t] for t < n, 0 beyond.
+// KW is the width the code is unrolled for (taps past W are zero).
+template <int KW>
 __device__ __forceinline__ void conv_staged(const uint16_t* rows, int stride, const uint16_t* w, int W, int n,
                                             float (&out)[kCT]) {
-    constexpr int KW = kMaxConvWidth;
     float xs[kCT + KW - 1];  // xs[KW - 1 + i] = input i (i < 0: history)
 #pragma unroll
     for (int i = -(KW - 1); i < kCT; ++i) {
@@ -141,6 +142,10 @@ __device__ __forceinline__ void conv_staged(const uint16_t* rows, int stride, co
     }
 }
 
+// KW: the conv width the producers' convs are unrolled for, 4 (conv widths up to 4) or
+// kMaxConvWidth: the shorter unrolling halves the conv's instructions and the kernel's code,
+// and the producers' conv phases are bound by issue, not by memory.
+template <int KW>
 __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeArgs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -328,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             {  // step 3 for channel i of q | k: conv + SiLU into the scratch
                 float qk[kCT];
                 const int lc = i, part = i / kDK;
-                conv_staged(graw + lc, 2 * kDK, gw + lc * W, W, n, qk);
+                conv_staged<KW>(graw + lc, 2 * kDK, gw + lc * W, W, n, qk);
 #pragma unroll
                 for (int t = 0; t < kCT; ++t) scr[t * kScrStride + lc] = qk[t];
                 if (!spec)  // the new history: the last W-1 raw inputs
@@ -466,13 +471,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 }
                 cp_async_commit();
             };
-            // the gate inputs of head hh's tokens (loaded one head ahead within the group)
+            // the gate inputs of head hh's tokens and its gate parameters (loaded one head ahead
+            // within the group, so that no load is outstanding at the barrier after the gates)
             uint16_t ga = 0, gbb = 0;
+            float gA = 0.f, gdt = 0.f;
             auto load_gates = [&](int hh) {
                 if (gi >= 0 && gi < kCT && gi < n) {
                     const size_t ai = ((size_t)tok0 + gi) * Hv + hh;
                     ga = p.a[ai];
                     gbb = p.b[ai];
+                    gA = __ldg(p.A_log + hh);
+                    gdt = __ldg(p.dt_bias + hh);
                 }
             };
             for (int j = 0; j < G; ++j, ++hu) {
@@ -513,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 named_barrier(kProducerBar, kProducers);
                 if (i < kDV) {  // v channel i of this head (step 3)
                     float vv[kCT];
-                    conv_staged(uraw + i, kDV, uw + i * W, W, n, vv);
+                    conv_staged<KW>(uraw + i, kDV, uw + i * W, W, n, vv);
 #pragma unroll
                     for (int t = 0; t < kCT; ++t) hv[t * kDV + i] = vv[t];
                     if (!spec)
@@ -521,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 } else if (gi < kCT) {  // steps 4, 5 per token (no decay and no write past the tokens)
                     float al = 1.f, be = 0.f;
                     if (gi < n) {
-                        gate_and_beta(ga, gbb, p.A_log[h], p.dt_bias[h], al, be);
+                        gate_and_beta(ga, gbb, gA, gdt, al, be);
                         if (spec) p.spec_alpha[((size_t)tok0 + gi) * Hv + h] = al;
                     }
                     ha[gi] = al;
@@ -869,12 +878,14 @@ cudaError_t chunk_grid_cap(int* cap) {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (sms_of[dev] == 0) {
-        if ((e = cudaFuncSetAttribute(decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)) !=
-            cudaSuccess)
+        if ((e = cudaFuncSetAttribute(decode_chunk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kSmemBytes)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(decode_chunk_kernel<kMaxConvWidth>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kSmemBytes)) != cudaSuccess)
             return e;
         int sms = 0, per_sm = 0;
         if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_chunk_kernel, kThreads, kSmemBytes)) !=
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_chunk_kernel<kMaxConvWidth>, kThreads, kSmemBytes)) !=
             cudaSuccess)
             return e;
         if (per_sm < 1) return cudaErrorInvalidConfiguration;
@@ -912,7 +923,8 @@ cudaError_t launch_decode_chunk(const DecodeArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_chunk_kernel, a);
+    return a.sh.W <= 4 ? cudaLaunchKernelEx(&cfg, decode_chunk_kernel<4>, a)
+                       : cudaLaunchKernelEx(&cfg, decode_chunk_kernel<kMaxConvWidth>, a);
 }
 
 }  // namespace gdn

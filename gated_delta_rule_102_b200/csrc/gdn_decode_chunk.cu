@@ -142,6 +142,29 @@ __device__ __forceinline__ void conv_staged(const uint16_t* rows, int stride, co
     }
 }
 
+// The same for the NT tokens t0 .. t0 + NT - 1 only (inputs t0 - (KW - 1) .. t0 + NT - 1).
+template <int KW, int NT>
+__device__ __forceinline__ void conv_staged_run(const uint16_t* rows, int stride, const uint16_t* w, int W, int n,
+                                                int t0, float (&out)[NT]) {
+    float xs[NT + KW - 1];  // xs[KW - 1 + j] = input t0 + j (negative: history)
+#pragma unroll
+    for (int j = -(KW - 1); j < NT; ++j) {
+        const int ii = t0 + j;
+        const bool in = ii < 0 ? -ii <= W - 1 : ii < n;
+        xs[KW - 1 + j] = in ? bf16_bits_to_float(rows[(W - 1 + ii) * stride]) : 0.f;
+    }
+    float wt[KW];
+#pragma unroll
+    for (int d = 0; d < KW; ++d) wt[d] = d < W ? bf16_bits_to_float(w[W - 1 - d]) : 0.f;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        float u = 0.f;
+#pragma unroll
+        for (int d = KW - 1; d >= 0; --d) u = fmaf(wt[d], xs[KW - 1 + t - d], u);
+        out[t] = t0 + t < n ? silu_fast(u) : 0.f;
+    }
+}
+
 // KW: the conv width the producers' convs are unrolled for, 4 (conv widths up to 4) or
 // kMaxConvWidth: the shorter unrolling halves the conv's instructions and the kernel's code,
 // and the producers' conv phases are bound by issue, not by memory.
@@ -447,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
             const float* KK = gram + gb * 2 * kCT * kCT;
             const float* QK = KK + kCT * kCT;
             bool stop = false;
-            const int gi = i - kDK;  // threads 128..143: the gates of token gi
+            const int gi = i - (kProducers - 32);  // the last producer warp's lanes 0..15: the gates of token gi
             // cp.async of head hh's v channel rows and weights into the staging area (free once every
             // producer has passed the group's Gram products, or the last head's v conv)
             uint16_t* uw = uraw + kRawRows * kDV;  // weights [128][W]
@@ -520,14 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                 // way: they are read only by the emit, after another wait of this kind or the drain's
                 cp_async_wait_all_but_newest();
                 named_barrier(kProducerBar, kProducers);
-                if (i < kDV) {  // v channel i of this head (step 3)
-                    float vv[kCT];
-                    conv_staged<KW>(uraw + i, kDV, uw + i * W, W, n, vv);
-#pragma unroll
-                    for (int t = 0; t < kCT; ++t) hv[t * kDV + i] = vv[t];
-                    if (!spec)
-                        for (int r = 0; r < W - 1; ++r) hist[(size_t)r * C + chv + i] = uraw[(n + r) * kDV + i];
-                } else if (gi < kCT) {  // steps 4, 5 per token (no decay and no write past the tokens)
+                if (gi >= 0 && gi < kCT) {  // steps 4, 5 per token (no decay and no write past the tokens)
                     float al = 1.f, be = 0.f;
                     if (gi < n) {
                         gate_and_beta(ga, gbb, gA, gdt, al, be);
@@ -535,6 +551,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                     }
                     ha[gi] = al;
                     hbeta[gi] = be;
+                }
+                {  // step 3 for v channel i % 128 of this head, tokens 8 (i / 128) .. 8 (i / 128) + 7
+                    constexpr int kHalf = kCT / 2;
+                    const int vc = i & (kDV - 1), t0 = (i / kDV) * kHalf;
+                    float vv[kHalf];
+                    conv_staged_run<KW, kHalf>(uraw + vc, kDV, uw + vc * W, W, n, t0, vv);
+#pragma unroll
+                    for (int t = 0; t < kHalf; ++t) hv[(t0 + t) * kDV + vc] = vv[t];
+                    if (!spec && t0 == 0)
+                        for (int r = 0; r < W - 1; ++r) hist[(size_t)r * C + chv + vc] = uraw[(n + r) * kDV + vc];
                 }
                 named_barrier(kProducerBar, kProducers);
                 if (j + 1 < G) {  // the staging area is free: the next head's v rows and gate inputs

@@ -232,8 +232,15 @@ def test_tmem_column_plan():
 def test_thread_maps_cover_each_element_once():
     ct, dk, dv, npr = K["kCT"], K["kDK"], K["kDV"], K["kProducers"]
     pw_count = npr // 32
-    # conv: producer i owns q|k channel i, and v channel i for i < dv; gates: i - dk < ct
-    assert npr == 2 * dk and dv <= npr and dk + ct <= npr
+    # q|k conv: producer i owns channel i (all tokens)
+    assert npr == 2 * dk
+    # v conv: producer i owns channel i % dv for the tokens 8 (i / dv) .. 8 (i / dv) + 7
+    half = ct // 2
+    cover = collections.Counter((i % dv, (i // dv) * half + t) for i in range(npr) for t in range(half))
+    assert cover == collections.Counter(itertools.product(range(dv), range(ct)))
+    # the gates of token gi on lanes 0..15 of the last producer warp (they prefetch its inputs too)
+    gates = [i - (npr - 32) for i in range(npr) if 0 <= i - (npr - 32) < ct]
+    assert gates == list(range(ct))
     # norms: warp pw takes tokens pw + 8 m
     assert sorted(pw + pw_count * m for pw in range(pw_count) for m in range(ct // pw_count)) == list(range(ct))
     # Gram products and solve coefficients: thread i one (t, s)

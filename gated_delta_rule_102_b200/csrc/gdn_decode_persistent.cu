@@ -103,6 +103,7 @@ struct WS {
     static constexpr int TOTAL = BARS + (4 * NSTAGE + QB + kRing) * 8;
     static_assert(CG >= 1 && RG >= 1 && RPL >= 4 && (RPL & (RPL - 1)) == 0 && RG * CG == 32, "consumer geometry");
     static_assert(TOTAL <= 232448, "shared memory");
+    static_assert(NSTAGE >= NTEAMS, "a team's previous unit of a stage is issued before its next one");
 };
 
 template <int DK, int DV>
@@ -469,7 +470,14 @@ decode_ws_kernel(const DecodeArgs p, const int ncl) {
         int parity_part = 0;
         for (int u = team;; u += L::NTEAMS) {
             const int s = u % NSTAGE, q = u % QB;
-            bool ok = wait(full + s, (u / NSTAGE) & 1);
+            // The teams take units in turn, so the stage's previous unit may be another team's
+            // and still incomplete (its tile landing); a parity wait on the full barrier two
+            // phases ahead would then pass at once. The previous unit's release comes first: it
+            // is at most one phase away (the loader has issued that unit, this team having
+            // passed a later one), and the loader waited on the same phase before issuing this
+            // unit's copies, so it costs nothing once the full barrier can complete.
+            bool ok = u < NSTAGE || wait(empty + s, ((u / NSTAGE) - 1) & 1);
+            ok = ok && wait(full + s, (u / NSTAGE) & 1);
             if (!ok) fail();
             if (L::TEAM_WARPS > 1) ok = named_barrier_and(1 + team, 32 * L::TEAM_WARPS, ok && !*abort_flag);
             else ok = __all_sync(0xffffffffu, ok && !*abort_flag);

@@ -28,12 +28,14 @@
 // cid + grid, ...; a group's G v-heads are its units):
 //  * warps 4-11, the producers: per group the conv + SiLU of its q and k channels, the
 //    L2 norms, the high/low operand tiles of [k | q] (K-major, 128-byte swizzle), k^T
-//    and the Gram products k.k, q.k; per unit the conv of its v channels, the gates and
-//    the unit's solve coefficients; raw rows arrive by cp.async into shared memory;
+//    and the Gram products k.k, q.k; per unit the conv of its v channels (two threads per
+//    channel), the gates and the unit's solve coefficients, and the gated RMSNorm and
+//    outputs of each solved unit; raw rows arrive by cp.async into shared memory, one
+//    group or head ahead;
 //  * warps 0-3, the consumers (thread c owns column c and TMEM lane c): state chunks
 //    into TMEM, the two GEMMs (issued by threads 0 and 32), the state copies (issued by
 //    thread 64: TMA bulk copies of 32 rows, 16 KiB, into a ring holding one tile), the
-//    solve, the gated RMSNorm and the stores.
+//    solve and the new state's stores.
 // Groups and units pass from producers to consumers through double buffers guarded by
 // mbarriers. Every wait is bounded by the SM cycle counter; on expiry the CTA sets the
 // timeout bit, all roles leave their loops, and what was issued completes before the

@@ -97,7 +97,7 @@ constexpr int OFF_BAR = OFF_HEAD + 2 * kHeadFloats * 4;
 // ring full [kRing], group full/empty [2] each, unit full/empty [2] each, the update's
 // MMAs, the first GEMM's MMAs (two issuing threads)
 constexpr int kNumBars = kRing + 8 + 2;
-constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;  // TMEM address, abort flag
+constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;  // TMEM address, abort flag, first-GEMM commits
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(OFF_X % 1024 == 0 && OFF_Z % 1024 == 0 && kXRegion % 1024 == 0, "swizzled operand alignment");
 static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
     uint64_t* g1_bar = mma_bar + 1;      // the first GEMM (threads 0 and 32)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    uint32_t* g1_commits = tmem_slot + 2;  // first-GEMM batches thread 0 has committed (for an abort)
 
     if (tid == 0) {
         for (int s = 0; s < kRing; ++s) mbar_init(ring_full + s, 1);
@@ -208,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         mbar_init(mma_bar, 1);
         mbar_init(g1_bar, 2);
         *abort_flag = 0;
+        *g1_commits = 0;
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -771,6 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
                         }
                     }
                     umma_commit(smem_addr(g1_bar));
+                    if (c == 0) ++*g1_commits;
                 }
                 pend = nullptr;
                 float vv[kCT];
@@ -883,8 +886,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(const DecodeA
         }
         if (!ok) {
             fail();
-            // an MMA batch that was issued and never waited for completes before TMEM is freed,
-            // and the state copies still in flight land before the CTA leaves
+            // an MMA batch of either GEMM that was issued and never waited for completes before
+            // TMEM is freed, and the state copies still in flight land before the CTA leaves
+            if (c == 0 && *g1_commits > g1_seen) mbar_wait_bounded(g1_bar, g1_seen & 1u);
             if (c == 0 && mma_issued > mma_seen) mbar_wait_bounded(mma_bar, mma_seen & 1u);
             if (c == kCopier)
                 for (int v = chunk; v < issued; ++v) mbar_wait_bounded(ring_full + v % kRing, (uint32_t)((v / kRing) & 1));

@@ -26,7 +26,14 @@ included; every read sees the data meant for it (ring chunks by the state tile t
 pool slot and v-head; staged rows by their group or head), no v rows landing in the scratch
 while a group phase uses it; every unit's outputs emitted once and its state stored once; no
 copy or MMA left in flight at the end; each group's and unit's rows staged once (the
-look-ahead always right). Each planted protocol mistake must be caught by some schedule."""
+look-ahead always right). Each planted protocol mistake must be caught by some schedule.
+
+The abort paths too: at a random moment one blocked wait gives up, as a wait bounded by the
+cycle counter would; every wait after it sees the abort flag, each role leaves by the
+kernel's own path (the producers after their copies have landed; the consumers after the MMA
+batches of either GEMM they issued and the state copies in flight have completed) and the
+model checks that nothing is still in flight when the CTA frees its TMEM and leaves.
+Dropping the consumers' wait for the first GEMM on that path must be caught."""
 import collections
 import random
 
@@ -76,6 +83,7 @@ class CTA:
         self.p_keys, self.c_keys = [], []
         self.emitted, self.stored = collections.Counter(), collections.Counter()
         self.group_stagings, self.unit_stagings = collections.Counter(), collections.Counter()
+        self.abort = False   # the CTA's abort flag (a wait gave up)
         self.graw = None
         self.uraw = None   # the head whose v rows are in the staging area
         self.cp = []       # committed cp.async groups in commit order: [kind, landing action, landed]
@@ -224,18 +232,25 @@ class CTA:
         self.ring[q].update(tile=tile, inflight=False, read=False)
         self.bars[f"ring_full{q}"].arrive()
 
-    # ---- the two roles, in the kernel's order
+    # ---- the two roles, in the kernel's order. A wait yields ("w", barrier, parity) and gets
+    # back whether it passed (False once the abort flag is set, or when it times out); a
+    # bounded wait of an abort path yields ("b", barrier, parity) and waits for the phase.
     def producer(self):
         Hk, G, grid, ng = self.Hk, self.G, self.grid, self.ngroups
         li = hu = 0
         emitted = gstaged = -1
+        stop = False
         for g in range(self.cta, ng, grid):
             gn = g + grid
             if not self.valid[g]:
                 continue
             gb, hk = li & 1, g % Hk
+            ok = True
             if li >= 2:
-                yield f"grp_empty{gb}", ((li >> 1) - 1) & 1
+                ok = yield ("w", f"grp_empty{gb}", ((li >> 1) - 1) & 1)
+            if not (ok and not self.abort):  # the producers agree, and leave together
+                self.abort |= not ok
+                break
             if gstaged != g:
                 self.stage_group(g)
                 gstaged = g
@@ -255,9 +270,14 @@ class CTA:
             for j in range(G):
                 hb, h = hu & 1, hk * G + j
                 self.p_keys.append((g, h))
+                ok = True
                 if hu >= 2 and self.mistake != "no_unit_empty_wait":
                     par = (hu >> 1) & 1 if self.mistake == "unit_empty_parity" else ((hu >> 1) - 1) & 1
-                    yield f"unit_empty{hb}", par
+                    ok = yield ("w", f"unit_empty{hb}", par)
+                if not (ok and not self.abort):
+                    self.abort |= not ok
+                    stop = True
+                    break
                 if j == 0:
                     self.stage_v(h)
                 if hu >= 2 and emitted < hu - 2:
@@ -273,24 +293,36 @@ class CTA:
                 self.bars[f"unit_full{hb}"].arrive()
                 if j + 1 < G:  # the next head's buffer: its previous unit leaves, its z rows start
                     nb = (hu + 1) & 1
+                    ok2 = True
                     if hu >= 1:
-                        yield f"unit_empty{nb}", ((hu - 1) >> 1) & 1
+                        ok2 = yield ("w", f"unit_empty{nb}", ((hu - 1) >> 1) & 1)
+                    if not (ok2 and not self.abort):
+                        self.abort |= not ok2
+                        stop = True
+                        break
                     if hu >= 1 and emitted < hu - 1:
                         self.emit(nb, hu - 1)
                         emitted = hu - 1
                     self.stage_z(nb, hu + 1)
                 hu += 1
+            if stop:
+                break
         if self.mistake != "drain_without_wait":
             self.cp_wait(0)
-        for u in range(emitted + 1, hu):  # the last units' outputs
-            yield f"unit_empty{u & 1}", (u >> 1) & 1
-            self.emit(u & 1, u)
-        self.cp_wait(0)
+        if not self.abort:
+            for u in range(emitted + 1, hu):  # the last units' outputs
+                got = yield ("w", f"unit_empty{u & 1}", (u >> 1) & 1)
+                if not (got and not self.abort):
+                    self.abort |= not got
+                    break
+                self.emit(u & 1, u)
+        self.cp_wait(0)  # no copy of this thread lands after the CTA has left
 
     def consumer(self):
         Hk, G, grid, ng = self.Hk, self.G, self.grid, self.ngroups
-        li = hu = chunk = issued = g1_seen = mma_seen = 0
+        li = hu = chunk = issued = g1_seen = mma_seen = mma_issued = g1_commits = 0
         pend = None
+        ok = True
 
         def next_group(frm):
             gg = frm
@@ -308,7 +340,10 @@ class CTA:
             if not self.valid[g]:
                 continue
             gb, hk = li & 1, g % Hk
-            yield f"grp_full{gb}", (li >> 1) & 1
+            got = yield ("w", f"grp_full{gb}", (li >> 1) & 1)
+            if not (got and not self.abort):
+                ok = False
+                break
             for j in range(G):
                 hb, h = hu & 1, hk * G + j
                 self.c_keys.append((g, h))
@@ -319,59 +354,100 @@ class CTA:
                     nt = self.tile(g2, 0) if g2 < ng else None
                 else:
                     nt = self.tile(g, j + 1)
-                yield f"unit_full{hb}", (hu >> 1) & 1
-                self.read_unit(hb, hu)
+                w = yield ("w", f"unit_full{hb}", (hu >> 1) & 1)
+                if w:
+                    self.read_unit(hb, hu)
                 for q in range(CHUNKS):
                     s = chunk % RING
-                    yield f"ring_full{s}", (chunk // RING) & 1
+                    if w:
+                        w = yield ("w", f"ring_full{s}", (chunk // RING) & 1)
                     if self.mistake == "copy_before_read" and nt is not None:
                         self.tma_issue(q, nt)
                         issued += 1
                     if pend is not None:
                         self.store_chunk(q, pend)
-                    self.take_chunk(s, q, self.tile(g, j), hu)
+                    if w:
+                        self.take_chunk(s, q, self.tile(g, j), hu)
+                    if not (w and not self.abort):  # the chunk's barrier
+                        ok = False
+                        break
                     chunk += 1
                     if nt is not None and self.mistake != "copy_before_read":  # after the chunk's barrier
                         self.tma_issue(q, nt)
                         issued += 1
+                if not ok:
+                    break
                 for q in range(CHUNKS):  # the first GEMM once the whole tile is in (threads 0 and 32)
                     self.gemm1(q, hu, gb, li)
+                g1_commits += 1
                 pend = None
-                yield "g1", g1_seen & 1
-                g1_seen += 1
-                self.read_d1(hu)
-                self.write_o(hb, hu)
+                w = yield ("w", "g1", g1_seen & 1)
+                if w:
+                    g1_seen += 1
+                    self.read_d1(hu)
+                    self.write_o(hb, hu)
+                    if not self.spec:
+                        self.write_y(hu)
+                if not (w and not self.abort):
+                    ok = False
+                    break
                 if not self.spec:
-                    self.write_y(hu)
                     self.gemm2(hu, gb, li)
+                    mma_issued += 1
                 self.bars[f"unit_empty{hb}"].arrive()
                 if not self.spec:
                     if self.mistake != "no_mma_wait":
-                        yield "mma", mma_seen & 1
-                        mma_seen += 1
+                        w = yield ("w", "mma", mma_seen & 1)
+                        if w:
+                            mma_seen += 1
                     pend = hu
+                if not (w and not self.abort):
+                    ok = False
+                    break
                 hu += 1
+            if not ok:
+                break
             self.bars[f"grp_empty{gb}"].arrive()
             li += 1
-        if pend is not None:
+        if ok and pend is not None:
             for q in range(CHUNKS):
                 self.store_chunk(q, pend)
+        if not ok:  # what was issued completes before TMEM is freed and the CTA leaves
+            self.abort = True
+            if g1_commits > g1_seen and self.mistake != "no_first_gemm_drain":
+                yield ("b", "g1", g1_seen & 1)
+            if mma_issued > mma_seen:
+                yield ("b", "mma", mma_seen & 1)
+            for v in range(chunk, issued):
+                yield ("b", f"ring_full{v % RING}", (v // RING) & 1)
         self.issued, self.chunks = issued, chunk
 
     # ---- the scheduler
-    def run(self, rng, policy):
+    def run(self, rng, policy, timeout_rate=0.0):
+        """timeout_rate: the chance per step that one blocked wait gives up (once per run)."""
         agents = {"P": self.producer(), "C": self.consumer()}
-        waits = {}
+        waits, resume = {}, {}
         for name in list(agents):
-            self._step(agents, waits, name)
+            self._step(agents, waits, resume, name)
+        timed_out = False
         for _ in range(1_000_000):
-            ready = [("agent", n) for n in agents if self.bars[waits[n][0]].passes(waits[n][1])]
+            def can_go(n):
+                kind, bar, par = waits[n]
+                return self.bars[bar].passes(par) or (kind == "w" and self.abort)
+            ready = [("agent", n) for n in agents if can_go(n)]
             pending = ([("fifo", t) for t in (0, 32) if self.fifo[t]] + [("tma", k) for k in range(len(self.tma))] +
                        [("cp", k) for k in range(len(self.cp_in_flight()))])
-            if not ready and not pending:
-                if agents:
-                    raise Deadlock({n: waits[n] for n in agents})
+            blocked = [n for n in agents if waits[n][0] == "w" and not can_go(n)]
+            if timeout_rate and not timed_out and blocked and rng.random() < timeout_rate:
+                n = rng.choice(blocked)  # this wait gives up: its agent sees False and sets the abort flag
+                timed_out = True
+                resume[n] = False
+                self._step(agents, waits, resume, n)
+                continue
+            if not agents:  # every role has left: the CTA frees its TMEM and leaves now
                 break
+            if not ready and not pending:
+                raise Deadlock({n: waits[n] for n in agents})
             if policy == "late_copies":  # copies land only when a wait needs them or nothing else runs
                 pool = ready + [e for e in pending if e[0] != "cp"] or pending
             elif policy == "agents_first" and ready:
@@ -382,7 +458,9 @@ class CTA:
                 pool = ready + pending
             kind, which = rng.choice(pool)
             if kind == "agent":
-                self._step(agents, waits, which)
+                bar_kind, bar, par = waits[which]
+                resume[which] = self.bars[bar].passes(par)
+                self._step(agents, waits, resume, which)
             elif kind == "fifo":
                 self.complete(self.fifo[which].popleft())
             elif kind == "cp":
@@ -393,16 +471,19 @@ class CTA:
             raise AssertionError("the model did not finish")
 
     @staticmethod
-    def _step(agents, waits, name):
+    def _step(agents, waits, resume, name):
         try:
-            waits[name] = next(agents[name])
+            waits[name] = agents[name].send(resume.pop(name, None))
         except StopIteration:
             del agents[name]
             waits.pop(name, None)
 
     def check_end(self):
+        assert not self.tma and not self.fifo[0] and not self.fifo[32] and not self.cp_in_flight(), \
+            "work in flight when the CTA frees its TMEM and leaves"
+        if self.abort:
+            return
         assert self.p_keys == self.c_keys, "producers and consumers ran different units"
-        assert not self.tma and not self.fifo[0] and not self.fifo[32] and not self.cp_in_flight(), "work in flight when the CTA leaves"
         assert self.issued == self.chunks, "state chunks copied that no unit took"
         for key in self.p_keys:
             assert self.emitted[key] == 1, key
@@ -410,6 +491,22 @@ class CTA:
         assert all(c == 1 for c in self.group_stagings.values())
         assert sorted(self.unit_stagings) == list(range(len(self.p_keys)))
         assert all(c == 1 for c in self.unit_stagings.values())
+
+
+def launch_with_timeout(B, Hk, G, grid, bad_seqs=(), spec=False, mistake=None, seed=0, policy="random",
+                        rate=0.05):
+    """All CTAs of one launch, one wait of each giving up at a random moment; returns how many
+    CTAs took their abort paths."""
+    ngroups = B * Hk
+    valid = [g // Hk not in bad_seqs for g in range(ngroups)]
+    slot = [(7 * (g // Hk) + 3) % 1000 for g in range(ngroups)]
+    aborted = 0
+    for cta in range(min(grid, ngroups)):
+        m = CTA(cta, grid, valid, slot, Hk, G, spec, mistake)
+        m.run(random.Random(1000 * seed + cta), policy, timeout_rate=rate)
+        m.check_end()
+        aborted += m.abort
+    return aborted
 
 
 def launch(B, Hk, G, grid, bad_seqs=(), spec=False, mistake=None, seed=0, policy="random"):
@@ -465,3 +562,27 @@ def test_planted_protocol_mistakes_are_caught(mistake):
                 except (AssertionError, Deadlock):
                     caught += 1
     assert caught > 0, mistake
+
+
+@pytest.mark.parametrize("spec", [False, True], ids=["decode", "verify"])
+def test_abort_paths_leave_nothing_in_flight(spec):
+    aborted = 0
+    for B, Hk, G, grid, bad in SCENARIOS:
+        for policy in POLICIES:
+            for seed in range(6):
+                for rate in (0.02, 0.2):
+                    aborted += launch_with_timeout(B, Hk, G, grid, bad, spec=spec, seed=seed, policy=policy, rate=rate)
+    assert aborted > 100  # the abort paths were taken, from many points
+
+
+def test_abort_without_the_first_gemm_drain_is_caught():
+    caught = 0
+    for B, Hk, G, grid, bad in SCENARIOS:
+        for policy in POLICIES:
+            for seed in range(6):
+                try:
+                    launch_with_timeout(B, Hk, G, grid, bad, mistake="no_first_gemm_drain", seed=seed, policy=policy,
+                                        rate=0.2)
+                except (AssertionError, Deadlock):
+                    caught += 1
+    assert caught > 0

@@ -17,6 +17,11 @@ from gated_delta_rule_102_b200 import synth
 # Tolerances (the derivation is in the design notes):
 OUT_ABS_TOL = 2e-3        # fp32 output vs oracle, O(1) outputs
 STATE_REL_TOL = 1e-4      # per (slot, head): max|dS| / max|S_ref|
+# Guards ten and five times inside those bars, where the fused fp32 kernels' errors sit ~100x
+# lower (1e-6 outputs, 1e-7..1e-6 states in short runs): a change that gives away an order of
+# magnitude of precision fails here long before it nears the bars.
+OUT_ABS_GUARD = 2e-4
+STATE_REL_GUARD = 2e-5
 
 
 def bf16_dev(a: np.ndarray, device="cuda") -> torch.Tensor:

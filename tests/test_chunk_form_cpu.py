@@ -134,3 +134,22 @@ def test_split_tf32_products_stay_inside_the_bars(s_std):
     oerr3 = np.abs(o3 - o_ref).max() / np.abs(o_ref).max()
     assert err3 < 2e-6 and oerr3 < 2e-6, (err3, oerr3)
     assert err1 > 10 * err3  # one truncated product is not enough
+
+
+def test_chunk_form_equals_the_recurrence_on_random_shapes():
+    # token counts 1..16 with every partial count, head sizes 8..64, decays from near 1 down to
+    # far below fp32's range, strengths 0..1, state scales 0..1
+    rng = np.random.default_rng(2024)
+    for case in range(40):
+        T = int(rng.integers(1, 17))
+        n = int(rng.integers(1, T + 1))
+        dk, dv = (int(x) for x in rng.choice([8, 16, 32, 64], 2))
+        decay = "wide" if case % 3 == 0 else "normal"
+        q, k, v, alpha, beta, S0 = problem(rng, T, dk, dv, decay, s_std=float(rng.choice([0.0, 0.02, 1.0])))
+        if case % 5 == 0:
+            beta[rng.integers(0, T)] = 0.0  # a token that writes nothing
+        o, S, _ = chunk_form(q, k, v, alpha, beta, S0, n)
+        o_ref, S_ref = oracle_tokens(q, k, v, alpha, beta, S0, n)
+        scale_o, scale_s = max(1.0, np.abs(o_ref).max()), max(1.0, np.abs(S_ref).max())
+        np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12 * scale_o, err_msg=f"case {case}: T={T} n={n}")
+        np.testing.assert_allclose(S, S_ref, rtol=0, atol=1e-12 * scale_s, err_msg=f"case {case}: T={T} n={n}")

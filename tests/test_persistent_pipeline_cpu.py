@@ -397,3 +397,43 @@ def test_planted_protocol_mistakes_are_caught(mistake, kw):
                 except (AssertionError, Deadlock):
                     caught += 1
     assert caught > 0, mistake
+
+
+def kernel_parameters():
+    """(dk, dv) -> (NSTAGE, QB, NTEAMS) as the kernel's WS<DK, DV> computes them (restated; keep in
+    step), and the namespace constants read from its source."""
+    import pathlib
+    import re
+    src = (pathlib.Path(__file__).resolve().parents[1] / "gated_delta_rule_102_b200" / "csrc" /
+           "gdn_decode_persistent.cu").read_text()
+    const = {name: int(re.search(rf"constexpr int {name} = (\d+);", src).group(1))
+             for name in ("kRing", "kFixedUnits", "kMaxConvWidthPersistent")}
+    rup = lambda x, m: (x + m - 1) // m * m  # noqa: E731
+    shapes = {}
+    for dk in (16, 32, 64, 128):
+        for dv in ((16,) if dk >= 32 else ()) + (32, 64, 128):
+            team_warps = 4 if dv >= 128 else (2 if dv >= 64 else 1)
+            maxnch = 2 * dk + dv
+            cstage = rup(const["kMaxConvWidthPersistent"] * maxnch * 2, 16) + \
+                rup(maxnch * const["kMaxConvWidthPersistent"] * 2, 16)
+            per_stage = dk * dv * 4 + cstage + dv * 6 + 32 + 2 * dk * 4 + 24 + 32
+            nstage = min(max((232448 - 3072 - 4 * dk * 4) // per_stage, 2), 8)
+            shapes[(dk, dv)] = (nstage, nstage + 2, 8 // team_warps)
+    return const, shapes
+
+
+def test_protocol_at_every_instantiated_shape():
+    const, shapes = kernel_parameters()
+    assert const["kFixedUnits"] >= 1
+    assert shapes[(128, 128)] == (3, 5, 2)  # the benchmark's shape: three stages, two teams
+    for (dk, dv), (nstage, qb, nteams) in shapes.items():
+        # the bounds the protocol rests on: at most NSTAGE + 1 relayed entries outstanding, and a
+        # team's previous unit of a stage issued before its next one
+        assert const["kRing"] >= nstage + 2, (dk, dv)
+        assert nstage >= nteams, (dk, dv)
+    for nstage, qb, nteams in sorted(set(shapes.values())):
+        for ngroups, ncl, G in ((9, 2, 2), (14, 3, 1), (6, 1, 4)):
+            for policy in POLICIES:
+                for seed in range(2):
+                    launch(ngroups, ncl, G, nstage, (ngroups // 2,), True, seed=seed, policy=policy,
+                           nteams=nteams, fixed=const["kFixedUnits"], ring=const["kRing"], qb=qb)
